@@ -1,0 +1,406 @@
+#!/usr/bin/env python
+"""Benchmark of KDA multi-token recurrent prefill on B200 (one JSON line on rank 0).
+
+A step is one full prefill (every kernel of the path) over one batch of
+synthetic inputs already resident in HBM.  Default workload: B8 T8192 H12
+(K = V = 128, BF16 q/k/v/beta, FP32 g in [-5, 0], no initial state), the
+shape the throughput target is stated on.  Inputs (1.2 GB) exceed the 126 MB
+L2, so no extra flush is needed between steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   # the FP64 CPU oracle on the host cores
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs the same per-GPU
+workload on its own seeded data (weak scaling, no collective on the data path);
+the step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "KDA prefill ms and Mtokens·heads/s at 1 B200; % tensor-core roofline"
+UNIT = "Mtokens·heads/s"
+# bytes every prefill must move per token and head: q, k, v (3 x 256) + g (512) + beta (2) + o (256)
+PATH_BYTES_PER_TOKHEAD = 1538
+STATE_BYTES = 128 * 128 * 4
+# per-kernel bytes per token and head, as designed (split variant)
+PREP_BYTES_PER_TOKHEAD = 768 + 512 + 2 + 1160     # reads q,k,v,g,beta; writes W,QG,U,Kd,Aqk,Gamma
+REC_BYTES_PER_TOKHEAD = 1160 + 256                 # reads the prepared tiles; writes o
+# tensor-core FLOPs per token and head at a fixed C = 64 count: 6 K V + 10 C d
+FLOPS_PER_TOKHEAD_C64 = 6 * 128 * 128 + 10 * 64 * 128
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_sha(files):
+    h = hashlib.sha256()
+    for f in files:
+        h.update(open(os.path.join(ROOT, "kda_chunked_recurrent_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel, units):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel is unchanged."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        d = json.load(open(p))[kernel]
+    except Exception:
+        return None
+    if d.get("source_sha") != kernel_source_sha(d.get("sources", [])):
+        return None
+    return float(d["dram_bytes_per_tokhead"]) * units
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.samples = []
+        self.proc = None
+        self.thread = None
+        self.t_on = self.t_off = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.gpu)], stdout=subprocess.PIPE,
+                stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), [x.strip() for x in line.split(",")]))
+
+    def mark_on(self):
+        self.t_on = time.time()
+
+    def mark_off(self):
+        self.t_off = time.time()
+
+    def stop(self):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        inside = [s for t, s in self.samples if self.t_on and self.t_off and
+                  self.t_on - 0.15 <= t <= self.t_off + 0.15]
+        use = inside if inside else [s for _, s in self.samples]
+        sm = [float(s[1]) for s in use if s[1].replace(".", "").isdigit()]
+        mx = [float(s[2]) for s in use if s[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for s in use for i in range(4)
+                          if len(s) > 5 + i and s[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(use), "in_window": bool(inside)}
+
+
+def dist_setup(n_gpus):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+_WL_CACHE = {}
+
+
+def cpu_baseline(inp_name, threads=0):
+    """The oracle as it stands on a bounded sample: sequence 0, every head, <= 8192 tokens."""
+    import oracle
+    from kda_chunked_recurrent_b200.inputs import workload
+    if inp_name not in _WL_CACHE:
+        _WL_CACHE[inp_name] = workload(inp_name)
+    inp = _WL_CACHE[inp_name]
+    L = min(inp.seqlens[0], 8192)
+    from kda_chunked_recurrent_b200.inputs import KDAInputs
+    import torch
+    sub = KDAInputs(q=inp.q[:L], k=inp.k[:L], v=inp.v[:L], g=inp.g[:L], beta=inp.beta[:L],
+                    scale=inp.scale, cu_seqlens=torch.tensor([0, L], dtype=torch.int32),
+                    h0=None if inp.h0 is None else inp.h0[:1])
+    oracle.build_oracle()
+    cores = threads if threads > 0 else (os.cpu_count() or 1)
+    t = time.perf_counter()
+    oracle.prefill(sub, threads=cores)
+    dt = time.perf_counter() - t
+    units = L * inp.num_heads
+    return {"value": units / dt / 1e6, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"sequence 0 of {inp_name}: {L} tokens x {inp.num_heads} heads "
+                      f"({units} token-heads), FP64 per-token recurrence, OpenMP over heads",
+            "seconds": dt}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    steps, warm = args.steps, args.warmup
+    for _ in range(warm):
+        cpu_baseline(args.workload)
+    vals, secs = [], []
+    for _ in range(steps):
+        r = cpu_baseline(args.workload)
+        vals.append(r["value"])
+        secs.append(r["seconds"])
+    value = statistics.median(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": steps, "warmup": warm,
+            "ms_per_step": 1e3 * statistics.median(secs), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "sample": r["sample"]},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": r["cores"], "kind": "oracle",
+                             "sample": r["sample"]},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="B8_T8192_H12")
+    ap.add_argument("--variant", type=int, default=0)
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        return run_reference(args, rank, world)
+
+    import torch
+    rank, world, local = dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    import kda_chunked_recurrent_b200 as K
+    from kda_chunked_recurrent_b200 import capi
+    from kda_chunked_recurrent_b200.inputs import WORKLOADS, make_inputs, ragged_lengths
+
+    w = WORKLOADS[args.workload]
+    lens = w["seqlens"] if w.get("seqlens") is not None else ragged_lengths(w["ragged"])
+    inp = make_inputs(lens, w["H"], w["seed"] + 7919 * rank, with_h0=w.get("h0", False),
+                      with_ckpt=w.get("ckpt", False), fixed_layout=w.get("fixed", False))
+    N, T, H = inp.num_seqs, inp.total_tokens, inp.num_heads
+    fixed = inp.fixed_layout
+    dev = torch.device("cuda", local)
+    q, k, v, g, beta = (x.to(dev) for x in (inp.q, inp.k, inp.v, inp.g, inp.beta))
+    cu = None if fixed else inp.cu_seqlens.to(dev)
+    h0 = None if inp.h0 is None else inp.h0.to(dev)
+    cko = None if inp.ckpt_offsets is None else inp.ckpt_offsets.to(dev)
+    out = torch.empty(T, H, 128, dtype=torch.bfloat16, device=dev)
+    ht = torch.empty(N, H, 128, 128, dtype=torch.float32, device=dev)
+    ck = None if cko is None else torch.empty(N, H, 128, 128, dtype=torch.float32, device=dev)
+    shape = capi.make_shape(N, T, H, max(lens))
+    opts = {"variant": args.variant}
+    ws = K.Workspace(capi.kda_prefill_workspace_size(shape, cko is not None, opts), dev)
+    stream = torch.cuda.current_stream(dev)
+    P = lambda t: None if t is None else t.data_ptr()
+
+    def step(events=None):
+        o = dict(opts)
+        if events is not None:
+            o["events"] = events
+        rc = capi.kda_prefill(P(q), P(k), P(v), P(g), P(beta), inp.scale, P(h0), P(cu), shape,
+                              P(out), P(ht), P(ck), P(cko), ws.ptr, ws.nbytes, o,
+                              stream.cuda_stream)
+        if rc != 0:
+            raise K.KDAError(rc)
+
+    launches_per_step = (0 if fixed else 1) + (1 if T > 0 else 0) + 1
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = ws.status()
+    if st != 0:
+        raise K.KDAError(st, "device status after warm-up")
+
+    # per-step events: start, after prepare, after recurrence
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+    ev_s = [mk() for _ in range(args.steps)]
+    ev_p = [mk() for _ in range(args.steps)]
+    ev_r = [mk() for _ in range(args.steps)]
+    for e in ev_p + ev_r:
+        e.record(stream)  # materialise the CUDA events before handing them to the library
+    torch.cuda.synchronize()
+    clk = ClockSampler(local if world > 1 else int(os.environ.get("CUDA_VISIBLE_DEVICES", "0").split(",")[0] or 0))
+    clk.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    clk.mark_on()
+    t_start, t_end = mk(), mk()
+    t_start.record(stream)
+    for i in range(args.steps):
+        ev_s[i].record(stream)
+        step([None, ev_p[i].cuda_event, ev_r[i].cuda_event])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    clk.mark_off()
+    barrier(world)
+    clk.stop()
+    ms_local = t_start.elapsed_time(t_end) / args.steps
+    ms = max_over_ranks(ms_local, world)
+    st = ws.status()
+    if st != 0:
+        raise K.KDAError(st, "device status after timed steps")
+    prep_ms = statistics.mean(ev_s[i].elapsed_time(ev_p[i]) for i in range(args.steps))
+    rec_ms = statistics.mean(ev_p[i].elapsed_time(ev_r[i]) for i in range(args.steps))
+
+    units = T * H
+    value = units * world / (ms / 1e3) / 1e6
+
+    # ---- roofline of the dominant kernel
+    peaks, peak_src = load_peaks()
+    state_io = N * H * STATE_BYTES * ((1 if h0 is not None else 0) + 1 + (1 if ck is not None else 0))
+    kernels = {
+        "kda_prepare_kernel": (prep_ms, PREP_BYTES_PER_TOKHEAD * units,
+                               ["kda_prepare.cu", "kda_common.cuh", "sm100_primitives.cuh"]),
+        "kda_recurrence_kernel": (rec_ms, REC_BYTES_PER_TOKHEAD * units + state_io,
+                                  ["kda_recurrence.cu", "kda_common.cuh", "sm100_primitives.cuh"]),
+    }
+    dom = max(kernels, key=lambda n: kernels[n][0])
+    dms, dbytes, _ = kernels[dom]
+    achieved = dbytes / (dms / 1e3) / 1e9
+    roof = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1),
+            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+            "traffic": ncu_traffic(dom, units), "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
+            if peak_src == "measured" else "fallback 6650 GB/s",
+            "kernel_ms": round(dms, 4),
+            "algorithmic_bytes": int(dbytes),
+            "per_kernel_ms": {n: round(kernels[n][0], 4) for n in kernels}}
+    path_bytes = PATH_BYTES_PER_TOKHEAD * units + state_io
+    flops = FLOPS_PER_TOKHEAD_C64 * units
+    s = ms / 1e3
+    path = {"bytes": int(path_bytes), "hbm_frac": round(path_bytes / s / 1e9 / peaks["hbm_gbs"], 4),
+            "tc_frac_c64_burst": round(flops / s / 1e12 / peaks["bf16_tflops"], 4),
+            "tc_frac_c64_sustained": round(flops / s / 1e12 / peaks["bf16_tflops_sustained"], 4),
+            "binding_frac": round(max(flops / (peaks["bf16_tflops_sustained"] * 1e12),
+                                      path_bytes / (peaks["hbm_gbs"] * 1e9)) / s, 4),
+            "executed_chunk": 64}
+
+    # ---- end to end through the C ABI with host buffers (pinned), copies inside the timing
+    e2e = None
+    if args.e2e_steps > 0:
+        hq, hk, hv, hg, hb = (x.pin_memory() for x in (inp.q, inp.k, inp.v, inp.g, inp.beta))
+        hh0 = None if inp.h0 is None else inp.h0.pin_memory()
+        ho = torch.empty(T, H, 128, dtype=torch.bfloat16).pin_memory()
+        hht = torch.empty(N, H, 128, 128, dtype=torch.float32).pin_memory()
+        h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hg, hb)) + \
+            (0 if hh0 is None else hh0.numel() * 4)
+        d2h = ho.numel() * 2 + hht.numel() * 4
+
+        def e2e_step():
+            for dst, src in ((q, hq), (k, hk), (v, hv), (g, hg), (beta, hb)):
+                dst.copy_(src, non_blocking=True)
+            if hh0 is not None:
+                h0.copy_(hh0, non_blocking=True)
+            step()
+            ho.copy_(out, non_blocking=True)
+            hht.copy_(ht, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        a, b = mk(), mk()
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = max_over_ranks(a.elapsed_time(b) / args.e2e_steps, world)
+        e2e = {"value": units * world / (e_ms / 1e3) / 1e6, "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": round(e_ms, 3)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(args.workload)
+        cpu.pop("seconds", None)
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": args.workload, "num_seqs": N, "seq_lens": "x".join(
+                    map(str, sorted(set(lens)))) if len(set(lens)) < 4 else "ragged",
+                    "total_tokens": T, "heads": H, "head_dim": 128, "h0": h0 is not None,
+                    "checkpoint": ck is not None, "variant": "split", "chunk": 64,
+                    "parallelism": f"dp{world}" if world > 1 else "single",
+                    "l2": "inputs (%.2f GB) larger than L2, no flush" % (
+                        (PATH_BYTES_PER_TOKHEAD - 256) * units / 1e9)},
+                "roofline": roof, "path_roofline": path,
+                "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
+                "clocks": clk.summary()}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

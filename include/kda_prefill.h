@@ -1,0 +1,191 @@
+/*
+ * kda_prefill.h — C ABI of the B200 (sm_100a) KDA multi-token recurrent prefill.
+ *
+ * Kimi Delta Attention (KDA) is a gated delta rule with one decay per key
+ * channel.  Per (sequence n, head h) a K x V = 128 x 128 FP32 state S is carried
+ * through the tokens of the sequence:
+ *
+ *     S   <- Diag(exp(g_t)) S
+ *     S   <- S + beta_t k_t (v_t - S^T k_t)^T      (S^T k_t taken after the decay)
+ *     o_t  = scale * S^T q_t                       (S after token t's update)
+ *
+ * Interface facts taken from the pages that describe this operation:
+ *   - K = V = 128, BF16 q/k/v/beta, FP32 recurrent state, gate bound in
+ *     [-5, 0]: lmdeploy PR #5050 "Motivation" (native path requirements);
+ *     FlashInfer PR #4262 "Dispatch contract".
+ *   - ragged batches packed with B = 1 plus cu_seqlens: FlashInfer PR #4262
+ *     "Dispatch contract"; FlashKDA item page "What Sets It Apart".
+ *   - initial state, final state updated in place when the two pointers are
+ *     the same allocation, partial overlap rejected: FlashInfer PR #4262
+ *     "Physical schedules and true in-place state update".
+ *   - checkpoint export of the state at a caller offset into caller-owned
+ *     contiguous buffers, the two checkpoint arguments paired, offset values
+ *     the caller's responsibility (no device-to-host read): lmdeploy PR #5050
+ *     "Motivation" and "Scope".
+ *   - caller-owned workspace, CUDA-graph-capturable calls once warm:
+ *     FlashInfer PR #4633 "Description"; FlashInfer PR #4262 "CUDA graph and
+ *     tensor-map safety".
+ *   - 16-byte base alignment for TMA operands: FlashInfer PR #4633 "Reviewer
+ *     Notes".
+ *
+ * General rules for every entry point below
+ *   - All tensor pointers are DEVICE pointers on the current CUDA device, owned
+ *     by the caller; the library never allocates, frees or keeps them.
+ *   - `stream` is a cudaStream_t (passed as void*; NULL = legacy default stream).
+ *     All device work is enqueued on it; no call synchronizes the host except
+ *     kda_prefill_status.
+ *   - Host-side validation happens before any launch and before any write to a
+ *     caller buffer; on an error code nothing has been enqueued.
+ *   - The library never reads cu_seqlens or ckpt_offsets on the host.  Their
+ *     values are the caller's responsibility; with KDA_FLAG_VALIDATE the
+ *     kernels check them and record KDA_ERR_BAD_CU_SEQLENS /
+ *     KDA_ERR_BAD_CKPT_OFFSET in the workspace status word (see
+ *     kda_prefill_status) instead of computing.
+ */
+#ifndef KDA_PREFILL_H_
+#define KDA_PREFILL_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define KDA_HEAD_DIM 128 /* K = V = 128, the only head size */
+
+typedef enum {
+  KDA_OK = 0,
+  KDA_ERR_NULL_ARG = 1,            /* a required pointer is NULL                    */
+  KDA_ERR_BAD_SHAPE = 2,           /* N < 1, H < 1, T < 0, max_seqlen out of range,
+                                      fixed layout with T not divisible by N        */
+  KDA_ERR_MISALIGNED = 3,          /* a pointer misses its required alignment        */
+  KDA_ERR_UNPAIRED_CKPT = 4,       /* exactly one of ckpt_state / ckpt_offsets given */
+  KDA_ERR_PARTIAL_ALIAS = 5,       /* h0 and ht overlap without being identical, or
+                                      ckpt_state overlaps h0 / ht                   */
+  KDA_ERR_OUT_ALIAS = 6,           /* an output overlaps an input or the workspace   */
+  KDA_ERR_WORKSPACE_TOO_SMALL = 7, /* workspace_bytes < kda_prefill_workspace_size   */
+  KDA_ERR_UNSUPPORTED_DEVICE = 8,  /* current device is not compute capability 10.0  */
+  KDA_ERR_LAUNCH_FAILED = 9,       /* the CUDA runtime refused a launch              */
+  KDA_ERR_BAD_OPTION = 10,         /* unknown variant / chunk / flag value           */
+  /* codes the kernels record in the workspace status word */
+  KDA_ERR_BAD_CU_SEQLENS = 16,     /* cu_seqlens[0] != 0, decreasing, or last != T,
+                                      or a length above max_seqlen (validate mode)   */
+  KDA_ERR_BAD_CKPT_OFFSET = 17,    /* an offset outside [0, len] (validate mode)     */
+  KDA_ERR_TIMEOUT = 18             /* a bounded on-chip wait gave up (the kernel
+                                      returned without finishing its work)          */
+} kda_status_t;
+
+/* Sizes known on the host.  No device memory is read to obtain them. */
+typedef struct {
+  int32_t num_seqs;     /* N >= 1: sequences (fixed layout: the batch B)              */
+  int32_t total_tokens; /* T_total >= 0: rows of q/k/v/g/beta/out                     */
+  int32_t num_heads;    /* H >= 1                                                      */
+  int32_t max_seqlen;   /* an upper bound on every sequence length; 0 = use T_total    */
+} kda_shape_t;
+
+typedef enum {
+  KDA_VARIANT_AUTO = 0,  /* per-shape choice from the measured table                   */
+  KDA_VARIANT_SPLIT = 1, /* prepare kernel over all chunks, then the recurrence kernel */
+  KDA_VARIANT_FUSED = 2  /* one kernel, one CTA per (sequence, head)                    */
+} kda_variant_t;
+
+enum {
+  KDA_FLAG_VALIDATE = 1u << 0,       /* kernels check cu_seqlens / ckpt_offsets values  */
+  KDA_FLAG_TEST_FORCE_TIMEOUT = 1u << 1 /* test hook: every bounded wait gives up at once;
+                                          exercises the error path, never for production */
+};
+
+typedef struct {
+  int32_t variant;  /* kda_variant_t                                               */
+  uint32_t flags;   /* KDA_FLAG_*                                                   */
+  /* Optional profiling hook: cudaEvent_t handles (created by the caller) that
+     kda_prefill records on `stream` right after its launches: [0] after the
+     metadata kernel (when one is launched), [1] after the prepare kernel, [2]
+     after the last kernel of the call.  NULL entries are skipped.  The events
+     let a caller time each kernel on the launching stream. */
+  void* events[3];
+  int32_t reserved[4];
+} kda_options_t;
+
+/*
+ * Bytes of workspace kda_prefill needs for this shape and option set (NULL
+ * options = defaults).  `has_ckpt` != 0 when checkpoint export is requested.
+ * Returns 0 for an invalid shape.  The workspace must be 256-byte aligned and,
+ * before its first use, initialised once with kda_workspace_init.
+ */
+size_t kda_prefill_workspace_size(const kda_shape_t* shape, int has_ckpt,
+                                  const kda_options_t* options);
+
+/*
+ * Initialise a workspace (clears its status word).  Enqueued on `stream`.
+ * Needed once per workspace allocation, before the first kda_prefill with it.
+ */
+kda_status_t kda_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Multi-token recurrent prefill (one launch sequence on `stream`).
+ *
+ *   q, k      [T_total, H, 128] BF16, contiguous, 16-byte aligned.  Rows of all
+ *             sequences packed back to back (fixed layout [B, T, H, 128] is the
+ *             same memory).  k is expected to be L2-normalised per row: the
+ *             FP16 tensor-core operands assume |S| and |v| well inside 65504.
+ *   v         [T_total, H, 128] BF16, contiguous, 16-byte aligned.
+ *   g         [T_total, H, 128] FP32 log-decay per key channel, contiguous,
+ *             16-byte aligned; expected in [-5, 0] (outside it the chunked
+ *             factorisation may overflow FP32; values are not checked).
+ *   beta      [T_total, H] BF16, contiguous, 2-byte aligned (read with plain loads).
+ *   scale     output scale (e.g. 1/sqrt(128)).
+ *   h0        [N, H, 128, 128] FP32 initial state S[k][v] (row index = key
+ *             channel), contiguous, 16-byte aligned; NULL = zero state.
+ *   cu_seqlens [N+1] INT32 device array of sequence starts, or NULL for the
+ *             fixed layout (N sequences of T_total / N tokens each).
+ *   shape     host struct, see kda_shape_t.
+ *   out       [T_total, H, 128] BF16 output o (round-to-nearest-even from FP32).
+ *   ht        [N, H, 128, 128] FP32 final state, or NULL.  May be exactly h0
+ *             (same pointer): the state is then updated in place.
+ *   ckpt_state [N, H, 128, 128] FP32 checkpoint states, or NULL.
+ *   ckpt_offsets [N] INT32 device array, or NULL; must be given together with
+ *             ckpt_state.  Offset p_n is a prefix length of sequence n,
+ *             0 <= p_n <= len_n: p = 0 exports h0, p = len the final state.
+ *   workspace, workspace_bytes  caller-owned scratch (see above).
+ *   options   NULL = defaults (auto variant, no flags).
+ *   stream    cudaStream_t.
+ *
+ * Returns KDA_OK when the work was enqueued; errors see kda_status_t.  A zero-
+ * length sequence leaves ht = h0 (also when h0 and ht alias).
+ */
+kda_status_t kda_prefill(const void* q, const void* k, const void* v, const float* g,
+                         const void* beta, float scale, const float* h0,
+                         const int32_t* cu_seqlens, const kda_shape_t* shape, void* out,
+                         float* ht, float* ckpt_state, const int32_t* ckpt_offsets,
+                         void* workspace, size_t workspace_bytes,
+                         const kda_options_t* options, void* stream);
+
+/*
+ * Read (and clear when `clear` != 0) the status word the kernels of earlier
+ * kda_prefill calls recorded in `workspace`.  Synchronises `stream`.  The word
+ * keeps the first device-side error since the last clear (KDA_OK if none).
+ */
+kda_status_t kda_prefill_status(void* workspace, void* stream, int32_t* device_status,
+                                 int clear);
+
+/* Static description of a status code (never NULL). */
+const char* kda_status_string(int status);
+
+/*
+ * Write a one-line description of what kda_prefill would launch for this
+ * shape (variant, chunk size, grids, workspace bytes) into buf (NUL-
+ * terminated, truncated to n bytes).  Host only.
+ */
+kda_status_t kda_prefill_describe(const kda_shape_t* shape, int has_ckpt,
+                                  const kda_options_t* options, char* buf, size_t n);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int kda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_PREFILL_H_ */

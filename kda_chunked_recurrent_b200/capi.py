@@ -1,0 +1,129 @@
+"""ctypes binding of libkda_prefill.so (the C ABI of include/kda_prefill.h).
+
+Argument marshalling only: every step of the prefill runs in the library's
+CUDA kernels.  The names match the C entry points.  There is no CPU fallback:
+importing this module fails loudly when the library has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libkda_prefill.so")
+
+# status codes (kda_status_t)
+KDA_OK = 0
+KDA_ERR_NULL_ARG = 1
+KDA_ERR_BAD_SHAPE = 2
+KDA_ERR_MISALIGNED = 3
+KDA_ERR_UNPAIRED_CKPT = 4
+KDA_ERR_PARTIAL_ALIAS = 5
+KDA_ERR_OUT_ALIAS = 6
+KDA_ERR_WORKSPACE_TOO_SMALL = 7
+KDA_ERR_UNSUPPORTED_DEVICE = 8
+KDA_ERR_LAUNCH_FAILED = 9
+KDA_ERR_BAD_OPTION = 10
+KDA_ERR_BAD_CU_SEQLENS = 16
+KDA_ERR_BAD_CKPT_OFFSET = 17
+KDA_ERR_TIMEOUT = 18
+
+KDA_VARIANT_AUTO = 0
+KDA_VARIANT_SPLIT = 1
+KDA_VARIANT_FUSED = 2
+KDA_FLAG_VALIDATE = 1
+KDA_FLAG_TEST_FORCE_TIMEOUT = 2
+
+
+class kda_shape_t(ctypes.Structure):
+    _fields_ = [("num_seqs", ctypes.c_int32), ("total_tokens", ctypes.c_int32),
+                ("num_heads", ctypes.c_int32), ("max_seqlen", ctypes.c_int32)]
+
+
+class kda_options_t(ctypes.Structure):
+    _fields_ = [("variant", ctypes.c_int32), ("flags", ctypes.c_uint32),
+                ("events", ctypes.c_void_p * 3), ("reserved", ctypes.c_int32 * 4)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m kda_chunked_recurrent_b200.build`"
+            " (there is no fallback implementation)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P = ctypes.c_void_p
+    lib.kda_version.restype = ctypes.c_int
+    lib.kda_status_string.restype = ctypes.c_char_p
+    lib.kda_status_string.argtypes = [ctypes.c_int]
+    lib.kda_prefill_workspace_size.restype = ctypes.c_size_t
+    lib.kda_prefill_workspace_size.argtypes = [ctypes.POINTER(kda_shape_t), ctypes.c_int,
+                                               ctypes.POINTER(kda_options_t)]
+    lib.kda_workspace_init.restype = ctypes.c_int
+    lib.kda_workspace_init.argtypes = [P, ctypes.c_size_t, P]
+    lib.kda_prefill.restype = ctypes.c_int
+    lib.kda_prefill.argtypes = [P, P, P, P, P, ctypes.c_float, P, P, ctypes.POINTER(kda_shape_t),
+                                P, P, P, P, P, ctypes.c_size_t, ctypes.POINTER(kda_options_t), P]
+    lib.kda_prefill_status.restype = ctypes.c_int
+    lib.kda_prefill_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32), ctypes.c_int]
+    lib.kda_prefill_describe.restype = ctypes.c_int
+    lib.kda_prefill_describe.argtypes = [ctypes.POINTER(kda_shape_t), ctypes.c_int,
+                                         ctypes.POINTER(kda_options_t), ctypes.c_char_p,
+                                         ctypes.c_size_t]
+    return lib
+
+
+lib = _load()
+
+
+def _opt(options):
+    if options is None:
+        return None
+    if isinstance(options, kda_options_t):
+        return ctypes.byref(options)
+    o = kda_options_t()
+    o.variant = int(options.get("variant", 0))
+    o.flags = int(options.get("flags", 0))
+    for i, ev in enumerate(options.get("events") or ()):
+        o.events[i] = ev
+    return ctypes.byref(o)
+
+
+def make_shape(num_seqs, total_tokens, num_heads, max_seqlen=0) -> kda_shape_t:
+    return kda_shape_t(int(num_seqs), int(total_tokens), int(num_heads), int(max_seqlen))
+
+
+def kda_version() -> int:
+    return int(lib.kda_version())
+
+
+def kda_status_string(code: int) -> str:
+    return lib.kda_status_string(int(code)).decode()
+
+
+def kda_prefill_workspace_size(shape: kda_shape_t, has_ckpt: bool, options=None) -> int:
+    return int(lib.kda_prefill_workspace_size(ctypes.byref(shape), int(bool(has_ckpt)),
+                                              _opt(options)))
+
+
+def kda_workspace_init(workspace: int, workspace_bytes: int, stream: int) -> int:
+    return int(lib.kda_workspace_init(workspace, workspace_bytes, stream))
+
+
+def kda_prefill(q, k, v, g, beta, scale, h0, cu_seqlens, shape, out, ht, ckpt_state,
+                ckpt_offsets, workspace, workspace_bytes, options, stream) -> int:
+    """All pointer arguments are integers (device addresses) or None."""
+    return int(lib.kda_prefill(q, k, v, g, beta, ctypes.c_float(scale), h0, cu_seqlens,
+                               ctypes.byref(shape), out, ht, ckpt_state, ckpt_offsets, workspace,
+                               int(workspace_bytes), _opt(options), stream))
+
+
+def kda_prefill_status(workspace: int, stream: int, clear: bool = False):
+    val = ctypes.c_int32(0)
+    rc = int(lib.kda_prefill_status(workspace, stream, ctypes.byref(val), int(bool(clear))))
+    return rc, int(val.value)
+
+
+def kda_prefill_describe(shape: kda_shape_t, has_ckpt: bool, options=None) -> str:
+    buf = ctypes.create_string_buffer(512)
+    lib.kda_prefill_describe(ctypes.byref(shape), int(bool(has_ckpt)), _opt(options), buf, 512)
+    return buf.value.decode()

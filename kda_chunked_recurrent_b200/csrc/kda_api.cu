@@ -1,0 +1,343 @@
+// kda_api.cu — host side of the C ABI declared in include/kda_prefill.h.
+//
+// Validation (pointers, sizes, alignment, aliasing, workspace) happens before
+// any launch or write, as the pages require of the native prefill path
+// ("validate paired checkpoint arguments ... before cache mutation", lmdeploy
+// PR #5050 "Motivation"; partial h0/ht overlap rejected, FlashInfer PR #4262
+// "Physical schedules and true in-place state update").  Device metadata
+// (cu_seqlens, ckpt_offsets) is never read on the host.  Launch order on the
+// caller's stream: [schedule] -> prepare -> recurrence.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/kda_prefill.h"
+#include "kda_common.cuh"
+
+namespace kda {
+__global__ void kda_schedule_kernel(const KdaParams p);
+__global__ void kda_prepare_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps);
+__global__ void kda_recurrence_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps);
+namespace prep { extern const uint32_t kSmemAllocBytes; }
+namespace rec { extern const uint32_t kSmemAllocBytes; }
+}  // namespace kda
+
+using namespace kda;
+
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+constexpr long long kDefaultWaitBudget = 2000000000LL;  // clock cycles (~1 s)
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+struct Range {
+  uintptr_t lo, hi;  // [lo, hi)
+  bool valid() const { return lo != 0 && hi > lo; }
+};
+Range rng(const void* p, size_t bytes) {
+  return Range{reinterpret_cast<uintptr_t>(p), reinterpret_cast<uintptr_t>(p) + bytes};
+}
+bool overlap(const Range& a, const Range& b) {
+  return a.valid() && b.valid() && a.lo < b.hi && b.lo < a.hi;
+}
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+struct Resolved {
+  int variant;
+  bool fixed;
+  WorkspaceLayout lay;
+};
+
+kda_status_t check_options(const kda_options_t* o) {
+  if (!o) return KDA_OK;
+  if (o->variant < KDA_VARIANT_AUTO || o->variant > KDA_VARIANT_FUSED) return KDA_ERR_BAD_OPTION;
+  if (o->flags & ~(static_cast<uint32_t>(KDA_FLAG_VALIDATE | KDA_FLAG_TEST_FORCE_TIMEOUT)))
+    return KDA_ERR_BAD_OPTION;
+  if (o->variant == KDA_VARIANT_FUSED) return KDA_ERR_BAD_OPTION;  // not available yet
+  return KDA_OK;
+}
+
+kda_status_t check_shape(const kda_shape_t* s, bool fixed) {
+  if (!s) return KDA_ERR_NULL_ARG;
+  if (s->num_seqs < 1 || s->num_heads < 1 || s->total_tokens < 0 || s->max_seqlen < 0)
+    return KDA_ERR_BAD_SHAPE;
+  if (fixed && (s->total_tokens % s->num_seqs) != 0) return KDA_ERR_BAD_SHAPE;
+  // 32-bit TMA coordinates of the per-record tiles: slots * H * 128 < 2^31
+  const int64_t slots = chunk_slots(s->num_seqs, s->total_tokens, fixed);
+  if (slots * static_cast<int64_t>(s->num_heads) * 128 >= (int64_t(1) << 31)) return KDA_ERR_BAD_SHAPE;
+  if (static_cast<int64_t>(s->num_seqs) * s->num_heads * 128 >= (int64_t(1) << 31))
+    return KDA_ERR_BAD_SHAPE;
+  return KDA_OK;
+}
+
+Resolved resolve(const kda_shape_t* s, bool fixed, bool ckpt, const kda_options_t* o) {
+  Resolved r{};
+  r.variant = KDA_VARIANT_SPLIT;
+  (void)o;
+  r.fixed = fixed;
+  r.lay = make_layout(s->num_seqs, s->total_tokens, s->num_heads, fixed, true, ckpt);
+  return r;
+}
+
+kda_status_t device_check() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return KDA_ERR_UNSUPPORTED_DEVICE;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return KDA_ERR_UNSUPPORTED_DEVICE;
+  if (major != 10 || minor != 0) return KDA_ERR_UNSUPPORTED_DEVICE;
+  return KDA_OK;
+}
+
+bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, void* base, uint64_t inner,
+                 uint64_t rows, uint32_t box_inner, uint32_t box_rows, uint32_t elem_bytes) {
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {inner * elem_bytes};
+  const cuuint32_t box[2] = {box_inner, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return encode_fn()(m, dt, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_map_tokens(CUtensorMap* m, const void* base, uint64_t T, uint64_t H) {
+  const cuuint64_t dims[3] = {128, H, T};
+  const cuuint64_t strides[2] = {128 * 2, H * 128 * 2};
+  const cuuint32_t box[3] = {64, 1, 64};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+extern "C" {
+
+int kda_version(void) { return kVersion; }
+
+const char* kda_status_string(int s) {
+  switch (s) {
+    case KDA_OK: return "ok";
+    case KDA_ERR_NULL_ARG: return "a required pointer is NULL";
+    case KDA_ERR_BAD_SHAPE: return "invalid shape";
+    case KDA_ERR_MISALIGNED: return "a pointer misses its required alignment";
+    case KDA_ERR_UNPAIRED_CKPT: return "ckpt_state and ckpt_offsets must be given together";
+    case KDA_ERR_PARTIAL_ALIAS: return "h0/ht/ckpt_state overlap without being identical";
+    case KDA_ERR_OUT_ALIAS: return "an output overlaps an input or the workspace";
+    case KDA_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case KDA_ERR_UNSUPPORTED_DEVICE: return "current device is not compute capability 10.0";
+    case KDA_ERR_LAUNCH_FAILED: return "kernel launch failed";
+    case KDA_ERR_BAD_OPTION: return "unknown or unavailable option";
+    case KDA_ERR_BAD_CU_SEQLENS: return "cu_seqlens invalid (validate mode)";
+    case KDA_ERR_BAD_CKPT_OFFSET: return "checkpoint offset outside its sequence (validate mode)";
+    case KDA_ERR_TIMEOUT: return "a bounded on-device wait timed out";
+    default: return "unknown status";
+  }
+}
+
+size_t kda_prefill_workspace_size(const kda_shape_t* shape, int has_ckpt,
+                                  const kda_options_t* options) {
+  if (check_options(options) != KDA_OK) return 0;
+  // the layout does not depend on whether cu_seqlens is given beyond the slot
+  // bound; size for the larger (packed) bound so one workspace serves both.
+  if (check_shape(shape, false) != KDA_OK) return 0;
+  const Resolved r = resolve(shape, false, has_ckpt != 0, options);
+  return r.lay.total;
+}
+
+kda_status_t kda_workspace_init(void* workspace, size_t workspace_bytes, void* stream) {
+  if (!workspace) return KDA_ERR_NULL_ARG;
+  if (!aligned(workspace, 256)) return KDA_ERR_MISALIGNED;
+  if (workspace_bytes < kHeaderBytes) return KDA_ERR_WORKSPACE_TOO_SMALL;
+  if (cudaMemsetAsync(workspace, 0, kHeaderBytes, static_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return KDA_ERR_LAUNCH_FAILED;
+  return KDA_OK;
+}
+
+kda_status_t kda_prefill_describe(const kda_shape_t* shape, int has_ckpt,
+                                  const kda_options_t* options, char* buf, size_t n) {
+  if (!buf || n == 0) return KDA_ERR_NULL_ARG;
+  kda_status_t st = check_options(options);
+  if (st == KDA_OK) st = check_shape(shape, false);
+  if (st != KDA_OK) {
+    snprintf(buf, n, "error: %s", kda_status_string(st));
+    return st;
+  }
+  const Resolved r = resolve(shape, false, has_ckpt != 0, options);
+  snprintf(buf, n,
+           "variant=split chunk=%d prepare_grid=(%lld,%d)x128 recurrence_grid=%lldx160 "
+           "workspace_bytes=%zu",
+           kC, static_cast<long long>(r.lay.slots), shape->num_heads,
+           static_cast<long long>(shape->num_seqs) * shape->num_heads, r.lay.total);
+  return KDA_OK;
+}
+
+kda_status_t kda_prefill(const void* q, const void* k, const void* v, const float* g,
+                         const void* beta, float scale, const float* h0,
+                         const int32_t* cu_seqlens, const kda_shape_t* shape, void* out,
+                         float* ht, float* ckpt_state, const int32_t* ckpt_offsets,
+                         void* workspace, size_t workspace_bytes,
+                         const kda_options_t* options, void* stream) {
+  // ---------------- host-side validation (no CUDA call before it passes)
+  kda_status_t st = check_options(options);
+  if (st != KDA_OK) return st;
+  const bool fixed = (cu_seqlens == nullptr);
+  if (!shape) return KDA_ERR_NULL_ARG;
+  st = check_shape(shape, fixed);
+  if (st != KDA_OK) return st;
+  const int64_t N = shape->num_seqs, T = shape->total_tokens, H = shape->num_heads;
+  if (T > 0 && (!q || !k || !v || !g || !beta || !out)) return KDA_ERR_NULL_ARG;
+  if (!workspace) return KDA_ERR_NULL_ARG;
+  if ((ckpt_state == nullptr) != (ckpt_offsets == nullptr)) return KDA_ERR_UNPAIRED_CKPT;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(g, 16) ||
+      !aligned(out, 16) || !aligned(beta, 2) || !aligned(h0, 16) || !aligned(ht, 16) ||
+      !aligned(ckpt_state, 16) || !aligned(cu_seqlens, 4) || !aligned(ckpt_offsets, 4) ||
+      !aligned(workspace, 256))
+    return KDA_ERR_MISALIGNED;
+  const size_t tok16 = static_cast<size_t>(T * H * 128 * 2);
+  const size_t state = static_cast<size_t>(N * H * 128 * 128 * 4);
+  const Range rq = rng(q, tok16), rk = rng(k, tok16), rv = rng(v, tok16),
+              rg = rng(g, tok16 * 2), rb = rng(beta, static_cast<size_t>(T * H * 2)),
+              rh0 = rng(h0, state), rht = rng(ht, state), rck = rng(ckpt_state, state),
+              rcu = rng(cu_seqlens, static_cast<size_t>((N + 1) * 4)),
+              rco = rng(ckpt_offsets, static_cast<size_t>(N * 4)),
+              rws = rng(workspace, workspace_bytes), ro = rng(out, tok16);
+  if (overlap(rh0, rht) && h0 != ht) return KDA_ERR_PARTIAL_ALIAS;
+  if (overlap(rck, rh0) || overlap(rck, rht)) return KDA_ERR_PARTIAL_ALIAS;
+  const Range inputs[] = {rq, rk, rv, rg, rb, rcu, rco};
+  for (const Range& in : inputs) {
+    if (overlap(ro, in) || overlap(rht, in) || overlap(rck, in) || overlap(rws, in))
+      return KDA_ERR_OUT_ALIAS;
+  }
+  if (overlap(ro, rh0) || overlap(ro, rht) || overlap(ro, rck) || overlap(ro, rws) ||
+      overlap(rws, rh0) || overlap(rws, rht) || overlap(rws, rck))
+    return KDA_ERR_OUT_ALIAS;
+  const bool ckpt = ckpt_state != nullptr;
+  const Resolved r = resolve(shape, fixed, ckpt, options);
+  const size_t need = kda_prefill_workspace_size(shape, ckpt ? 1 : 0, options);
+  if (workspace_bytes < need || workspace_bytes < r.lay.total) return KDA_ERR_WORKSPACE_TOO_SMALL;
+
+  // ---------------- device
+  st = device_check();
+  if (st != KDA_OK) return st;
+  if (encode_fn() == nullptr) return KDA_ERR_LAUNCH_FAILED;
+  const uint32_t flags = options ? options->flags : 0u;
+
+  KdaParams p{};
+  p.q = static_cast<const uint16_t*>(q);
+  p.k = static_cast<const uint16_t*>(k);
+  p.v = static_cast<const uint16_t*>(v);
+  p.g = g;
+  p.beta = static_cast<const uint16_t*>(beta);
+  p.scale = scale;
+  p.h0 = h0;
+  p.cu_seqlens = cu_seqlens;
+  p.ckpt_offsets = ckpt_offsets;
+  p.out = static_cast<uint16_t*>(out);
+  p.ht = ht;
+  p.ckpt = ckpt_state;
+  p.N = static_cast<int32_t>(N);
+  p.T = static_cast<int32_t>(T);
+  p.H = static_cast<int32_t>(H);
+  p.max_len = shape->max_seqlen;
+  p.fixed_len = fixed ? static_cast<int32_t>(T / N) : 0;
+  p.ws = static_cast<uint8_t*>(workspace);
+  p.lay = r.lay;
+  p.slots = r.lay.slots;
+  p.flags = flags;
+  p.wait_budget = (flags & KDA_FLAG_TEST_FORCE_TIMEOUT) ? -1 : kDefaultWaitBudget;
+
+  // ---------------- tensor maps (encoded per call; passed by value)
+  SplitMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  const uint64_t recs = static_cast<uint64_t>(r.lay.slots) * H;
+  uint8_t* ws = p.ws;
+  bool mok = true;
+  if (T > 0) {
+    mok &= make_map_tokens(&maps.v_in, v, T, H);
+    mok &= make_map_2d(&maps.wt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ws + r.lay.wt, 64, recs * 128, 64, 128, 2);
+    mok &= make_map_2d(&maps.qgt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ws + r.lay.qgt, 64, recs * 128, 64, 128, 2);
+    mok &= make_map_2d(&maps.ut, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws + r.lay.ut, 64, recs * 128, 64, 128, 2);
+    mok &= make_map_2d(&maps.kdt, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws + r.lay.kdt, 64, recs * 128, 64, 128, 2);
+    mok &= make_map_2d(&maps.aqk, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws + r.lay.aqk, 64, recs * 64, 64, 64, 2);
+    if (ckpt)
+      mok &= make_map_2d(&maps.kpt, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws + r.lay.kpt, 64,
+                         static_cast<uint64_t>(N * H * 128), 64, 128, 2);
+  }
+  if (!mok) return KDA_ERR_LAUNCH_FAILED;
+
+  // ---------------- launches
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] {
+    cudaError_t e1 = cudaFuncSetAttribute(kda_prepare_kernel,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          prep::kSmemAllocBytes);
+    cudaError_t e2 = cudaFuncSetAttribute(kda_recurrence_kernel,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          rec::kSmemAllocBytes);
+    attr_err = (e1 != cudaSuccess) ? e1 : e2;
+  });
+  if (attr_err != cudaSuccess) return KDA_ERR_LAUNCH_FAILED;
+  (void)cudaGetLastError();
+  void* const* ev = options ? options->events : nullptr;
+  auto mark = [&](int i) {
+    if (ev && ev[i]) cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), s);
+  };
+  if (!fixed || (flags & KDA_FLAG_VALIDATE)) {
+    kda_schedule_kernel<<<1, 1024, 0, s>>>(p);
+    mark(0);
+  }
+  if (T > 0) {
+    dim3 pg(static_cast<unsigned>(r.lay.slots), static_cast<unsigned>(H));
+    kda_prepare_kernel<<<pg, 128, prep::kSmemAllocBytes, s>>>(p, maps);
+  }
+  mark(1);
+  kda_recurrence_kernel<<<static_cast<unsigned>(N * H), 160, rec::kSmemAllocBytes, s>>>(p, maps);
+  mark(2);
+  if (cudaGetLastError() != cudaSuccess) return KDA_ERR_LAUNCH_FAILED;
+  return KDA_OK;
+}
+
+kda_status_t kda_prefill_status(void* workspace, void* stream, int32_t* device_status,
+                                 int clear) {
+  if (!workspace || !device_status) return KDA_ERR_NULL_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t val = 0;
+  if (cudaMemcpyAsync(&val, workspace, sizeof(int32_t), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return KDA_ERR_LAUNCH_FAILED;
+  if (clear && cudaMemsetAsync(workspace, 0, sizeof(int32_t), s) != cudaSuccess)
+    return KDA_ERR_LAUNCH_FAILED;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return KDA_ERR_LAUNCH_FAILED;
+  *device_status = val;
+  return KDA_OK;
+}
+
+}  // extern "C"

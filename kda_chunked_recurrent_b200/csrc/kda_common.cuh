@@ -1,0 +1,166 @@
+// kda_common.cuh — shapes, workspace layout and launch parameters shared by the
+// KDA prefill kernels and their host launcher.
+//
+// Chunked form used by every kernel (one (sequence, head), chunk of C = 64
+// tokens, local r = 0..63, G_r = running sum of g within the chunk, Gamma_r =
+// exp(G_r), beta folded into the triangular factor):
+//   A[r,s]   = sum_k k_r[k] k_s[k] exp(G_r[k] - G_s[k])          (s < r)
+//   T        = (I + diag(beta) A)^-1,   Tb = T diag(beta)
+//   W        = Tb (K * Gamma),            U = Tb V
+//   Aqk[r,s] = sum_k q_r[k] k_s[k] exp(G_r[k] - G_s[k])          (s <= r)
+//   Ud       = U - W S0
+//   O        = scale [ (Q * Gamma) S0 + Aqk Ud ]
+//   S1       = Diag(Gamma_63) S0 + (K * exp(G_63 - G))^T Ud
+// This is the chunk-wise factorisation the pages name for the prepare /
+// recurrence split ("decomp runs prepare and recurrence as two launches",
+// FlashInfer PR #4633 "Description"); the algebra is derived from the per-token
+// recurrence.  exp(G_r - G_s) is formed from 16-token sub-blocks so that no FP32
+// factor leaves [e^-80, e^80] when every g lies in [-5, 0] (the gate bound of
+// lmdeploy PR #5050 "Motivation").
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+
+namespace kda {
+
+constexpr int kD = 128;        // K = V = 128
+constexpr int kC = 64;         // chunk length
+constexpr int kSB = 16;        // sub-block length for the decay factorisation
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ---- workspace layout --------------------------------------------------------
+// header (status word, per-call validity) | chunk table | per-record tiles.
+// A "record" is one (chunk slot, head) pair: rec = slot * H + h.
+constexpr size_t kHeaderBytes = 1024;
+constexpr size_t kTileWT = 128 * 64 * 2;   // W^T   [128 k][64 tok] bf16
+constexpr size_t kTileQGT = 128 * 64 * 2;  // (Q*Gamma)^T [128 k][64 tok] bf16
+constexpr size_t kTileUT = 128 * 64 * 2;   // U^T   [128 v][64 tok] f16
+constexpr size_t kTileKdT = 128 * 64 * 2;  // Kd^T  [128 k][64 tok] f16
+constexpr size_t kTileAqk = 64 * 64 * 2;   // Aqk   [64 r][64 s]  f16
+constexpr size_t kTileGC = 128 * 4;        // Gamma at the chunk end, f32 [128]
+
+struct WorkspaceLayout {
+  size_t chunk_base;   // int32 [N+1]   first slot of each sequence
+  size_t seq_order;    // int32 [N]     longest-first order of sequences
+  size_t wt, qgt, ut, kdt, aqk, gc;   // per-record tiles (split variant)
+  size_t kpt, gp;      // checkpoint tiles per (sequence, head)
+  size_t total;
+  int64_t slots;       // chunk slots (upper bound on the number of chunks)
+};
+
+__host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Number of chunk slots that always suffices: sum_n ceil(len_n / C) <= T/C + N.
+__host__ __device__ inline int64_t chunk_slots(int64_t N, int64_t T, bool fixed) {
+  if (fixed) return N * ((T / N + kC - 1) / kC);
+  return T / kC + N;
+}
+
+inline WorkspaceLayout make_layout(int64_t N, int64_t T, int64_t H, bool fixed, bool split,
+                                   bool ckpt) {
+  WorkspaceLayout L{};
+  size_t off = kHeaderBytes;
+  L.chunk_base = off;
+  off = align_up(off + sizeof(int32_t) * (N + 1), 256);
+  L.seq_order = off;
+  off = align_up(off + sizeof(int32_t) * N, 1024);
+  L.slots = (N > 0 && T > 0) ? chunk_slots(N, T, fixed) : 0;
+  const size_t recs = split ? static_cast<size_t>(L.slots * H) : 0;
+  L.wt = off;  off = align_up(off + recs * kTileWT, 1024);
+  L.qgt = off; off = align_up(off + recs * kTileQGT, 1024);
+  L.ut = off;  off = align_up(off + recs * kTileUT, 1024);
+  L.kdt = off; off = align_up(off + recs * kTileKdT, 1024);
+  L.aqk = off; off = align_up(off + recs * kTileAqk, 1024);
+  L.gc = off;  off = align_up(off + recs * kTileGC, 1024);
+  const size_t crecs = ckpt ? static_cast<size_t>(N * H) : 0;
+  L.kpt = off; off = align_up(off + crecs * kTileKdT, 1024);
+  L.gp = off;  off = align_up(off + crecs * kTileGC, 1024);
+  L.total = off;
+  return L;
+}
+
+// Status words at the start of the workspace header.
+struct WsHeader {
+  int32_t status;    // first device error since the last clear (sticky)
+  int32_t call_ok;   // 1 when the schedule kernel of this call found valid metadata
+  int32_t pad[254];
+};
+
+// ---- kernel parameters ----------------------------------------------------------
+struct KdaParams {
+  // inputs
+  const uint16_t* q;
+  const uint16_t* k;
+  const uint16_t* v;
+  const float* g;
+  const uint16_t* beta;
+  float scale;
+  const float* h0;
+  const int32_t* cu_seqlens;     // NULL: fixed layout
+  const int32_t* ckpt_offsets;   // NULL: no checkpoint
+  // outputs
+  uint16_t* out;
+  float* ht;
+  float* ckpt;
+  // sizes
+  int32_t N, T, H, max_len;
+  int32_t fixed_len;             // sequence length in the fixed layout
+  int64_t slots;
+  // workspace
+  uint8_t* ws;
+  WorkspaceLayout lay;
+  uint32_t flags;
+  long long wait_budget;         // clock cycles per bounded wait; < 0 forces a timeout
+};
+
+// Tensor maps of the split variant (passed by value, __grid_constant__).
+struct SplitMaps {
+  CUtensorMap v_in;     // v [T][H][128] bf16, box (64 ch, 1 head, 64 tok), 128B swizzle
+  CUtensorMap wt;       // [recs*128][64] bf16, box (64, 128)
+  CUtensorMap qgt;      // [recs*128][64] bf16
+  CUtensorMap ut;       // [recs*128][64] f16
+  CUtensorMap kdt;      // [recs*128][64] f16
+  CUtensorMap aqk;      // [recs*64][64] f16, box (64, 64)
+  CUtensorMap kpt;      // [N*H*128][64] f16 (checkpoint)
+};
+
+enum : int32_t {
+  kStatusOk = 0,
+  kStatusBadCuSeqlens = 16,
+  kStatusBadCkptOffset = 17,
+  kStatusTimeout = 18,
+};
+
+enum : uint32_t { kFlagValidate = 1u, kFlagForceTimeout = 2u };
+
+__device__ __forceinline__ void record_status(uint8_t* ws, int32_t code) {
+  atomicCAS(reinterpret_cast<int32_t*>(ws), 0, code);
+}
+
+// Per-sequence geometry: start row, length, first chunk slot.  Values from
+// device metadata are clamped so that every derived address stays in bounds.
+struct SeqInfo {
+  int32_t start, len;
+  int64_t slot0;
+};
+
+__device__ __forceinline__ SeqInfo seq_info(const KdaParams& p, int32_t n) {
+  SeqInfo s;
+  if (p.cu_seqlens == nullptr) {
+    s.start = n * p.fixed_len;
+    s.len = p.fixed_len;
+    s.slot0 = static_cast<int64_t>(n) * ((p.fixed_len + kC - 1) / kC);
+  } else {
+    int32_t a = p.cu_seqlens[n], b = p.cu_seqlens[n + 1];
+    a = min(max(a, 0), p.T);
+    b = min(max(b, a), p.T);
+    s.start = a;
+    s.len = b - a;
+    const int32_t* cb = reinterpret_cast<const int32_t*>(p.ws + p.lay.chunk_base);
+    s.slot0 = cb[n];
+  }
+  return s;
+}
+
+}  // namespace kda

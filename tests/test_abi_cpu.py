@@ -1,0 +1,141 @@
+"""C ABI checks that need no GPU: the library loads, exports every declared entry
+point, and rejects bad arguments on the host before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from kda_chunked_recurrent_b200 import capi
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kda_prefill.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(kda_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("kda_prefill", "kda_prefill_workspace_size", "kda_prefill_status",
+              "kda_status_string", "kda_prefill_describe", "kda_workspace_init", "kda_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(capi.LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_status_strings_cover_all_codes():
+    for code in (0, 1, 2, 3, 4, 5, 6, 7, 8, 9, 10, 16, 17, 18):
+        s = capi.kda_status_string(code)
+        assert s and s != "unknown status"
+    assert capi.kda_status_string(12345) == "unknown status"
+
+
+def test_workspace_size_grows_with_work():
+    a = capi.kda_prefill_workspace_size(capi.make_shape(1, 512, 12), False)
+    b = capi.kda_prefill_workspace_size(capi.make_shape(1, 8192, 12), False)
+    c = capi.kda_prefill_workspace_size(capi.make_shape(1, 8192, 12), True)
+    assert 0 < a < b < c
+    assert capi.kda_prefill_workspace_size(capi.make_shape(0, 512, 12), False) == 0
+    assert capi.kda_prefill_workspace_size(capi.make_shape(1, 512, 0), False) == 0
+    assert capi.kda_prefill_workspace_size(capi.make_shape(1, -1, 1), False) == 0
+
+
+def test_describe_reports_grid_and_variant():
+    d = capi.kda_prefill_describe(capi.make_shape(8, 65536, 12, 8192), False)
+    assert "variant=split" in d and "chunk=64" in d and "recurrence_grid=96x160" in d
+
+
+# --- host-side validation with fake, never-dereferenced device addresses ----------
+BASE = 0x7F0000000000
+MB = 1 << 20
+
+
+def fake_args(T=128, H=2, N=1, ckpt=False, **over):
+    a = dict(q=BASE, k=BASE + 1 * MB, v=BASE + 2 * MB, g=BASE + 3 * MB, beta=BASE + 5 * MB,
+             scale=0.088, h0=BASE + 6 * MB, cu=None, shape=capi.make_shape(N, T, H),
+             out=BASE + 8 * MB, ht=BASE + 10 * MB, ck=None, cko=None,
+             ws=BASE + 64 * MB, wsb=capi.kda_prefill_workspace_size(capi.make_shape(N, T, H), ckpt),
+             opts=None)
+    if ckpt:
+        a["ck"] = BASE + 12 * MB
+        a["cko"] = BASE + 14 * MB
+    a.update(over)
+    return a
+
+
+def call(a):
+    return capi.kda_prefill(a["q"], a["k"], a["v"], a["g"], a["beta"], a["scale"], a["h0"], a["cu"],
+                            a["shape"], a["out"], a["ht"], a["ck"], a["cko"], a["ws"], a["wsb"],
+                            a["opts"], None)
+
+
+@pytest.mark.parametrize("field", ["q", "k", "v", "g", "beta", "out", "ws"])
+def test_null_pointer_rejected(field):
+    assert call(fake_args(**{field: None})) == capi.KDA_ERR_NULL_ARG
+
+
+def test_bad_shapes_rejected():
+    assert call(fake_args(shape=capi.make_shape(0, 128, 2))) == capi.KDA_ERR_BAD_SHAPE
+    assert call(fake_args(shape=capi.make_shape(1, 128, 0))) == capi.KDA_ERR_BAD_SHAPE
+    assert call(fake_args(shape=capi.make_shape(1, -5, 2))) == capi.KDA_ERR_BAD_SHAPE
+    # fixed layout needs T divisible by N
+    assert call(fake_args(shape=capi.make_shape(3, 128, 2))) == capi.KDA_ERR_BAD_SHAPE
+
+
+@pytest.mark.parametrize("field,delta", [("q", 8), ("k", 2), ("v", 4), ("g", 4), ("out", 8),
+                                         ("beta", 1), ("h0", 4), ("ht", 8), ("ws", 128)])
+def test_misaligned_rejected(field, delta):
+    a = fake_args()
+    a[field] = a[field] + delta
+    assert call(a) == capi.KDA_ERR_MISALIGNED
+
+
+def test_unpaired_checkpoint_rejected():
+    a = fake_args(ckpt=True)
+    assert call(dict(a, cko=None)) == capi.KDA_ERR_UNPAIRED_CKPT
+    assert call(dict(a, ck=None)) == capi.KDA_ERR_UNPAIRED_CKPT
+
+
+def test_partial_state_alias_rejected():
+    a = fake_args()
+    assert call(dict(a, ht=a["h0"] + 65536)) == capi.KDA_ERR_PARTIAL_ALIAS
+    b = fake_args(ckpt=True)
+    assert call(dict(b, ck=b["h0"])) == capi.KDA_ERR_PARTIAL_ALIAS
+
+
+def test_output_alias_rejected():
+    a = fake_args()
+    assert call(dict(a, out=a["q"])) == capi.KDA_ERR_OUT_ALIAS
+    assert call(dict(a, out=a["h0"])) == capi.KDA_ERR_OUT_ALIAS
+    assert call(dict(a, ht=a["g"])) == capi.KDA_ERR_OUT_ALIAS
+    assert call(dict(a, ws=a["v"])) == capi.KDA_ERR_OUT_ALIAS
+
+
+def test_workspace_too_small_rejected():
+    a = fake_args()
+    assert call(dict(a, wsb=a["wsb"] - 1)) == capi.KDA_ERR_WORKSPACE_TOO_SMALL
+
+
+def test_bad_options_rejected():
+    o = capi.kda_options_t()
+    o.variant = 7
+    assert call(fake_args(opts=o)) == capi.KDA_ERR_BAD_OPTION
+    o.variant = 0
+    o.flags = 1 << 9
+    assert call(fake_args(opts=o)) == capi.KDA_ERR_BAD_OPTION
+
+
+def test_valid_arguments_reach_the_device_check_without_gpu():
+    torch = pytest.importorskip("torch")
+    if torch.cuda.is_available():
+        pytest.skip("would launch on fake pointers")
+    assert call(fake_args()) == capi.KDA_ERR_UNSUPPORTED_DEVICE
+    assert call(fake_args(ht=BASE + 6 * MB)) == capi.KDA_ERR_UNSUPPORTED_DEVICE  # exact alias ok
