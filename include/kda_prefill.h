@@ -181,6 +181,43 @@ const char* kda_status_string(int status);
 kda_status_t kda_prefill_describe(const kda_shape_t* shape, int has_ckpt,
                                   const kda_options_t* options, char* buf, size_t n);
 
+/*
+ * Prefill without any device allocation by the caller.  (Not an operation of
+ * the method itself: the pages have no counterpart; it is an interface for
+ * callers that cannot allocate.)
+ *
+ * For callers that cannot call cudaMalloc — code running while a CUDA graph is
+ * captured into a memory pool it does not own, plugins whose host application
+ * owns every device allocation, or real-time paths where an allocation and the
+ * synchronisation it may cause are not allowed — and so cannot provide the
+ * workspace kda_prefill needs.  This entry point uses a scratch area built into
+ * the library instead: a static device array of KDA_NOALLOC_SCRATCH_BYTES that
+ * every GPU which loads the library holds until the process exits.  The caller
+ * still passes all inputs and outputs (same meaning, layout and rules as for
+ * kda_prefill); the library calls no cudaMalloc/cudaFree or allocating routine.
+ *
+ *   - Shapes whose kda_prefill_workspace_size exceeds KDA_NOALLOC_SCRATCH_BYTES
+ *     are refused with KDA_ERR_WORKSPACE_TOO_SMALL before anything is enqueued
+ *     (48 MiB covers, e.g., 12 heads x 2048 tokens, or 8 x 1024 tokens at H = 4).
+ *   - The first call on a device looks up the area's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     outside any stream capture.
+ *   - All calls on a device share the one area: calls that may overlap on the
+ *     GPU (different streams without ordering between them) race and must not
+ *     be issued.  Calls ordered on one stream are fine; nothing in the area has
+ *     to be cleared between calls.
+ *   - The device status word lives in the built-in area and is not readable
+ *     through this entry point; use kda_prefill with your own workspace when
+ *     validate mode or status reporting is needed.
+ */
+#define KDA_NOALLOC_SCRATCH_BYTES ((size_t)48 << 20)
+kda_status_t kda_prefill_noalloc(const void* q, const void* k, const void* v, const float* g,
+                                 const void* beta, float scale, const float* h0,
+                                 const int32_t* cu_seqlens, const kda_shape_t* shape,
+                                 void* out, float* ht, float* ckpt_state,
+                                 const int32_t* ckpt_offsets, const kda_options_t* options,
+                                 void* stream);
+
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
 int kda_version(void);
 

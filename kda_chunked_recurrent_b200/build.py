@@ -14,7 +14,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libkda_prefill.so")
-SOURCES = ["kda_api.cu", "kda_schedule.cu", "kda_prepare.cu", "kda_recurrence.cu"]
+SOURCES = ["kda_api.cu", "kda_schedule.cu", "kda_prepare.cu", "kda_recurrence.cu",
+           "kda_noalloc.cu"]
 HEADERS = ["kda_common.cuh", "sm100_primitives.cuh"]
 
 
