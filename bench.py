@@ -178,7 +178,9 @@ def cpu_baseline(inp_name, threads=0):
                     scale=inp.scale, cu_seqlens=torch.tensor([0, L], dtype=torch.int32),
                     h0=None if inp.h0 is None else inp.h0[:1])
     oracle.build_oracle()
-    cores = threads if threads > 0 else (os.cpu_count() or 1)
+    # OpenMP runs over the (sequence, head) units of the sample, so at most that
+    # many threads can be busy
+    cores = min(threads if threads > 0 else (os.cpu_count() or 1), inp.num_heads)
     t = time.perf_counter()
     oracle.prefill(sub, threads=cores)
     dt = time.perf_counter() - t

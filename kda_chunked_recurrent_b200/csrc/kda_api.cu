@@ -23,7 +23,7 @@ __global__ void kda_schedule_kernel(const KdaParams p);
 __global__ void kda_prepare_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps);
 __global__ void kda_recurrence_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps);
 namespace prep { extern const uint32_t kSmemAllocBytes; }
-namespace rec { extern const uint32_t kSmemAllocBytes; }
+namespace rec { extern const uint32_t kSmemAllocBytes; extern const int kThreadsPerCta; }
 }  // namespace kda
 
 using namespace kda;
@@ -79,13 +79,13 @@ kda_status_t check_options(const kda_options_t* o) {
   return KDA_OK;
 }
 
-kda_status_t check_shape(const kda_shape_t* s, bool fixed) {
+kda_status_t check_shape(const kda_shape_t* s, bool fixed, bool ckpt) {
   if (!s) return KDA_ERR_NULL_ARG;
   if (s->num_seqs < 1 || s->num_heads < 1 || s->total_tokens < 0 || s->max_seqlen < 0)
     return KDA_ERR_BAD_SHAPE;
   if (fixed && (s->total_tokens % s->num_seqs) != 0) return KDA_ERR_BAD_SHAPE;
   // 32-bit TMA coordinates of the per-record tiles: slots * H * 128 < 2^31
-  const int64_t slots = chunk_slots(s->num_seqs, s->total_tokens, fixed);
+  const int64_t slots = chunk_slots(s->num_seqs, s->total_tokens, fixed, ckpt);
   if (slots * static_cast<int64_t>(s->num_heads) * 128 >= (int64_t(1) << 31)) return KDA_ERR_BAD_SHAPE;
   if (static_cast<int64_t>(s->num_seqs) * s->num_heads * 128 >= (int64_t(1) << 31))
     return KDA_ERR_BAD_SHAPE;
@@ -99,6 +99,13 @@ Resolved resolve(const kda_shape_t* s, bool fixed, bool ckpt, const kda_options_
   r.fixed = fixed;
   r.lay = make_layout(s->num_seqs, s->total_tokens, s->num_heads, fixed, true, ckpt);
   return r;
+}
+
+int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
 }
 
 kda_status_t device_check() {
@@ -165,7 +172,7 @@ size_t kda_prefill_workspace_size(const kda_shape_t* shape, int has_ckpt,
   if (check_options(options) != KDA_OK) return 0;
   // the layout does not depend on whether cu_seqlens is given beyond the slot
   // bound; size for the larger (packed) bound so one workspace serves both.
-  if (check_shape(shape, false) != KDA_OK) return 0;
+  if (check_shape(shape, false, has_ckpt != 0) != KDA_OK) return 0;
   const Resolved r = resolve(shape, false, has_ckpt != 0, options);
   return r.lay.total;
 }
@@ -184,14 +191,15 @@ kda_status_t kda_prefill_describe(const kda_shape_t* shape, int has_ckpt,
                                   const kda_options_t* options, char* buf, size_t n) {
   if (!buf || n == 0) return KDA_ERR_NULL_ARG;
   kda_status_t st = check_options(options);
-  if (st == KDA_OK) st = check_shape(shape, false);
+  if (st == KDA_OK) st = check_shape(shape, false, has_ckpt != 0);
   if (st != KDA_OK) {
     snprintf(buf, n, "error: %s", kda_status_string(st));
     return st;
   }
   const Resolved r = resolve(shape, false, has_ckpt != 0, options);
   snprintf(buf, n,
-           "variant=split chunk=%d prepare_grid=(%lld,%d)x128 recurrence_grid=%lldx160 "
+           "variant=split chunk=%d prepare_items=%lldx%d (persistent, 2 CTAs/SM, 256 threads) "
+           "recurrence_grid=%lldx448 "
            "workspace_bytes=%zu",
            kC, static_cast<long long>(r.lay.slots), shape->num_heads,
            static_cast<long long>(shape->num_seqs) * shape->num_heads, r.lay.total);
@@ -209,7 +217,7 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
   if (st != KDA_OK) return st;
   const bool fixed = (cu_seqlens == nullptr);
   if (!shape) return KDA_ERR_NULL_ARG;
-  st = check_shape(shape, fixed);
+  st = check_shape(shape, fixed, ckpt_state != nullptr);
   if (st != KDA_OK) return st;
   const int64_t N = shape->num_seqs, T = shape->total_tokens, H = shape->num_heads;
   if (T > 0 && (!q || !k || !v || !g || !beta || !out)) return KDA_ERR_NULL_ARG;
@@ -286,9 +294,6 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
     mok &= make_map_2d(&maps.ut, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws + r.lay.ut, 64, recs * 128, 64, 128, 2);
     mok &= make_map_2d(&maps.kdt, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws + r.lay.kdt, 64, recs * 128, 64, 128, 2);
     mok &= make_map_2d(&maps.aqk, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws + r.lay.aqk, 64, recs * 64, 64, 64, 2);
-    if (ckpt)
-      mok &= make_map_2d(&maps.kpt, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws + r.lay.kpt, 64,
-                         static_cast<uint64_t>(N * H * 128), 64, 128, 2);
   }
   if (!mok) return KDA_ERR_LAUNCH_FAILED;
 
@@ -311,16 +316,19 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
   auto mark = [&](int i) {
     if (ev && ev[i]) cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), s);
   };
-  if (!fixed || (flags & KDA_FLAG_VALIDATE)) {
+  if (!fixed || ckpt || (flags & KDA_FLAG_VALIDATE)) {
     kda_schedule_kernel<<<1, 1024, 0, s>>>(p);
     mark(0);
   }
   if (T > 0) {
-    dim3 pg(static_cast<unsigned>(r.lay.slots), static_cast<unsigned>(H));
-    kda_prepare_kernel<<<pg, 128, prep::kSmemAllocBytes, s>>>(p, maps);
+    // persistent prepare grid: two CTAs per SM walk the (chunk slot, head) items
+    const int64_t items = r.lay.slots * H;
+    const int64_t grid = std::min<int64_t>(items, 2 * static_cast<int64_t>(sm_count()));
+    kda_prepare_kernel<<<static_cast<unsigned>(grid), 256, prep::kSmemAllocBytes, s>>>(p, maps);
   }
   mark(1);
-  kda_recurrence_kernel<<<static_cast<unsigned>(N * H), 160, rec::kSmemAllocBytes, s>>>(p, maps);
+  kda_recurrence_kernel<<<static_cast<unsigned>(N * H), rec::kThreadsPerCta, rec::kSmemAllocBytes, s>>>(
+      p, maps);
   mark(2);
   if (cudaGetLastError() != cudaSuccess) return KDA_ERR_LAUNCH_FAILED;
   return KDA_OK;

@@ -44,17 +44,19 @@ struct WorkspaceLayout {
   size_t chunk_base;   // int32 [N+1]   first slot of each sequence
   size_t seq_order;    // int32 [N]     longest-first order of sequences
   size_t wt, qgt, ut, kdt, aqk, gc;   // per-record tiles (split variant)
-  size_t kpt, gp;      // checkpoint tiles per (sequence, head)
   size_t total;
   int64_t slots;       // chunk slots (upper bound on the number of chunks)
 };
 
 __host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// Number of chunk slots that always suffices: sum_n ceil(len_n / C) <= T/C + N.
-__host__ __device__ inline int64_t chunk_slots(int64_t N, int64_t T, bool fixed) {
-  if (fixed) return N * ((T / N + kC - 1) / kC);
-  return T / kC + N;
+// Number of chunk slots that always suffices.  A sequence of length L is cut into
+// ceil(L / C) chunks; a checkpoint offset p (0 < p < L) adds one chunk boundary
+// at p, so sum_n chunks_n <= T / C + 2 N.  The fixed layout without checkpoints
+// is exactly N ceil(L / C).
+__host__ __device__ inline int64_t chunk_slots(int64_t N, int64_t T, bool fixed, bool ckpt) {
+  if (fixed && !ckpt) return N * ((T / N + kC - 1) / kC);
+  return T / kC + (ckpt ? 2 : 1) * N;
 }
 
 inline WorkspaceLayout make_layout(int64_t N, int64_t T, int64_t H, bool fixed, bool split,
@@ -65,7 +67,7 @@ inline WorkspaceLayout make_layout(int64_t N, int64_t T, int64_t H, bool fixed, 
   off = align_up(off + sizeof(int32_t) * (N + 1), 256);
   L.seq_order = off;
   off = align_up(off + sizeof(int32_t) * N, 1024);
-  L.slots = (N > 0 && T > 0) ? chunk_slots(N, T, fixed) : 0;
+  L.slots = (N > 0 && T > 0) ? chunk_slots(N, T, fixed, ckpt) : 0;
   const size_t recs = split ? static_cast<size_t>(L.slots * H) : 0;
   L.wt = off;  off = align_up(off + recs * kTileWT, 1024);
   L.qgt = off; off = align_up(off + recs * kTileQGT, 1024);
@@ -73,9 +75,6 @@ inline WorkspaceLayout make_layout(int64_t N, int64_t T, int64_t H, bool fixed, 
   L.kdt = off; off = align_up(off + recs * kTileKdT, 1024);
   L.aqk = off; off = align_up(off + recs * kTileAqk, 1024);
   L.gc = off;  off = align_up(off + recs * kTileGC, 1024);
-  const size_t crecs = ckpt ? static_cast<size_t>(N * H) : 0;
-  L.kpt = off; off = align_up(off + crecs * kTileKdT, 1024);
-  L.gp = off;  off = align_up(off + crecs * kTileGC, 1024);
   L.total = off;
   return L;
 }
@@ -122,7 +121,6 @@ struct SplitMaps {
   CUtensorMap ut;       // [recs*128][64] f16
   CUtensorMap kdt;      // [recs*128][64] f16
   CUtensorMap aqk;      // [recs*64][64] f16, box (64, 64)
-  CUtensorMap kpt;      // [N*H*128][64] f16 (checkpoint)
 };
 
 enum : int32_t {
@@ -138,29 +136,58 @@ __device__ __forceinline__ void record_status(uint8_t* ws, int32_t code) {
   atomicCAS(reinterpret_cast<int32_t*>(ws), 0, code);
 }
 
-// Per-sequence geometry: start row, length, first chunk slot.  Values from
-// device metadata are clamped so that every derived address stays in bounds.
+// Per-sequence geometry: start row, length, first chunk slot and the chunk split
+// at the checkpoint.  Values from device metadata are clamped so that every
+// derived address stays in bounds whatever the metadata holds.
 struct SeqInfo {
   int32_t start, len;
-  int64_t slot0;
+  int32_t ck;     // checkpoint prefix length clamped to [0, len], or -1 without checkpoints
+  int32_t nA;     // chunks covering [0, ck) when 0 < ck < len, else 0
+  int32_t nch;    // chunks of the sequence
+  int64_t slot0;  // first chunk slot
 };
 
-__device__ __forceinline__ SeqInfo seq_info(const KdaParams& p, int32_t n) {
+__device__ __forceinline__ SeqInfo seq_info(const KdaParams& p, int32_t n, bool need_slot = true) {
   SeqInfo s;
   if (p.cu_seqlens == nullptr) {
     s.start = n * p.fixed_len;
     s.len = p.fixed_len;
-    s.slot0 = static_cast<int64_t>(n) * ((p.fixed_len + kC - 1) / kC);
   } else {
     int32_t a = p.cu_seqlens[n], b = p.cu_seqlens[n + 1];
     a = min(max(a, 0), p.T);
     b = min(max(b, a), p.T);
     s.start = a;
     s.len = b - a;
-    const int32_t* cb = reinterpret_cast<const int32_t*>(p.ws + p.lay.chunk_base);
-    s.slot0 = cb[n];
+  }
+  s.ck = -1;
+  s.nA = 0;
+  if (p.ckpt_offsets != nullptr) {
+    s.ck = min(max(p.ckpt_offsets[n], 0), s.len);
+    if (s.ck > 0 && s.ck < s.len) s.nA = (s.ck + kC - 1) / kC;
+  }
+  const int32_t rest = s.len - (s.nA > 0 ? s.ck : 0);
+  s.nch = s.nA + (rest + kC - 1) / kC;
+  s.slot0 = 0;
+  if (need_slot) {
+    if (p.cu_seqlens == nullptr && p.ckpt_offsets == nullptr) {
+      s.slot0 = static_cast<int64_t>(n) * ((p.fixed_len + kC - 1) / kC);
+    } else {
+      s.slot0 = reinterpret_cast<const int32_t*>(p.ws + p.lay.chunk_base)[n];
+    }
   }
   return s;
+}
+
+// Token range of chunk j of a sequence: [t0, t0 + c), t0 relative to the sequence.
+__device__ __forceinline__ void chunk_span(const SeqInfo& s, int32_t j, int32_t& t0, int32_t& c) {
+  if (j < s.nA) {
+    t0 = j * kC;
+    c = min(kC, s.ck - t0);
+  } else {
+    const int32_t base = (s.nA > 0) ? s.ck : 0;
+    t0 = base + (j - s.nA) * kC;
+    c = min(kC, s.len - t0);
+  }
 }
 
 }  // namespace kda

@@ -1,7 +1,8 @@
 // kda_schedule.cu — per-call metadata for packed batches (one CTA).
 //
-// From cu_seqlens it builds the chunk table chunk_base[n] = sum_{m<n}
-// ceil(len_m / 64) (so every (chunk, head) gets a workspace slot) and a
+// From cu_seqlens (and the checkpoint offsets, which add one chunk boundary each)
+// it builds the chunk table chunk_base[n] = sum_{m<n} chunks_m (so every
+// (chunk, head) gets a workspace slot) and a
 // longest-first order of the sequences for the recurrence grid, the tail-
 // utilisation ordering FlashInfer PR #4262 "Dispatch contract" exposes as
 // seq_order.  In validate mode it checks the metadata the host never reads
@@ -36,28 +37,23 @@ __global__ void __launch_bounds__(kSchedThreads) kda_schedule_kernel(const KdaPa
     const int n = base + tid;
     int32_t cnt = 0, len = 0;
     if (n < p.N) {
-      int32_t a, b;
-      if (p.cu_seqlens != nullptr) {
-        a = p.cu_seqlens[n];
-        b = p.cu_seqlens[n + 1];
-        if (validate) {
+      if (validate) {
+        int32_t a = n * p.fixed_len, b = a + p.fixed_len;
+        if (p.cu_seqlens != nullptr) {
+          a = p.cu_seqlens[n];
+          b = p.cu_seqlens[n + 1];
           if (b < a || (n == 0 && a != 0) || (n == p.N - 1 && b != p.T) ||
               (p.max_len > 0 && b - a > p.max_len))
             atomicExch(&bad_cu, 1);
         }
-      } else {
-        a = n * p.fixed_len;
-        b = a + p.fixed_len;
+        if (p.ckpt_offsets != nullptr) {
+          const int32_t o = p.ckpt_offsets[n];
+          if (o < 0 || o > b - a) atomicExch(&bad_ck, 1);
+        }
       }
-      const int32_t raw_len = b - a;
-      a = min(max(a, 0), p.T);
-      b = min(max(b, a), p.T);
-      len = b - a;
-      cnt = (len + kC - 1) / kC;
-      if (validate && p.ckpt_offsets != nullptr) {
-        const int32_t o = p.ckpt_offsets[n];
-        if (o < 0 || o > raw_len) atomicExch(&bad_ck, 1);
-      }
+      const SeqInfo si = seq_info(p, n, false);  // clamped geometry, checkpoint split included
+      len = si.len;
+      cnt = si.nch;
       if (p.N <= kLptMax) s_len[n] = len;
     }
     // block-wide exclusive scan of cnt

@@ -50,7 +50,7 @@ def test_workspace_size_grows_with_work():
 
 def test_describe_reports_grid_and_variant():
     d = capi.kda_prefill_describe(capi.make_shape(8, 65536, 12, 8192), False)
-    assert "variant=split" in d and "chunk=64" in d and "recurrence_grid=96x160" in d
+    assert "variant=split" in d and "chunk=64" in d and "recurrence_grid=96x448" in d
 
 
 # --- host-side validation with fake, never-dereferenced device addresses ----------
