@@ -5,10 +5,10 @@
 // in TMEM/registers across chunks via tcgen05 GEMMs fed by TMA" and (c) "an
 // output kernel fusing the intra-chunk causal term with q.S").  The state is
 // kept transposed, S^T[v][k], in TMEM lanes v = 0..127, so every UMMA has M = 128:
-//   P_W^T = S0^T W^T                            (N=64, K=128; bf16)
+//   P_W^T = S0^T W^T                            (N=64, K=128; bf16; B = W^T, MN-major)
 //   Ud^T  = U^T - P_W^T                         (threads; f16 operand)
-//   S^T   = S0^T Diag(Gamma_end) + Ud^T Kd      (N=128, K=64; f16)
-//   O^T   = scale (S0^T (Q Gamma)^T + Ud^T Aqk^T)  (N=64; bf16 then f16)
+//   S^T   = S0^T Diag(Gamma_end) + Ud^T Kd      (N=128, K=64; f16; B = Kd rows, MN-major)
+//   O^T   = scale (S0^T (Q Gamma)^T + Ud^T Aqk^T)  (N=64; B = Q Gamma rows, K-major)
 // A checkpoint offset p is a chunk boundary of the schedule, so the checkpoint
 // state is S after the chunk that ends at p (h0 for p = 0, the final state for
 // p = len).
@@ -40,9 +40,10 @@
 namespace kda {
 
 namespace rec {
-constexpr uint32_t kWQ = 0;          // 32 KB [W^T | (Q Gamma)^T] MN-major B, 2 panels [128 k][64]
+constexpr uint32_t kWQ = 0;          // 16 KB W^T [128 k][64 tok] bf16, MN-major B;
+                                     // 16 KB Q Gamma [64 tok][128 k] bf16, K-major B, 2 panels
 constexpr uint32_t kUT = 32768;      // 16 KB U^T  [128 v][64 tok] f16 (128B swizzle)
-constexpr uint32_t kKd = 49152;      // 16 KB Kd^T [128 k][64 tok] f16, K-major B
+constexpr uint32_t kKd = 49152;      // 16 KB Kd [64 tok][128 k] f16, MN-major B, 2 panels
 constexpr uint32_t kAqk = 65536;     //  8 KB Aqk  [64 r][64 s] f16, K-major B
 constexpr uint32_t kGC = 73728;      // 512 B Gamma_end f32 [128]
 constexpr uint32_t kStage = 74752;
@@ -130,9 +131,11 @@ kda_recurrence_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps)
         uint8_t* base = sm + st * kStage;
         mbar_arrive_expect_tx(&full_bar[st], kStageTx);
         tma_load_2d(base + kWQ, &maps.wt, &full_bar[st], 0, recr * 128);
-        tma_load_2d(base + kWQ + 16384, &maps.qgt, &full_bar[st], 0, recr * 128);
+        tma_load_2d(base + kWQ + 16384, &maps.qg, &full_bar[st], 0, recr * 64);
+        tma_load_2d(base + kWQ + 16384 + 8192, &maps.qg, &full_bar[st], 64, recr * 64);
         tma_load_2d(base + kUT, &maps.ut, &full_bar[st], 0, recr * 128);
-        tma_load_2d(base + kKd, &maps.kdt, &full_bar[st], 0, recr * 128);
+        tma_load_2d(base + kKd, &maps.kd, &full_bar[st], 0, recr * 64);
+        tma_load_2d(base + kKd + 8192, &maps.kd, &full_bar[st], 64, recr * 64);
         tma_load_2d(base + kAqk, &maps.aqk, &full_bar[st], 0, recr * 64);
         bulk_load(base + kGC, p.ws + p.lay.gc + static_cast<size_t>(recr) * kTileGC, 512,
                   &full_bar[st]);
@@ -140,9 +143,9 @@ kda_recurrence_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps)
       };
       if (nch > 0) {
         prefetch_tmap(&maps.wt);
-        prefetch_tmap(&maps.qgt);
+        prefetch_tmap(&maps.qg);
         prefetch_tmap(&maps.ut);
-        prefetch_tmap(&maps.kdt);
+        prefetch_tmap(&maps.kd);
         prefetch_tmap(&maps.aqk);
       }
       for (int j = 0; j < nch && j < 2; ++j) load(j);
@@ -167,7 +170,8 @@ kda_recurrence_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps)
       uint64_t* last_commit = nullptr;
       uint32_t last_parity = 0;
       const uint32_t id_p = idesc_f16(128, 64, kFmtBF16, kKMajor, kMNMajor);
-      const uint32_t id_s = idesc_f16(128, 128, kFmtF16, kKMajor, kKMajor);
+      const uint32_t id_q = idesc_f16(128, 64, kFmtBF16, kKMajor, kKMajor);
+      const uint32_t id_s = idesc_f16(128, 128, kFmtF16, kKMajor, kMNMajor);
       const uint32_t id_o = idesc_f16(128, 64, kFmtF16, kKMajor, kKMajor);
       const uint32_t aUd = smem_u32(sm + kUdT);
       bool ok = true;
@@ -196,7 +200,7 @@ kda_recurrence_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           umma_f16(tbase + reg + 64, sdesc_sw128(aS0 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                   sdesc_sw128(bQ + kk * 2048, 16384, 1024), id_p, kk > 0);
+                   sdesc_sw128(bQ + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id_q, kk > 0);
         last_commit = &mma1_bar;
         last_parity = j & 1;
         ok = mbar_wait(&ud_bar, j & 1, budget) && !*abort_flag;
@@ -205,7 +209,7 @@ kda_recurrence_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps)
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           umma_f16(tbase + kColS, sdesc_sw128(aUd + kk * 32, 16, 1024),
-                   sdesc_sw128(bKd + kk * 32, 16, 1024), id_s, 1);
+                   sdesc_sw128(bKd + kk * 2048, 8192, 1024), id_s, 1);
         umma_commit(&sready_bar);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
