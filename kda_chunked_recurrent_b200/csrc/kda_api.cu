@@ -141,6 +141,20 @@ bool make_map_tokens(CUtensorMap* m, const void* base, uint64_t T, uint64_t H) {
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Token rows of one head, whole: box (128 channels, 1 head, 64 tokens), no swizzle,
+// so a chunk lands in shared memory as [64 tok][128 ch].
+bool make_map_rows(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t T,
+                   uint64_t H, uint32_t elem_bytes) {
+  const cuuint64_t dims[3] = {128, H, T};
+  const cuuint64_t strides[2] = {128ull * elem_bytes, H * 128ull * elem_bytes};
+  const cuuint32_t box[3] = {128, 1, 64};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return encode_fn()(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 extern "C" {
@@ -289,6 +303,9 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
   bool mok = true;
   if (T > 0) {
     mok &= make_map_tokens(&maps.v_in, v, T, H);
+    mok &= make_map_rows(&maps.q_in, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, T, H, 2);
+    mok &= make_map_rows(&maps.k_in, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, k, T, H, 2);
+    mok &= make_map_rows(&maps.g_in, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, g, T, H, 4);
     mok &= make_map_2d(&maps.wt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ws + r.lay.wt, 64, recs * 128, 64, 128, 2);
     mok &= make_map_2d(&maps.qg, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ws + r.lay.qg, 128, recs * 64, 64, 64, 2);
     mok &= make_map_2d(&maps.ut, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws + r.lay.ut, 64, recs * 128, 64, 128, 2);

@@ -116,6 +116,9 @@ struct KdaParams {
 // Tensor maps of the split variant (passed by value, __grid_constant__).
 struct SplitMaps {
   CUtensorMap v_in;     // v [T][H][128] bf16, box (64 ch, 1 head, 64 tok), 128B swizzle
+  CUtensorMap q_in;     // q [T][H][128] bf16, box (128 ch, 1 head, 64 tok), no swizzle
+  CUtensorMap k_in;     // k, as q
+  CUtensorMap g_in;     // g [T][H][128] f32, box (128 ch, 1 head, 64 tok), no swizzle
   CUtensorMap wt;       // [recs*128][64] bf16, box (64, 128)
   CUtensorMap qg;       // [recs*64][128] bf16, box (64, 64): one 64-channel panel
   CUtensorMap ut;       // [recs*128][64] f16, box (64, 128)

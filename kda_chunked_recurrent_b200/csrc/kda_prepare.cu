@@ -17,6 +17,11 @@
 // system per chunk and emits W and U"; the split into prepare and recurrence
 // launches is the "decomp" variant of FlashInfer PR #4633 "Description").
 //
+// Inputs of a chunk: q, k (bf16) and g (f32) arrive by TMA as whole [64 tok][128 ch]
+// tiles into shared memory the previous chunk no longer needs (issued as soon as
+// that chunk's second UMMA has completed, with the rows already prefetched into
+// L2 one chunk earlier); v follows by TMA straight into its UMMA operand layout.
+//
 // Thread mapping for the element-wise part: thread t owns the channel pair
 // (2p, 2p+1), p = t % 64, in sub-block b = t / 64 (tokens 16b .. 16b+15), so a
 // warp writes one full 128-byte row of one operand per store.
@@ -56,6 +61,12 @@ constexpr uint32_t kKG = 16384;      // 16 KB  K*Gamma tile, MN-major A of W^T
 constexpr uint32_t kL = 32768;       // 32 KB  [K+; Q+], K-major A: 2 panels [128 rows][64 ch]
 constexpr uint32_t kR = 65536;       // 40 KB  R^0..R^3, K-major B: 2 panels [160 rows][64 ch]
 constexpr uint32_t kBytes = 65536 + 40960;
+// raw input tiles of a chunk, landed before its element-wise pass (which reads
+// them into registers before anything overwrites these regions)
+constexpr uint32_t kQraw = kV;                  // q [64 tok][128 ch] bf16
+constexpr uint32_t kKraw = kKG;                 // k [64 tok][128 ch] bf16
+constexpr uint32_t kGraw = kR;                  // g [64 tok][128 ch] f32 (32 KB)
+constexpr uint32_t kRawTx = 16384 + 16384 + 32768;
 // aliases of [K+; Q+] once the first UMMA has completed: the solve scratch, and
 // after the solve the staging tiles of the W^T / U^T TMA stores
 constexpr int kLdh = 72;
@@ -243,7 +254,7 @@ kda_prepare_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
-  __shared__ uint64_t tma_bar, mma_bar;
+  __shared__ uint64_t tma_bar, mma_bar, raw_bar;
   __shared__ uint32_t tmem_slot;
   __shared__ float s_beta[kC];
   __shared__ float2 s_tot[4][64];     // per sub-block sums of g (log2 domain), channel pairs
@@ -259,8 +270,12 @@ kda_prepare_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps) {
   if (tid == 0) {
     mbar_init(&tma_bar, 1);
     mbar_init(&mma_bar, 1);
+    mbar_init(&raw_bar, 1);
     fence_mbar_init();
     prefetch_tmap(&maps.v_in);
+    prefetch_tmap(&maps.q_in);
+    prefetch_tmap(&maps.k_in);
+    prefetch_tmap(&maps.g_in);
     prefetch_tmap(&maps.wt);
     prefetch_tmap(&maps.ut);
     prefetch_tmap(&maps.aqk);
@@ -276,6 +291,14 @@ kda_prepare_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps) {
   bool ok = true;
   int mma_commits = 0;     // UMMA commits issued so far (their mbarrier phases)
   int tma_issued = 0;      // v tiles issued so far (tma_bar phases)
+  int raw_issued = 0;      // raw q/k/g tile sets issued so far (raw_bar phases)
+  bool raw_for_cur = false;  // the current item's raw tiles are already in flight
+  auto issue_raw = [&](const PrepItem& it) {  // thread 0 only
+    mbar_arrive_expect_tx(&raw_bar, kRawTx);
+    tma_load_3d(sm + kQraw, &maps.q_in, &raw_bar, 0, it.h, it.t0);
+    tma_load_3d(sm + kKraw, &maps.k_in, &raw_bar, 0, it.h, it.t0);
+    tma_load_3d(sm + kGraw, &maps.g_in, &raw_bar, 0, it.h, it.t0);
+  };
 
   PrepItem cur;
   bool cur_valid = blockIdx.x < nitems && locate_item(p, blockIdx.x, cur);
@@ -291,39 +314,15 @@ kda_prepare_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps) {
     const int32_t t0 = cur.t0, c = cur.c;
     const int64_t rec = cur.rec;
 
-    // ---- loads: g (float2), k, q (bf16x2) for 16 tokens x 2 channels; beta
     const int cp = tid & 63;         // channel pair
     const int blk = tid >> 6;        // sub-block 0..3
-    const int ch0 = 2 * cp;
-    const int64_t rstride = static_cast<int64_t>(p.H) * kD;
-    const int64_t base_el = (static_cast<int64_t>(t0) * p.H + h) * kD + ch0;
-    float2 G[16];
-    uint32_t kw[16], qw[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int r = blk * 16 + i;
-      const int64_t el = base_el + r * rstride;
-      if (r < c) {
-        G[i] = __ldg(reinterpret_cast<const float2*>(p.g + el));
-        kw[i] = __ldg(reinterpret_cast<const unsigned int*>(p.k + el));
-        qw[i] = __ldg(reinterpret_cast<const unsigned int*>(p.q + el));
-      } else {
-        G[i] = make_float2(0.f, 0.f);
-        kw[i] = 0u;
-        qw[i] = 0u;
-      }
+    if (!raw_for_cur) {
+      if (tid == 0) issue_raw(cur);
+      ++raw_issued;
     }
+    raw_for_cur = false;
     uint16_t beta_raw = 0;   // consumed only after the operand pass, so its latency hides
     if (tid < c) beta_raw = p.beta[static_cast<int64_t>(t0 + tid) * p.H + h];
-
-    // ---- TMA: v tile straight into the MN-major A operand of U^T
-    if (tid == 0) {
-      mbar_arrive_expect_tx(&tma_bar, 16384);
-      tma_load_3d(sm + kV, &maps.v_in, &tma_bar, 0, h, t0);
-      tma_load_3d(sm + kV + 8192, &maps.v_in, &tma_bar, 64, h, t0);
-    }
-    const uint32_t tma_parity = static_cast<uint32_t>(tma_issued & 1);
-    ++tma_issued;
 
     // ---- L2 prefetch of the next item's rows (q, k, v: 256 B, g: 512 B per token; beta)
     if (nxt_valid) {
@@ -348,6 +347,22 @@ kda_prepare_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps) {
       }
     }
 
+    // ---- raw tiles -> registers: g (float2), k, q (bf16x2) for 16 tokens x 2 channels
+    ok = mbar_wait(&raw_bar, static_cast<uint32_t>((raw_issued - 1) & 1), budget);
+    float2 G[16];
+    uint32_t kw[16], qw[16];
+    {
+      const float2* gs = reinterpret_cast<const float2*>(sm + kGraw) + blk * 16 * 64 + cp;
+      const uint32_t* ks = reinterpret_cast<const uint32_t*>(sm + kKraw) + blk * 16 * 64 + cp;
+      const uint32_t* qs = reinterpret_cast<const uint32_t*>(sm + kQraw) + blk * 16 * 64 + cp;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const bool in = ok && blk * 16 + i < c;   // rows past the chunk read as zero
+        G[i] = in ? gs[i * 64] : make_float2(0.f, 0.f);
+        kw[i] = in ? ks[i * 64] : 0u;
+        qw[i] = in ? qs[i * 64] : 0u;
+      }
+    }
     // ---- gate scan within the sub-block; one exchange gives every sub-block start
     {
       float2 run = make_float2(0.f, 0.f);
@@ -362,7 +377,17 @@ kda_prepare_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps) {
     }
     // the previous item's TMA stores have finished reading their staging tiles
     if (tid == 0) bulk_wait_read();
-    __syncthreads();
+    ok = !__syncthreads_or(!ok);
+    if (!ok) break;
+    // ---- TMA: v tile straight into the MN-major A operand of U^T (the raw q tile
+    // in that region has been read by every thread)
+    if (tid == 0) {
+      mbar_arrive_expect_tx(&tma_bar, 16384);
+      tma_load_3d(sm + kV, &maps.v_in, &tma_bar, 0, h, t0);
+      tma_load_3d(sm + kV + 8192, &maps.v_in, &tma_bar, 64, h, t0);
+    }
+    const uint32_t tma_parity = static_cast<uint32_t>(tma_issued & 1);
+    ++tma_issued;
     float2 Bs[4];   // B_i: G at the first token of sub-block i
     float2 E;       // G at the chunk end
     {
@@ -615,6 +640,17 @@ kda_prepare_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps) {
       ok = mbar_wait(&mma_bar, static_cast<uint32_t>((mma_commits - 1) & 1), budget);
     }
     ok = !__syncthreads_or(!ok);
+    // the next item's raw tiles go into v / K Gamma / R, all free now that the
+    // second UMMA has completed (the Aqk staging tile in R has been read once
+    // the bulk group is drained)
+    if (ok && nxt_valid) {
+      if (tid == 0) {
+        bulk_wait_read();
+        issue_raw(nxt);
+      }
+      ++raw_issued;
+      raw_for_cur = true;
+    }
     if (ok) {
       tc_fence_after();
       // warps 0-3: W^T rows (lane = k); warps 4-7: U^T rows (lane = v), into the
@@ -667,6 +703,8 @@ kda_prepare_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps) {
         mbar_wait(&tma_bar, static_cast<uint32_t>((tma_issued - 1) & 1), drain_budget);
       if (mma_commits > 0)
         mbar_wait(&mma_bar, static_cast<uint32_t>((mma_commits - 1) & 1), drain_budget);
+      if (raw_issued > 0)
+        mbar_wait(&raw_bar, static_cast<uint32_t>((raw_issued - 1) & 1), drain_budget);
     }
     bulk_wait_all();   // the tile stores this thread issued are complete
   }
