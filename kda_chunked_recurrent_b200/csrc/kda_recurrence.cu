@@ -5,26 +5,35 @@
 // in TMEM/registers across chunks via tcgen05 GEMMs fed by TMA" and (c) "an
 // output kernel fusing the intra-chunk causal term with q.S").  The state is
 // kept transposed, S^T[v][k], in TMEM lanes v = 0..127, so every UMMA has M = 128:
-//   P_W^T = S0^T W^T                            (N=64, K=128; bf16; B = W^T, MN-major)
+//   [P_W^T | P_Q^T] = S0^T [W^T | (Q Gamma)^T]  (N=128, K=128; bf16; MN-major B)
 //   Ud^T  = U^T - P_W^T                         (threads; f16 operand)
 //   S^T   = S0^T Diag(Gamma_end) + Ud^T Kd      (N=128, K=64; f16; B = Kd rows, MN-major)
-//   O^T   = scale (S0^T (Q Gamma)^T + Ud^T Aqk^T)  (N=64; B = Q Gamma rows, K-major)
+//   O^T   = scale (P_Q^T + Ud^T Aqk^T)          (N=64, K=64; f16)
 // A checkpoint offset p is a chunk boundary of the schedule, so the checkpoint
 // state is S after the chunk that ends at p (h0 for p = 0, the final state for
 // p = len).
 //
-// Serial chain per chunk: S ready -> (state warps) S0^T operand + decayed S ->
-// P_W -> (state warps) Ud -> S update.  P_Q is issued right after P_W and runs
-// while the state warps form Ud; the Ud Aqk output product follows the S update.
-// The P/O accumulators are triple-buffered in TMEM (S: 128 columns + 3 x 128) so
-// the output warps drain chunk j while chunks j+1 and j+2 proceed.
+// Serial chain per chunk: S ready -> (state warps) bf16 S0^T into TMEM + decayed S
+// -> [P_W | P_Q] -> (state warps) f16 Ud^T into TMEM -> S update.  S0^T and Ud^T
+// are the A operands of their UMMAs straight from tensor memory, so shared memory
+// only feeds the B tiles.  P_W and P_Q share one N = 128 product (an M = 128 UMMA
+// costs about the same at N = 64 and N = 128); the Ud Aqk output product follows
+// the S update.  [P_W | P_Q/O] alternate between two TMEM regions, so the output
+// warps drain chunk j while chunk j+1 proceeds; the chunk operands stream
+// through a three-stage TMA ring.
+//
+// Tensor memory (512 columns):
+//   [0, 128)    S^T f32 (lane v, column k)
+//   [128, 384)  two regions: P_W^T (64 columns) then P_Q^T / O^T (64 columns)
+//   [384, 448)  S0^T bf16, two k per column (A operand of [P_W | P_Q])
+//   [448, 480)  Ud^T f16, two tokens per column (A operand of the update and O)
 //
 // Warp roles:
 //   warps 0-7   state warps: warp w serves TMEM lanes 32 (w % 4) .. + 31 and half
 //               w / 4 of every state row (64 columns; 32 tokens of P_W / Ud);
 //   warps 8-11  output warps: read O^T out of TMEM and store o;
 //   warp 12     lane 0 issues every UMMA;
-//   warp 13     lane 0 streams the 2-stage TMA ring (kept apart from the UMMA
+//   warp 13     lane 0 streams the operand ring (kept apart from the UMMA
 //               issuer so a stage refill never delays the next chunk's P_W).
 //
 // In-place state update (ht == h0) is safe: each thread reads its part of the h0
@@ -40,21 +49,21 @@
 namespace kda {
 
 namespace rec {
-constexpr uint32_t kWQ = 0;          // 16 KB W^T [128 k][64 tok] bf16, MN-major B;
-                                     // 16 KB Q Gamma [64 tok][128 k] bf16, K-major B, 2 panels
+constexpr uint32_t kWQ = 0;          // 32 KB [W^T | (Q Gamma)^T], MN-major B, 2 panels [128 k][64 tok]
 constexpr uint32_t kUT = 32768;      // 16 KB U^T  [128 v][64 tok] f16 (128B swizzle)
 constexpr uint32_t kKd = 49152;      // 16 KB Kd [64 tok][128 k] f16, MN-major B, 2 panels
 constexpr uint32_t kAqk = 65536;     //  8 KB Aqk  [64 r][64 s] f16, K-major B
 constexpr uint32_t kGC = 73728;      // 512 B Gamma_end f32 [128]
 constexpr uint32_t kStage = 74752;
-constexpr uint32_t kS0T = 2 * kStage;        // 32 KB S0^T bf16, K-major A, 2 panels [128 v][64 k]
-constexpr uint32_t kUdT = kS0T + 32768;      // 16 KB Ud^T f16, K-major A [128 v][64 tok]
-constexpr uint32_t kBytes = kUdT + 16384;
+constexpr int kStages = 3;
+constexpr uint32_t kBytes = kStages * kStage;
 constexpr uint32_t kSmemAlloc = kBytes + 1024;
 constexpr uint32_t kStageTx = 32768 + 16384 + 16384 + 8192 + 512;
-// TMEM columns: S^T, then three P/O regions (W part cols +0..63, Q/O part +64..127)
 constexpr uint32_t kColS = 0;
-constexpr int kRegions = 3;
+constexpr uint32_t kColP = 128;
+constexpr uint32_t kColS0 = 384;
+constexpr uint32_t kColUd = 448;
+constexpr int kRegions = 2;
 constexpr int kStateWarps = 8, kOutWarps = 4;
 constexpr int kMmaWarp = kStateWarps + kOutWarps;
 constexpr int kTmaWarp = kMmaWarp + 1;
@@ -64,9 +73,10 @@ constexpr uint32_t kOutThreads = kOutWarps * 32;
 extern const uint32_t kSmemAllocBytes = kSmemAlloc;
 extern const int kThreadsPerCta = kThreads;
 static_assert(kSmemAlloc <= 227 * 1024, "shared memory budget");
+static_assert(kColP + kRegions * 128 <= kColS0 && kColUd + 32 <= 512, "tensor memory budget");
 }  // namespace rec
 
-__device__ __forceinline__ uint32_t region_col(int j) { return 128u + 128u * (j % rec::kRegions); }
+__device__ __forceinline__ uint32_t region_col(int j) { return rec::kColP + 128u * (j % rec::kRegions); }
 
 __global__ void __launch_bounds__(rec::kThreads, 1)
 kda_recurrence_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps) {
@@ -74,7 +84,7 @@ kda_recurrence_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
-  __shared__ uint64_t full_bar[2], empty_bar[2], oready_bar[kRegions], ofree_bar[kRegions];
+  __shared__ uint64_t full_bar[kStages], empty_bar[kStages], oready_bar[kRegions], ofree_bar[kRegions];
   __shared__ uint64_t s0_bar, ud_bar, mma1_bar, sready_bar;
   __shared__ uint32_t tmem_slot;
   __shared__ int32_t s_abort;
@@ -96,9 +106,9 @@ kda_recurrence_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps)
   const long long drain_budget = 4000000000LL;
 
   if (tid == 0) {
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kStages; ++i) {
       mbar_init(&full_bar[i], 1);
-      mbar_init(&empty_bar[i], 1);
+      mbar_init(&empty_bar[i], 2);   // the last UMMA commit of the chunk + the output store
     }
     for (int i = 0; i < kRegions; ++i) {
       mbar_init(&oready_bar[i], 1);
@@ -122,17 +132,16 @@ kda_recurrence_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps)
   if (warp == kTmaWarp) {
     // =========================== TMA producer ====================================
     if ((tid & 31) == 0) {
-      int issued[2] = {0, 0};
+      int issued[kStages] = {0, 0, 0};
       auto load = [&](int j) {
-        const int st = j & 1;
+        const int st = j % kStages;
         const int64_t slot = si.slot0 + j;
         if (slot < 0 || slot >= p.slots) return;  // corrupt metadata: nothing to load
         const int32_t recr = static_cast<int32_t>(slot * p.H + h);
         uint8_t* base = sm + st * kStage;
         mbar_arrive_expect_tx(&full_bar[st], kStageTx);
         tma_load_2d(base + kWQ, &maps.wt, &full_bar[st], 0, recr * 128);
-        tma_load_2d(base + kWQ + 16384, &maps.qg, &full_bar[st], 0, recr * 64);
-        tma_load_2d(base + kWQ + 16384 + 8192, &maps.qg, &full_bar[st], 64, recr * 64);
+        tma_load_2d(base + kWQ + 16384, &maps.qgt, &full_bar[st], 0, recr * 128);
         tma_load_2d(base + kUT, &maps.ut, &full_bar[st], 0, recr * 128);
         tma_load_2d(base + kKd, &maps.kd, &full_bar[st], 0, recr * 64);
         tma_load_2d(base + kKd + 8192, &maps.kd, &full_bar[st], 64, recr * 64);
@@ -143,24 +152,24 @@ kda_recurrence_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps)
       };
       if (nch > 0) {
         prefetch_tmap(&maps.wt);
-        prefetch_tmap(&maps.qg);
+        prefetch_tmap(&maps.qgt);
         prefetch_tmap(&maps.ut);
         prefetch_tmap(&maps.kd);
         prefetch_tmap(&maps.aqk);
       }
-      for (int j = 0; j < nch && j < 2; ++j) load(j);
+      for (int j = 0; j < nch && j < kStages; ++j) load(j);
       bool ok = true;
-      for (int j = 0; j + 2 < nch && ok; ++j) {
-        // stage j % 2 is free once every UMMA of chunk j has completed
-        ok = mbar_wait_sleep(&empty_bar[j & 1], (j >> 1) & 1, budget) && !*abort_flag;
-        if (ok) load(j + 2);
+      for (int j = 0; j + kStages < nch && ok; ++j) {
+        // stage j % kStages is free once every UMMA of chunk j has completed
+        ok = mbar_wait_sleep(&empty_bar[j % kStages], (j / kStages) & 1, budget) && !*abort_flag;
+        if (ok) load(j + kStages);
       }
       if (!ok) {
         *abort_flag = 1;
         record_status(p.ws, kStatusTimeout);
       }
       // drain: every TMA load this thread issued completes before exit
-      for (int st = 0; st < 2; ++st)
+      for (int st = 0; st < kStages; ++st)
         if (issued[st] > 0)
           mbar_wait(&full_bar[st], static_cast<uint32_t>((issued[st] - 1) & 1), drain_budget);
     }
@@ -169,56 +178,45 @@ kda_recurrence_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps)
     if ((tid & 31) == 0) {
       uint64_t* last_commit = nullptr;
       uint32_t last_parity = 0;
-      const uint32_t id_p = idesc_f16(128, 64, kFmtBF16, kKMajor, kMNMajor);
-      const uint32_t id_q = idesc_f16(128, 64, kFmtBF16, kKMajor, kKMajor);
+      const uint32_t id_p = idesc_f16(128, 128, kFmtBF16, kKMajor, kMNMajor);
       const uint32_t id_s = idesc_f16(128, 128, kFmtF16, kKMajor, kMNMajor);
       const uint32_t id_o = idesc_f16(128, 64, kFmtF16, kKMajor, kKMajor);
-      const uint32_t aUd = smem_u32(sm + kUdT);
+      const uint32_t tS0 = tbase + kColS0, tUd = tbase + kColUd;
       bool ok = true;
       for (int j = 0; j < nch && ok; ++j) {
-        const int st = j & 1;
+        const int st = j % kStages;
         const int rg = j % kRegions;
-        const uint32_t reg = region_col(j);
-        const uint32_t aS0 = smem_u32(sm + kS0T);
+        const uint32_t tP = tbase + region_col(j);
         const uint32_t bW = smem_u32(sm + st * kStage + kWQ);
-        const uint32_t bQ = bW + 16384;
         const uint32_t bKd = smem_u32(sm + st * kStage + kKd);
         const uint32_t bAq = smem_u32(sm + st * kStage + kAqk);
-        ok = mbar_wait(&s0_bar, j & 1, budget) && !*abort_flag;
-        // the output warps must have drained this region (chunk j - 3)
+        ok = mbar_wait_spin(&s0_bar, j & 1, budget) && !*abort_flag;
+        // the output warps must have drained this region (chunk j - 2)
         if (ok && j >= kRegions)
-          ok = mbar_wait(&ofree_bar[rg], ((j - kRegions) / kRegions) & 1, budget) && !*abort_flag;
+          ok = mbar_wait_spin(&ofree_bar[rg], ((j - kRegions) / kRegions) & 1, budget) && !*abort_flag;
         if (!ok) break;
         tc_fence_after();
-        // P_W^T = S0^T W^T (the chain needs it) then P_Q^T = S0^T (Q Gamma)^T, which
-        // runs while the state warps form Ud
+        // [P_W^T | P_Q^T] = S0^T [W^T | (Q Gamma)^T]
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          umma_f16(tbase + reg, sdesc_sw128(aS0 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                   sdesc_sw128(bW + kk * 2048, 16384, 1024), id_p, kk > 0);
+          umma_f16_ta(tP, tS0 + kk * 8, sdesc_sw128(bW + kk * 2048, 16384, 1024), id_p, kk > 0);
         umma_commit(&mma1_bar);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_f16(tbase + reg + 64, sdesc_sw128(aS0 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                   sdesc_sw128(bQ + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id_q, kk > 0);
         last_commit = &mma1_bar;
         last_parity = j & 1;
-        ok = mbar_wait(&ud_bar, j & 1, budget) && !*abort_flag;
+        ok = mbar_wait_spin(&ud_bar, j & 1, budget) && !*abort_flag;
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          umma_f16(tbase + kColS, sdesc_sw128(aUd + kk * 32, 16, 1024),
-                   sdesc_sw128(bKd + kk * 2048, 8192, 1024), id_s, 1);
+          umma_f16_ta(tbase + kColS, tUd + kk * 8, sdesc_sw128(bKd + kk * 2048, 8192, 1024), id_s, 1);
         umma_commit(&sready_bar);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          umma_f16(tbase + reg + 64, sdesc_sw128(aUd + kk * 32, 16, 1024),
-                   sdesc_sw128(bAq + kk * 32, 16, 1024), id_o, 1);
+          umma_f16_ta(tP + 64, tUd + kk * 8, sdesc_sw128(bAq + kk * 32, 16, 1024), id_o, 1);
         umma_commit(&oready_bar[rg]);
         umma_commit(&empty_bar[st]);
         last_commit = &empty_bar[st];
-        last_parity = (j >> 1) & 1;
+        last_parity = (j / kStages) & 1;
       }
       if (!ok) {
         *abort_flag = 1;
@@ -229,19 +227,25 @@ kda_recurrence_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps)
     }
   } else if (warp >= kStateWarps) {
     // =========================== output warps ===================================
+    // A full chunk leaves through the stage's [W^T | (Q Gamma)^T] tiles (dead once
+    // [P_W | P_Q] has completed) as one TMA tile store; a partial chunk (the end of
+    // a sequence, or a checkpoint boundary) uses plain stores so that nothing past
+    // the chunk is written.  The stage is released once the store has read it.
     const int qw = warp - kStateWarps;
     const int v = qw * 32 + (tid & 31);
+    const bool leader = (tid == kStateWarps * 32);
     const uint32_t lane_base = static_cast<uint32_t>(qw * 32);
     const int64_t ostride = static_cast<int64_t>(p.H) * kD;
     bool ok = true;
     for (int j = 0; j < nch; ++j) {
       const int rg = j % kRegions;
-      ok = mbar_wait_sleep(&oready_bar[rg], (j / kRegions) & 1, budget) && !*abort_flag;
+      const int st = j % kStages;
+      ok = mbar_wait(&oready_bar[rg], (j / kRegions) & 1, budget) && !*abort_flag;
+      ok = !named_bar_or(2, kOutThreads, !ok);   // the same decision in every output thread
       if (!ok) break;
       tc_fence_after();
       int32_t t0, c;
       chunk_span(si, j, t0, c);
-      uint16_t* orow = p.out + (static_cast<int64_t>(si.start + t0) * p.H + h) * kD + v;
       uint32_t a[32], b[32];
       const uint32_t reg = region_col(j);
       tmem_ld32(tmem_addr(tbase, lane_base, reg + 64), a);
@@ -249,18 +253,39 @@ kda_recurrence_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps)
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(&ofree_bar[rg]);
+      if (c == kC) {
+        uint8_t* stile = sm + st * kStage + kWQ;   // O [64 tok][128 v] bf16
+        uint16_t* so = reinterpret_cast<uint16_t*>(stile) + v;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        if (i < c)
-          orow[i * ostride] = __bfloat16_as_ushort(__float2bfloat16_rn(p.scale * __uint_as_float(a[i])));
-      }
+        for (int i = 0; i < 32; ++i) {
+          so[i * kD] = __bfloat16_as_ushort(__float2bfloat16_rn(p.scale * __uint_as_float(a[i])));
+          so[(32 + i) * kD] = __bfloat16_as_ushort(__float2bfloat16_rn(p.scale * __uint_as_float(b[i])));
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(1, kOutThreads);
+        if (leader) {
+          tma_store_3d(&maps.o_out, stile, 0, h, si.start + t0);
+          bulk_commit();
+          bulk_wait_read();
+          mbar_arrive(&empty_bar[st]);
+        }
+      } else {
+        uint16_t* orow = p.out + (static_cast<int64_t>(si.start + t0) * p.H + h) * kD + v;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        if (32 + i < c)
-          orow[(32 + i) * ostride] =
-              __bfloat16_as_ushort(__float2bfloat16_rn(p.scale * __uint_as_float(b[i])));
+        for (int i = 0; i < 32; ++i) {
+          if (i < c)
+            orow[i * ostride] = __bfloat16_as_ushort(__float2bfloat16_rn(p.scale * __uint_as_float(a[i])));
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          if (32 + i < c)
+            orow[(32 + i) * ostride] =
+                __bfloat16_as_ushort(__float2bfloat16_rn(p.scale * __uint_as_float(b[i])));
+        }
+        if (leader) mbar_arrive(&empty_bar[st]);
       }
     }
+    if (leader) bulk_wait_all();   // every tile store of this CTA is complete
     if (!ok) {
       *abort_flag = 1;
       record_status(p.ws, kStatusTimeout);
@@ -302,36 +327,31 @@ kda_recurrence_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps)
     }
     bool ok = true;
     for (int j = 0; j < nch; ++j) {
-      const int st = j & 1;
+      const int st = j % kStages;
       const uint8_t* stg = sm + st * kStage;
-      ok = mbar_wait(&full_bar[st], (j >> 1) & 1, budget) && !*abort_flag;
-      if (ok && j > 0) ok = mbar_wait(&sready_bar, (j - 1) & 1, budget) && !*abort_flag;
+      ok = mbar_wait(&full_bar[st], (j / kStages) & 1, budget) && !*abort_flag;
+      if (ok && j > 0) ok = mbar_wait_spin(&sready_bar, (j - 1) & 1, budget) && !*abort_flag;
       if (!ok) break;
       tc_fence_after();
       // checkpoint: the state after the chunk that ends at the offset
       if (ckc && si.nA > 0 && j == si.nA) store_state(ckc);
-      // (b) S0^T half row -> bf16 A operand, signalled at once so P_W can start;
-      // then the S half row scaled by Gamma_end goes back to TMEM while P_W runs
-      // (the S update that accumulates onto it is issued only after Ud).
+      // (b) S0^T half row -> bf16 A operand in TMEM, signalled at once so P_W can
+      // start; then the S half row scaled by Gamma_end goes back to TMEM while P_W
+      // runs (the S update that accumulates onto it is issued only after Ud).
       {
         const float4* gc4 = reinterpret_cast<const float4*>(stg + kGC) + hw * 16;
         uint32_t a[32], b[32];
         tmem_ld32(tmem_addr(tbase, lane_base, kColS + hw * 64), a);
         tmem_ld32(tmem_addr(tbase, lane_base, kColS + hw * 64 + 32), b);
         tmem_wait_ld();
-        uint8_t* a_panel = sm + kS0T + hw * 16384;
+        uint32_t pk[32];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const uint32_t* src = (q < 4) ? a : b;
-          const int o = (q & 3) * 8;
-          uint4 w;
-          w.x = pack_bf16(__uint_as_float(src[o + 0]), __uint_as_float(src[o + 1]));
-          w.y = pack_bf16(__uint_as_float(src[o + 2]), __uint_as_float(src[o + 3]));
-          w.z = pack_bf16(__uint_as_float(src[o + 4]), __uint_as_float(src[o + 5]));
-          w.w = pack_bf16(__uint_as_float(src[o + 6]), __uint_as_float(src[o + 7]));
-          *reinterpret_cast<uint4*>(a_panel + sw128_offset(v, q)) = w;
+        for (int i = 0; i < 16; ++i) {
+          pk[i] = pack_bf16(__uint_as_float(a[2 * i]), __uint_as_float(a[2 * i + 1]));
+          pk[16 + i] = pack_bf16(__uint_as_float(b[2 * i]), __uint_as_float(b[2 * i + 1]));
         }
-        fence_proxy_async_smem();
+        tmem_st32(tmem_addr(tbase, lane_base, kColS0 + hw * 32), pk);
+        tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&s0_bar);
 #pragma unroll
@@ -350,8 +370,8 @@ kda_recurrence_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps)
         tmem_st32(tmem_addr(tbase, lane_base, kColS + hw * 64 + 32), b);
         tmem_wait_st();
       }
-      // (e) Ud^T = U^T - P_W^T (tokens 32 hw .. 32 hw + 31) -> f16 A operand
-      ok = mbar_wait(&mma1_bar, j & 1, budget) && !*abort_flag;
+      // (e) Ud^T = U^T - P_W^T (tokens 32 hw .. 32 hw + 31) -> f16 A operand in TMEM
+      ok = mbar_wait_spin(&mma1_bar, j & 1, budget) && !*abort_flag;
       if (!ok) break;
       tc_fence_after();
       {
@@ -359,26 +379,25 @@ kda_recurrence_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps)
         tmem_ld32(tmem_addr(tbase, lane_base, region_col(j) + hw * 32), r);
         tmem_wait_ld();
         const uint8_t* ut = stg + kUT;
+        uint32_t ud[16];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const uint4 uq = *reinterpret_cast<const uint4*>(ut + sw128_offset(v, hw * 4 + q));
           const uint32_t uw[4] = {uq.x, uq.y, uq.z, uq.w};
-          uint32_t ow[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const float2 uf = __half22float2(*reinterpret_cast<const __half2*>(&uw[e]));
-            ow[e] = pack_f16(uf.x - __uint_as_float(r[q * 8 + 2 * e]),
-                             uf.y - __uint_as_float(r[q * 8 + 2 * e + 1]));
+            ud[q * 4 + e] = pack_f16(uf.x - __uint_as_float(r[q * 8 + 2 * e]),
+                                     uf.y - __uint_as_float(r[q * 8 + 2 * e + 1]));
           }
-          *reinterpret_cast<uint4*>(sm + kUdT + sw128_offset(v, hw * 4 + q)) =
-              make_uint4(ow[0], ow[1], ow[2], ow[3]);
         }
+        tmem_st16(tmem_addr(tbase, lane_base, kColUd + hw * 16), ud);
+        tmem_wait_st();
       }
-      fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&ud_bar);
     }
-    if (ok && nch > 0) ok = mbar_wait(&sready_bar, (nch - 1) & 1, budget) && !*abort_flag;
+    if (ok && nch > 0) ok = mbar_wait_spin(&sready_bar, (nch - 1) & 1, budget) && !*abort_flag;
     if (!ok) {
       *abort_flag = 1;
       record_status(p.ws, kStatusTimeout);
