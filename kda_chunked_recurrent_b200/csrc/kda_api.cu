@@ -213,10 +213,11 @@ kda_status_t kda_prefill_describe(const kda_shape_t* shape, int has_ckpt,
   const Resolved r = resolve(shape, false, has_ckpt != 0, options);
   snprintf(buf, n,
            "variant=split chunk=%d prepare_items=%lldx%d (persistent, 2 CTAs/SM, 256 threads) "
-           "recurrence_grid=%lldx448 "
+           "recurrence_grid=%lldx%d "
            "workspace_bytes=%zu",
            kC, static_cast<long long>(r.lay.slots), shape->num_heads,
-           static_cast<long long>(shape->num_seqs) * shape->num_heads, r.lay.total);
+           static_cast<long long>(shape->num_seqs) * shape->num_heads, rec::kThreadsPerCta,
+           r.lay.total);
   return KDA_OK;
 }
 

@@ -13,14 +13,15 @@
 // state is S after the chunk that ends at p (h0 for p = 0, the final state for
 // p = len).
 //
-// Serial chain per chunk: S ready -> (state warps) bf16 S0^T into TMEM + decayed S
-// -> [P_W | P_Q] -> (state warps) f16 Ud^T into TMEM -> S update.  S0^T and Ud^T
-// are the A operands of their UMMAs straight from tensor memory, so shared memory
-// only feeds the B tiles.  P_W and P_Q share one N = 128 product (an M = 128 UMMA
-// costs about the same at N = 64 and N = 128); the Ud Aqk output product follows
-// the S update.  [P_W | P_Q/O] alternate between two TMEM regions, so the output
-// warps drain chunk j while chunk j+1 proceeds; the chunk operands stream
-// through a three-stage TMA ring.
+// Serial chain per chunk: S ready -> (state warps) bf16 S0^T into TMEM ->
+// [P_W | P_Q] -> (state warps) f16 Ud^T into TMEM and the decayed S -> S update.
+// S0^T and Ud^T are the A operands of their UMMAs straight from tensor memory,
+// so shared memory only feeds the B tiles.  The state warps and the issuing
+// warp meet at two hardware named barriers per chunk (S0^T ready, Ud^T ready):
+// an mbarrier hand-off between warps costs several hundred cycles inside this
+// kernel, a named barrier a few tens.  [P_W | P_Q/O] alternate between two TMEM
+// regions, so the output warps drain chunk j while chunk j+1 proceeds; the
+// chunk operands stream through a three-stage TMA ring.
 //
 // Tensor memory (512 columns):
 //   [0, 128)    S^T f32 (lane v, column k)
@@ -32,9 +33,11 @@
 //   warps 0-7   state warps: warp w serves TMEM lanes 32 (w % 4) .. + 31 and half
 //               w / 4 of every state row (64 columns; 32 tokens of P_W / Ud);
 //   warps 8-11  output warps: read O^T out of TMEM and store o;
-//   warp 12     lane 0 issues every UMMA;
-//   warp 13     lane 0 streams the operand ring (kept apart from the UMMA
-//               issuer so a stage refill never delays the next chunk's P_W).
+//   warp 12     issues every UMMA (lane 0) after the named barriers;
+//   warp 13     lane 0 streams the operand ring.
+//
+// Every wait is bounded; a failed wait is combined across the participants of
+// the next named barrier (bar.red.or), so all of them leave together.
 //
 // In-place state update (ht == h0) is safe: each thread reads its part of the h0
 // column before writing the same part of ht, and a (sequence, head) pair is
@@ -70,6 +73,8 @@ constexpr int kTmaWarp = kMmaWarp + 1;
 constexpr int kThreads = (kTmaWarp + 1) * 32;
 constexpr uint32_t kStateThreads = kStateWarps * 32;
 constexpr uint32_t kOutThreads = kOutWarps * 32;
+constexpr uint32_t kChainThreads = kStateThreads + 32;   // state warps + the issuing warp
+constexpr uint32_t kBarS0 = 1, kBarUd = 2, kBarOut = 3, kBarOutOr = 4;   // named barriers
 extern const uint32_t kSmemAllocBytes = kSmemAlloc;
 extern const int kThreadsPerCta = kThreads;
 static_assert(kSmemAlloc <= 227 * 1024, "shared memory budget");
@@ -85,7 +90,7 @@ kda_recurrence_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps)
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
   __shared__ uint64_t full_bar[kStages], empty_bar[kStages], oready_bar[kRegions], ofree_bar[kRegions];
-  __shared__ uint64_t s0_bar, ud_bar, mma1_bar, sready_bar;
+  __shared__ uint64_t mma1_bar, sready_bar, drain_bar;
   __shared__ uint32_t tmem_slot;
   __shared__ int32_t s_abort;
   volatile int32_t* abort_flag = &s_abort;
@@ -108,16 +113,15 @@ kda_recurrence_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps)
   if (tid == 0) {
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&full_bar[i], 1);
-      mbar_init(&empty_bar[i], 2);   // the last UMMA commit of the chunk + the output store
+      mbar_init(&empty_bar[i], 2);   // the issuer's last commit of the chunk + the output store
     }
     for (int i = 0; i < kRegions; ++i) {
       mbar_init(&oready_bar[i], 1);
       mbar_init(&ofree_bar[i], kOutThreads);
     }
-    mbar_init(&s0_bar, kStateThreads);
-    mbar_init(&ud_bar, kStateThreads);
     mbar_init(&mma1_bar, 1);
     mbar_init(&sready_bar, 1);
+    mbar_init(&drain_bar, 1);
     s_abort = 0;
     fence_mbar_init();
   }
@@ -175,36 +179,39 @@ kda_recurrence_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps)
     }
   } else if (warp == kMmaWarp) {
     // =========================== UMMA issuer =====================================
-    if ((tid & 31) == 0) {
-      uint64_t* last_commit = nullptr;
-      uint32_t last_parity = 0;
-      const uint32_t id_p = idesc_f16(128, 128, kFmtBF16, kKMajor, kMNMajor);
-      const uint32_t id_s = idesc_f16(128, 128, kFmtF16, kKMajor, kMNMajor);
-      const uint32_t id_o = idesc_f16(128, 64, kFmtF16, kKMajor, kKMajor);
-      const uint32_t tS0 = tbase + kColS0, tUd = tbase + kColUd;
-      bool ok = true;
-      for (int j = 0; j < nch && ok; ++j) {
-        const int st = j % kStages;
-        const int rg = j % kRegions;
-        const uint32_t tP = tbase + region_col(j);
-        const uint32_t bW = smem_u32(sm + st * kStage + kWQ);
-        const uint32_t bKd = smem_u32(sm + st * kStage + kKd);
-        const uint32_t bAq = smem_u32(sm + st * kStage + kAqk);
-        ok = mbar_wait_spin(&s0_bar, j & 1, budget) && !*abort_flag;
+    const bool lead = (tid & 31) == 0;
+    const uint32_t id_p = idesc_f16(128, 128, kFmtBF16, kKMajor, kMNMajor);
+    const uint32_t id_s = idesc_f16(128, 128, kFmtF16, kKMajor, kMNMajor);
+    const uint32_t id_o = idesc_f16(128, 64, kFmtF16, kKMajor, kKMajor);
+    const uint32_t tS0 = tbase + kColS0, tUd = tbase + kColUd;
+    bool ok = true, issued = false;
+    for (int j = 0; j < nch; ++j) {
+      const int st = j % kStages;
+      const int rg = j % kRegions;
+      const uint32_t tP = tbase + region_col(j);
+      const uint32_t bW = smem_u32(sm + st * kStage + kWQ);
+      const uint32_t bKd = smem_u32(sm + st * kStage + kKd);
+      const uint32_t bAq = smem_u32(sm + st * kStage + kAqk);
+      ok = !named_bar_or(kBarS0, kChainThreads, !ok || *abort_flag);   // S0^T is in TMEM
+      if (!ok) break;
+      if (lead) {
         // the output warps must have drained this region (chunk j - 2)
-        if (ok && j >= kRegions)
-          ok = mbar_wait_spin(&ofree_bar[rg], ((j - kRegions) / kRegions) & 1, budget) && !*abort_flag;
-        if (!ok) break;
-        tc_fence_after();
-        // [P_W^T | P_Q^T] = S0^T [W^T | (Q Gamma)^T]
+        if (j >= kRegions)
+          ok = mbar_wait(&ofree_bar[rg], ((j - kRegions) / kRegions) & 1, budget);
+        if (ok) {
+          tc_fence_after();
+          // [P_W^T | P_Q^T] = S0^T [W^T | (Q Gamma)^T]
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_f16_ta(tP, tS0 + kk * 8, sdesc_sw128(bW + kk * 2048, 16384, 1024), id_p, kk > 0);
-        umma_commit(&mma1_bar);
-        last_commit = &mma1_bar;
-        last_parity = j & 1;
-        ok = mbar_wait_spin(&ud_bar, j & 1, budget) && !*abort_flag;
-        if (!ok) break;
+          for (int kk = 0; kk < 8; ++kk)
+            umma_f16_ta(tP, tS0 + kk * 8, sdesc_sw128(bW + kk * 2048, 16384, 1024), id_p, kk > 0);
+          umma_commit(&mma1_bar);
+          issued = true;
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      ok = !named_bar_or(kBarUd, kChainThreads, !ok || *abort_flag);   // Ud^T and decayed S are in TMEM
+      if (!ok) break;
+      if (lead) {
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
@@ -215,15 +222,19 @@ kda_recurrence_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps)
           umma_f16_ta(tP + 64, tUd + kk * 8, sdesc_sw128(bAq + kk * 32, 16, 1024), id_o, 1);
         umma_commit(&oready_bar[rg]);
         umma_commit(&empty_bar[st]);
-        last_commit = &empty_bar[st];
-        last_parity = (j / kStages) & 1;
       }
+      __syncwarp();
+    }
+    if (lead) {
       if (!ok) {
         *abort_flag = 1;
         record_status(p.ws, kStatusTimeout);
       }
-      // drain: every UMMA this thread issued completes before the CTA frees TMEM
-      if (last_commit) mbar_wait(last_commit, last_parity, drain_budget);
+      // drain: every UMMA this warp issued completes before the CTA frees TMEM
+      if (issued) {
+        umma_commit(&drain_bar);
+        mbar_wait(&drain_bar, 0, drain_budget);
+      }
     }
   } else if (warp >= kStateWarps) {
     // =========================== output warps ===================================
@@ -241,7 +252,7 @@ kda_recurrence_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps)
       const int rg = j % kRegions;
       const int st = j % kStages;
       ok = mbar_wait(&oready_bar[rg], (j / kRegions) & 1, budget) && !*abort_flag;
-      ok = !named_bar_or(2, kOutThreads, !ok);   // the same decision in every output thread
+      ok = !named_bar_or(kBarOutOr, kOutThreads, !ok);   // the same decision in every output thread
       if (!ok) break;
       tc_fence_after();
       int32_t t0, c;
@@ -262,7 +273,7 @@ kda_recurrence_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps)
           so[(32 + i) * kD] = __bfloat16_as_ushort(__float2bfloat16_rn(p.scale * __uint_as_float(b[i])));
         }
         fence_proxy_async_smem();
-        named_bar_sync(1, kOutThreads);
+        named_bar_sync(kBarOut, kOutThreads);
         if (leader) {
           tma_store_3d(&maps.o_out, stile, 0, h, si.start + t0);
           bulk_commit();
@@ -329,31 +340,33 @@ kda_recurrence_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps)
     for (int j = 0; j < nch; ++j) {
       const int st = j % kStages;
       const uint8_t* stg = sm + st * kStage;
-      ok = mbar_wait(&full_bar[st], (j / kStages) & 1, budget) && !*abort_flag;
-      if (ok && j > 0) ok = mbar_wait_spin(&sready_bar, (j - 1) & 1, budget) && !*abort_flag;
-      if (!ok) break;
+      ok = ok && mbar_wait(&full_bar[st], (j / kStages) & 1, budget) && !*abort_flag;
+      if (ok && j > 0) ok = mbar_wait(&sready_bar, (j - 1) & 1, budget) && !*abort_flag;
       tc_fence_after();
-      // checkpoint: the state after the chunk that ends at the offset
-      if (ckc && si.nA > 0 && j == si.nA) store_state(ckc);
-      // (b) S0^T half row -> bf16 A operand in TMEM, signalled at once so P_W can
-      // start; then the S half row scaled by Gamma_end goes back to TMEM while P_W
-      // runs (the S update that accumulates onto it is issued only after Ud).
-      {
-        const float4* gc4 = reinterpret_cast<const float4*>(stg + kGC) + hw * 16;
-        uint32_t a[32], b[32];
+      uint32_t a[32], b[32];
+      if (ok) {
+        // checkpoint: the state after the chunk that ends at the offset
+        if (ckc && si.nA > 0 && j == si.nA) store_state(ckc);
+        // (b) S0^T half row -> bf16 A operand in TMEM
         tmem_ld32(tmem_addr(tbase, lane_base, kColS + hw * 64), a);
         tmem_ld32(tmem_addr(tbase, lane_base, kColS + hw * 64 + 32), b);
         tmem_wait_ld();
-        uint32_t pk[32];
+        uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          pk[i] = pack_bf16(__uint_as_float(a[2 * i]), __uint_as_float(a[2 * i + 1]));
-          pk[16 + i] = pack_bf16(__uint_as_float(b[2 * i]), __uint_as_float(b[2 * i + 1]));
-        }
-        tmem_st32(tmem_addr(tbase, lane_base, kColS0 + hw * 32), pk);
+        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(__uint_as_float(a[2 * i]), __uint_as_float(a[2 * i + 1]));
+        tmem_st16(tmem_addr(tbase, lane_base, kColS0 + hw * 32), pk);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(__uint_as_float(b[2 * i]), __uint_as_float(b[2 * i + 1]));
+        tmem_st16(tmem_addr(tbase, lane_base, kColS0 + hw * 32 + 16), pk);
         tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(&s0_bar);
+      }
+      tc_fence_before();
+      ok = !named_bar_or(kBarS0, kChainThreads, !ok);
+      if (!ok) break;
+      // the S half row scaled by Gamma_end goes back to TMEM while [P_W | P_Q]
+      // runs (the update that accumulates onto it is issued after the next barrier)
+      {
+        const float4* gc4 = reinterpret_cast<const float4*>(stg + kGC) + hw * 16;
 #pragma unroll
         for (int i4 = 0; i4 < 8; ++i4) {
           const float4 ga = gc4[i4], gb = gc4[8 + i4];
@@ -368,13 +381,11 @@ kda_recurrence_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps)
         }
         tmem_st32(tmem_addr(tbase, lane_base, kColS + hw * 64), a);
         tmem_st32(tmem_addr(tbase, lane_base, kColS + hw * 64 + 32), b);
-        tmem_wait_st();
       }
       // (e) Ud^T = U^T - P_W^T (tokens 32 hw .. 32 hw + 31) -> f16 A operand in TMEM
-      ok = mbar_wait_spin(&mma1_bar, j & 1, budget) && !*abort_flag;
-      if (!ok) break;
+      ok = mbar_wait(&mma1_bar, j & 1, budget) && !*abort_flag;
       tc_fence_after();
-      {
+      if (ok) {
         uint32_t r[32];
         tmem_ld32(tmem_addr(tbase, lane_base, region_col(j) + hw * 32), r);
         tmem_wait_ld();
@@ -392,12 +403,13 @@ kda_recurrence_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps)
           }
         }
         tmem_st16(tmem_addr(tbase, lane_base, kColUd + hw * 16), ud);
-        tmem_wait_st();
       }
+      tmem_wait_st();   // Ud^T and the decayed S row are in TMEM
       tc_fence_before();
-      mbar_arrive(&ud_bar);
+      ok = !named_bar_or(kBarUd, kChainThreads, !ok);
+      if (!ok) break;
     }
-    if (ok && nch > 0) ok = mbar_wait_spin(&sready_bar, (nch - 1) & 1, budget) && !*abort_flag;
+    if (ok && nch > 0) ok = mbar_wait(&sready_bar, (nch - 1) & 1, budget) && !*abort_flag;
     if (!ok) {
       *abort_flag = 1;
       record_status(p.ws, kStatusTimeout);
