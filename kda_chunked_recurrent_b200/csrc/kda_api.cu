@@ -309,7 +309,7 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
     mok &= make_map_rows(&maps.g_in, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, g, T, H, 4);
     mok &= make_map_rows(&maps.o_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, out, T, H, 2);
     mok &= make_map_2d(&maps.wt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ws + r.lay.wt, 64, recs * 128, 64, 128, 2);
-    mok &= make_map_2d(&maps.qgt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ws + r.lay.qgt, 64, recs * 128, 64, 128, 2);
+    mok &= make_map_2d(&maps.qg, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ws + r.lay.qg, 128, recs * 64, 64, 64, 2);
     mok &= make_map_2d(&maps.ut, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws + r.lay.ut, 64, recs * 128, 64, 128, 2);
     mok &= make_map_2d(&maps.kd, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws + r.lay.kd, 128, recs * 64, 64, 64, 2);
     mok &= make_map_2d(&maps.aqk, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws + r.lay.aqk, 64, recs * 64, 64, 64, 2);

@@ -34,7 +34,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 // A "record" is one (chunk slot, head) pair: rec = slot * H + h.
 constexpr size_t kHeaderBytes = 1024;
 constexpr size_t kTileWT = 128 * 64 * 2;   // W^T   [128 k][64 tok] bf16
-constexpr size_t kTileQGT = 128 * 64 * 2;  // (Q*Gamma)^T [128 k][64 tok] bf16
+constexpr size_t kTileQG = 64 * 128 * 2;   // Q*Gamma [64 tok][128 k] bf16 (token rows)
 constexpr size_t kTileUT = 128 * 64 * 2;   // U^T   [128 v][64 tok] f16
 constexpr size_t kTileKd = 64 * 128 * 2;   // Kd    [64 tok][128 k] f16 (token rows)
 constexpr size_t kTileAqk = 64 * 64 * 2;   // Aqk   [64 r][64 s]  f16
@@ -43,7 +43,7 @@ constexpr size_t kTileGC = 128 * 4;        // Gamma at the chunk end, f32 [128]
 struct WorkspaceLayout {
   size_t chunk_base;   // int32 [N+1]   first slot of each sequence
   size_t seq_order;    // int32 [N]     longest-first order of sequences
-  size_t wt, qgt, ut, kd, aqk, gc;    // per-record tiles (split variant)
+  size_t wt, qg, ut, kd, aqk, gc;     // per-record tiles (split variant)
   size_t total;
   int64_t slots;       // chunk slots (upper bound on the number of chunks)
 };
@@ -70,7 +70,7 @@ inline WorkspaceLayout make_layout(int64_t N, int64_t T, int64_t H, bool fixed, 
   L.slots = (N > 0 && T > 0) ? chunk_slots(N, T, fixed, ckpt) : 0;
   const size_t recs = split ? static_cast<size_t>(L.slots * H) : 0;
   L.wt = off;  off = align_up(off + recs * kTileWT, 1024);
-  L.qgt = off; off = align_up(off + recs * kTileQGT, 1024);
+  L.qg = off;  off = align_up(off + recs * kTileQG, 1024);
   L.ut = off;  off = align_up(off + recs * kTileUT, 1024);
   L.kd = off;  off = align_up(off + recs * kTileKd, 1024);
   L.aqk = off; off = align_up(off + recs * kTileAqk, 1024);
@@ -121,7 +121,7 @@ struct SplitMaps {
   CUtensorMap g_in;     // g [T][H][128] f32, box (128 ch, 1 head, 64 tok), no swizzle
   CUtensorMap o_out;    // out [T][H][128] bf16, box (128 ch, 1 head, 64 tok), no swizzle
   CUtensorMap wt;       // [recs*128][64] bf16, box (64, 128)
-  CUtensorMap qgt;      // [recs*128][64] bf16, box (64, 128)
+  CUtensorMap qg;       // [recs*64][128] bf16, box (64, 64): one 64-channel panel
   CUtensorMap ut;       // [recs*128][64] f16, box (64, 128)
   CUtensorMap kd;       // [recs*64][128] f16, box (64, 64)
   CUtensorMap aqk;      // [recs*64][64] f16, box (64, 64)

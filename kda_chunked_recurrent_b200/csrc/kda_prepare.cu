@@ -6,10 +6,9 @@
 // writes the per-chunk operands the recurrence kernel consumes:
 //   W^T [128 k][64 tok] bf16, U^T [128 v][64 tok] f16, Aqk [64][64] f16
 //   (UMMA results, staged in shared memory and written by TMA tile stores),
-//   (Q*Gamma)^T [128 k][64 tok] bf16 (transposed in registers, staged in the v
-//   region before v arrives, TMA tile store),
-//   Kd [64 tok][128 k] f16 (token rows, written straight from the element-wise
-//   pass with 128-byte warp stores), Gamma_end [128] f32.
+//   Q*Gamma [64 tok][128 k] bf16, Kd [64 tok][128 k] f16 (token rows, written
+//   straight from the element-wise pass with 128-byte warp stores),
+//   Gamma_end [128] f32.
 // A checkpoint offset p inside a sequence is a chunk boundary of the schedule
 // (the chunks cover [0, p) and [p, len) separately), so the checkpoint state is
 // the state after a chunk and needs no extra operands here.
@@ -21,8 +20,7 @@
 // Inputs of a chunk: q, k (bf16) and g (f32) arrive by TMA as whole [64 tok][128 ch]
 // tiles into shared memory the previous chunk no longer needs (issued as soon as
 // that chunk's second UMMA has completed, with the rows already prefetched into
-// L2 one chunk earlier); v follows by TMA straight into its UMMA operand layout
-// once the (Q*Gamma)^T staging tile in that region has been stored.
+// L2 one chunk earlier); v follows by TMA straight into its UMMA operand layout.
 //
 // Thread mapping for the element-wise part: thread t owns the channel pair
 // (2p, 2p+1), p = t % 64, in sub-block b = t / 64 (tokens 16b .. 16b+15), so a
@@ -68,9 +66,6 @@ constexpr uint32_t kBytes = 65536 + 40960;
 constexpr uint32_t kQraw = kV;                  // q [64 tok][128 ch] bf16
 constexpr uint32_t kKraw = kKG;                 // k [64 tok][128 ch] bf16
 constexpr uint32_t kGraw = kR;                  // g [64 tok][128 ch] f32 (32 KB)
-// (Q*Gamma)^T staging [128 k][64 tok] bf16, 128B swizzle, between the raw q tile
-// and the v tile in the same region
-constexpr uint32_t kQGs = kV;
 constexpr uint32_t kRawTx = 16384 + 16384 + 32768;
 // aliases of [K+; Q+] once the first UMMA has completed: the solve scratch, and
 // after the solve the staging tiles of the W^T / U^T TMA stores
@@ -282,7 +277,6 @@ kda_prepare_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps) {
     prefetch_tmap(&maps.k_in);
     prefetch_tmap(&maps.g_in);
     prefetch_tmap(&maps.wt);
-    prefetch_tmap(&maps.qgt);
     prefetch_tmap(&maps.ut);
     prefetch_tmap(&maps.aqk);
   }
@@ -385,6 +379,15 @@ kda_prepare_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps) {
     if (tid == 0) bulk_wait_read();
     ok = !__syncthreads_or(!ok);
     if (!ok) break;
+    // ---- TMA: v tile straight into the MN-major A operand of U^T (the raw q tile
+    // in that region has been read by every thread)
+    if (tid == 0) {
+      mbar_arrive_expect_tx(&tma_bar, 16384);
+      tma_load_3d(sm + kV, &maps.v_in, &tma_bar, 0, h, t0);
+      tma_load_3d(sm + kV + 8192, &maps.v_in, &tma_bar, 64, h, t0);
+    }
+    const uint32_t tma_parity = static_cast<uint32_t>(tma_issued & 1);
+    ++tma_issued;
     float2 Bs[4];   // B_i: G at the first token of sub-block i
     float2 E;       // G at the chunk end
     {
@@ -429,8 +432,8 @@ kda_prepare_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps) {
       const uint32_t cB2 = pack_bf16(cB.x, cB.y);
       const uint32_t c1b = pack_bf16(c1.x, c1.y), c2b = pack_bf16(c2.x, c2.y),
                      c3b = pack_bf16(c3.x, c3.y);
-      // Kd token rows: this thread's channel pair of rows 16 blk + i
-      uint32_t qg[16];
+      // Q Gamma and Kd token rows: this thread's channel pair of rows 16 blk + i
+      uint32_t* qg_out = reinterpret_cast<uint32_t*>(p.ws + p.lay.qg + rec * kTileQG) + blk * 16 * 64 + cp;
       uint32_t* kd_out = reinterpret_cast<uint32_t*>(p.ws + p.lay.kd + rec * kTileKd) + blk * 16 * 64 + cp;
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
@@ -449,7 +452,7 @@ kda_prepare_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps) {
         if (blk < 3) sts32(bR + xo + 96u * 128u, hmul2_bf16(rd2, c3b));
         const uint32_t gm2 = hmul2_bf16(e2, cB2);
         sts32(bKG + xo, hmul2_bf16(kw[i], gm2));
-        qg[i] = hmul2_bf16(qw[i], gm2);
+        qg_out[i * 64] = hmul2_bf16(qw[i], gm2);
         // Kd feeds the FP16 state update: FP32 products, one rounding
         const float2 kf = bf2_to_f2(kw[i]);
         kd_out[i * 64] = pack_f16(kf.x * i0 * cE.x, kf.y * i1 * cE.y);
@@ -457,21 +460,6 @@ kda_prepare_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps) {
       if (blk == 0)
         reinterpret_cast<float2*>(p.ws + p.lay.gc + rec * kTileGC)[cp] =
             make_float2(ex2(E.x), ex2(E.y));
-      // (Q Gamma)^T rows 2 cp and 2 cp + 1, tokens 16 blk .. 16 blk + 15 (two 16-byte chunks each)
-      uint32_t lo[8], hi[8];
-#pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        lo[m] = __byte_perm(qg[2 * m], qg[2 * m + 1], 0x5410);
-        hi[m] = __byte_perm(qg[2 * m], qg[2 * m + 1], 0x7632);
-      }
-      uint8_t* qs = sm + kQGs;
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        *reinterpret_cast<uint4*>(qs + sw128_offset(2 * cp, 2 * blk + hh)) =
-            make_uint4(lo[4 * hh], lo[4 * hh + 1], lo[4 * hh + 2], lo[4 * hh + 3]);
-        *reinterpret_cast<uint4*>(qs + sw128_offset(2 * cp + 1, 2 * blk + hh)) =
-            make_uint4(hi[4 * hh], hi[4 * hh + 1], hi[4 * hh + 2], hi[4 * hh + 3]);
-      }
     }
     if (tid < kC) s_beta[tid] = bf16_to_f32(beta_raw);
 
@@ -490,16 +478,7 @@ kda_prepare_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps) {
         umma_f16(tbase, ad, bd, idesc, kk > 0);
       }
       umma_commit(&mma_bar);
-      // (Q Gamma)^T out; once its staging tile has been read, v takes the region
-      tma_store_2d(&maps.qgt, sm + kQGs, 0, static_cast<int32_t>(rec * 128));
-      bulk_commit();
-      bulk_wait_read();
-      mbar_arrive_expect_tx(&tma_bar, 16384);
-      tma_load_3d(sm + kV, &maps.v_in, &tma_bar, 0, h, t0);
-      tma_load_3d(sm + kV + 8192, &maps.v_in, &tma_bar, 64, h, t0);
     }
-    const uint32_t tma_parity = static_cast<uint32_t>(tma_issued & 1);
-    ++tma_issued;
     ++mma_commits;
     ok = mbar_wait(&mma_bar, static_cast<uint32_t>((mma_commits - 1) & 1), budget);
     ok = !__syncthreads_or(!ok);

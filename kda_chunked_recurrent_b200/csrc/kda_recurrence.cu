@@ -5,7 +5,8 @@
 // in TMEM/registers across chunks via tcgen05 GEMMs fed by TMA" and (c) "an
 // output kernel fusing the intra-chunk causal term with q.S").  The state is
 // kept transposed, S^T[v][k], in TMEM lanes v = 0..127, so every UMMA has M = 128:
-//   [P_W^T | P_Q^T] = S0^T [W^T | (Q Gamma)^T]  (N=128, K=128; bf16; MN-major B)
+//   P_W^T = S0^T W^T                            (N=64, K=128; bf16; B = W^T, MN-major)
+//   P_Q^T = S0^T (Q Gamma)^T                    (N=64, K=128; bf16; B = Q Gamma rows, K-major)
 //   Ud^T  = U^T - P_W^T                         (threads; f16 operand)
 //   S^T   = S0^T Diag(Gamma_end) + Ud^T Kd      (N=128, K=64; f16; B = Kd rows, MN-major)
 //   O^T   = scale (P_Q^T + Ud^T Aqk^T)          (N=64, K=64; f16)
@@ -13,8 +14,9 @@
 // state is S after the chunk that ends at p (h0 for p = 0, the final state for
 // p = len).
 //
-// Serial chain per chunk: S ready -> (state warps) bf16 S0^T into TMEM ->
-// [P_W | P_Q] -> (state warps) f16 Ud^T into TMEM and the decayed S -> S update.
+// Serial chain per chunk: S ready -> (state warps) bf16 S0^T into TMEM -> P_W
+// -> (state warps) f16 Ud^T into TMEM and the decayed S -> S update.  P_Q is
+// issued right behind P_W and runs while the state warps form Ud.
 // S0^T and Ud^T are the A operands of their UMMAs straight from tensor memory,
 // so shared memory only feeds the B tiles.  The state warps and the issuing
 // warp meet at two hardware named barriers per chunk (S0^T ready, Ud^T ready):
@@ -26,7 +28,7 @@
 // Tensor memory (512 columns):
 //   [0, 128)    S^T f32 (lane v, column k)
 //   [128, 384)  two regions: P_W^T (64 columns) then P_Q^T / O^T (64 columns)
-//   [384, 448)  S0^T bf16, two k per column (A operand of [P_W | P_Q])
+//   [384, 448)  S0^T bf16, two k per column (A operand of P_W and P_Q)
 //   [448, 480)  Ud^T f16, two tokens per column (A operand of the update and O)
 //
 // Warp roles:
@@ -52,7 +54,8 @@
 namespace kda {
 
 namespace rec {
-constexpr uint32_t kWQ = 0;          // 32 KB [W^T | (Q Gamma)^T], MN-major B, 2 panels [128 k][64 tok]
+constexpr uint32_t kWQ = 0;          // 16 KB W^T [128 k][64 tok] bf16, MN-major B;
+                                     // 16 KB Q Gamma [64 tok][128 k] bf16, K-major B, 2 panels
 constexpr uint32_t kUT = 32768;      // 16 KB U^T  [128 v][64 tok] f16 (128B swizzle)
 constexpr uint32_t kKd = 49152;      // 16 KB Kd [64 tok][128 k] f16, MN-major B, 2 panels
 constexpr uint32_t kAqk = 65536;     //  8 KB Aqk  [64 r][64 s] f16, K-major B
@@ -145,7 +148,8 @@ kda_recurrence_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps)
         uint8_t* base = sm + st * kStage;
         mbar_arrive_expect_tx(&full_bar[st], kStageTx);
         tma_load_2d(base + kWQ, &maps.wt, &full_bar[st], 0, recr * 128);
-        tma_load_2d(base + kWQ + 16384, &maps.qgt, &full_bar[st], 0, recr * 128);
+        tma_load_2d(base + kWQ + 16384, &maps.qg, &full_bar[st], 0, recr * 64);
+        tma_load_2d(base + kWQ + 16384 + 8192, &maps.qg, &full_bar[st], 64, recr * 64);
         tma_load_2d(base + kUT, &maps.ut, &full_bar[st], 0, recr * 128);
         tma_load_2d(base + kKd, &maps.kd, &full_bar[st], 0, recr * 64);
         tma_load_2d(base + kKd + 8192, &maps.kd, &full_bar[st], 64, recr * 64);
@@ -156,7 +160,7 @@ kda_recurrence_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps)
       };
       if (nch > 0) {
         prefetch_tmap(&maps.wt);
-        prefetch_tmap(&maps.qgt);
+        prefetch_tmap(&maps.qg);
         prefetch_tmap(&maps.ut);
         prefetch_tmap(&maps.kd);
         prefetch_tmap(&maps.aqk);
@@ -180,7 +184,8 @@ kda_recurrence_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps)
   } else if (warp == kMmaWarp) {
     // =========================== UMMA issuer =====================================
     const bool lead = (tid & 31) == 0;
-    const uint32_t id_p = idesc_f16(128, 128, kFmtBF16, kKMajor, kMNMajor);
+    const uint32_t id_p = idesc_f16(128, 64, kFmtBF16, kKMajor, kMNMajor);
+    const uint32_t id_q = idesc_f16(128, 64, kFmtBF16, kKMajor, kKMajor);
     const uint32_t id_s = idesc_f16(128, 128, kFmtF16, kKMajor, kMNMajor);
     const uint32_t id_o = idesc_f16(128, 64, kFmtF16, kKMajor, kKMajor);
     const uint32_t tS0 = tbase + kColS0, tUd = tbase + kColUd;
@@ -200,12 +205,17 @@ kda_recurrence_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps)
           ok = mbar_wait(&ofree_bar[rg], ((j - kRegions) / kRegions) & 1, budget);
         if (ok) {
           tc_fence_after();
-          // [P_W^T | P_Q^T] = S0^T [W^T | (Q Gamma)^T]
+          // P_W^T = S0^T W^T (the chain needs it), then P_Q^T = S0^T (Q Gamma)^T
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             umma_f16_ta(tP, tS0 + kk * 8, sdesc_sw128(bW + kk * 2048, 16384, 1024), id_p, kk > 0);
           umma_commit(&mma1_bar);
           issued = true;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            umma_f16_ta(tP + 64, tS0 + kk * 8,
+                        sdesc_sw128(bW + 16384 + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id_q,
+                        kk > 0);
         }
       }
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
