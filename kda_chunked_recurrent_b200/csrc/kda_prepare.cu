@@ -220,14 +220,21 @@ struct PrepItem {
   int64_t slot, rec;
 };
 __device__ __forceinline__ bool locate_item(const KdaParams& p, int64_t w, PrepItem& it) {
-  it.slot = w / p.H;
-  it.h = static_cast<int32_t>(w % p.H);
+  if (w < 0x7fffffff) {   // 32-bit divisions (every realistic grid)
+    const uint32_t w32 = static_cast<uint32_t>(w), H = static_cast<uint32_t>(p.H);
+    it.slot = w32 / H;
+    it.h = static_cast<int32_t>(w32 - static_cast<uint32_t>(it.slot) * H);
+  } else {
+    it.slot = w / p.H;
+    it.h = static_cast<int32_t>(w % p.H);
+  }
   if (it.slot >= p.slots) return false;
   int32_t n = 0, j = 0;
   if (p.cu_seqlens == nullptr && p.ckpt_offsets == nullptr) {
-    const int32_t cps = (p.fixed_len + kC - 1) / kC;
-    n = static_cast<int32_t>(it.slot / cps);
-    j = static_cast<int32_t>(it.slot % cps);
+    const uint32_t cps = static_cast<uint32_t>((p.fixed_len + kC - 1) / kC);
+    const uint32_t s32 = static_cast<uint32_t>(it.slot);   // slot < slots < 2^31 here
+    n = static_cast<int32_t>(s32 / cps);
+    j = static_cast<int32_t>(s32 - static_cast<uint32_t>(n) * cps);
   } else {
     const int32_t* cb = reinterpret_cast<const int32_t*>(p.ws + p.lay.chunk_base);
     if (it.slot >= cb[p.N]) return false;
@@ -324,17 +331,14 @@ kda_prepare_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps) {
     uint16_t beta_raw = 0;   // consumed only after the operand pass, so its latency hides
     if (tid < c) beta_raw = p.beta[static_cast<int64_t>(t0 + tid) * p.H + h];
 
-    // ---- L2 prefetch of the next item's rows (q, k, v: 256 B, g: 512 B per token; beta)
+    // ---- L2 prefetch of the next item's tiles (q, k, g, v) and beta rows
     if (nxt_valid) {
-      const int which = tid >> 6, r = tid & 63;
-      if (r < nxt.c) {
-        const int64_t row = (static_cast<int64_t>(nxt.t0) + r) * p.H + nxt.h;
-        if (which == 0) bulk_prefetch_l2(p.q + row * kD, 256);
-        else if (which == 1) bulk_prefetch_l2(p.k + row * kD, 256);
-        else if (which == 2) bulk_prefetch_l2(p.v + row * kD, 256);
-        else bulk_prefetch_l2(p.g + row * kD, 512);
-      }
       if (tid == 0) {
+        tma_prefetch_3d(&maps.q_in, 0, nxt.h, nxt.t0);
+        tma_prefetch_3d(&maps.k_in, 0, nxt.h, nxt.t0);
+        tma_prefetch_3d(&maps.g_in, 0, nxt.h, nxt.t0);
+        tma_prefetch_3d(&maps.v_in, 0, nxt.h, nxt.t0);
+        tma_prefetch_3d(&maps.v_in, 64, nxt.h, nxt.t0);
         // beta rows of the next chunk, all heads: 16-byte aligned and inside the tensor
         const uintptr_t lo =
             reinterpret_cast<uintptr_t>(p.beta + static_cast<int64_t>(nxt.t0) * p.H) & ~uintptr_t(15);
