@@ -306,6 +306,8 @@ def main():
     shape = capi.make_shape(N, T, H, max(lens))
     opts = {"variant": args.variant}
     ws = K.Workspace(capi.kda_prefill_workspace_size(shape, cko is not None, opts), dev)
+    desc = capi.kda_prefill_describe(shape, cko is not None, opts)
+    variant = "fused" if "variant=fused" in desc else "split"
     stream = torch.cuda.current_stream(dev)
     P = lambda t: None if t is None else t.data_ptr()
 
@@ -319,8 +321,10 @@ def main():
         if rc != 0:
             raise K.KDAError(rc)
 
-    # schedule (packed layout or checkpoints), prepare, recurrence
-    launches_per_step = (0 if fixed and cko is None else 1) + (1 if T > 0 else 0) + 1
+    # schedule (packed layout or checkpoints), then prepare + recurrence (split) or
+    # the single cooperative launch (fused)
+    launches_per_step = (0 if fixed and cko is None else 1) + \
+        (1 if variant == "fused" else (1 if T > 0 else 0) + 1)
     in_bytes = sum(x.numel() * x.element_size() for x in (q, k, v, g, beta))
     flush = None
     if in_bytes < 2 * L2_BYTES:
@@ -375,12 +379,23 @@ def main():
     # ---- roofline of the dominant kernel
     peaks, peak_src = load_peaks()
     state_io = N * H * STATE_BYTES * ((1 if h0 is not None else 0) + 1 + (1 if ck is not None else 0))
-    kernels = {
-        "kda_prepare_kernel": (prep_ms, PREP_BYTES_PER_TOKHEAD * units,
-                               ["kda_prepare.cu", "kda_common.cuh", "sm100_primitives.cuh"]),
-        "kda_recurrence_kernel": (rec_ms, REC_BYTES_PER_TOKHEAD * units + state_io,
-                                  ["kda_recurrence.cu", "kda_common.cuh", "sm100_primitives.cuh"]),
-    }
+    if variant == "fused":
+        # one launch moves both halves' bytes (the records still go through HBM/L2)
+        kernels = {
+            "kda_fused_kernel": (prep_ms + rec_ms,
+                                 (PREP_BYTES_PER_TOKHEAD + REC_BYTES_PER_TOKHEAD) * units + state_io,
+                                 ["kda_fused.cu", "kda_prepare.cuh", "kda_recurrence.cuh",
+                                  "kda_common.cuh", "sm100_primitives.cuh"]),
+        }
+    else:
+        kernels = {
+            "kda_prepare_kernel": (prep_ms, PREP_BYTES_PER_TOKHEAD * units,
+                                   ["kda_prepare.cu", "kda_prepare.cuh", "kda_common.cuh",
+                                    "sm100_primitives.cuh"]),
+            "kda_recurrence_kernel": (rec_ms, REC_BYTES_PER_TOKHEAD * units + state_io,
+                                      ["kda_recurrence.cu", "kda_recurrence.cuh", "kda_common.cuh",
+                                       "sm100_primitives.cuh"]),
+        }
     dom = max(kernels, key=lambda n: kernels[n][0])
     dms, dbytes, _ = kernels[dom]
     achieved = dbytes / (dms / 1e3) / 1e9
@@ -448,7 +463,7 @@ def main():
                 "config": {"workload": args.workload, "num_seqs": N, "seq_lens": "x".join(
                     map(str, sorted(set(lens)))) if len(set(lens)) < 4 else "ragged",
                     "total_tokens": T, "heads": H, "head_dim": 128, "h0": h0 is not None,
-                    "checkpoint": ck is not None, "variant": "split", "chunk": 64,
+                    "checkpoint": ck is not None, "variant": variant, "chunk": 64,
                     "parallelism": f"dp{world}" if world > 1 else "single",
                     "l2": ("inputs (%.2f GB) larger than L2, no flush" % (in_bytes / 1e9))
                     if flush is None else

@@ -6,7 +6,8 @@
 // PR #5050 "Motivation"; partial h0/ht overlap rejected, FlashInfer PR #4262
 // "Physical schedules and true in-place state update").  Device metadata
 // (cu_seqlens, ckpt_offsets) is never read on the host.  Launch order on the
-// caller's stream: [schedule] -> prepare -> recurrence.
+// caller's stream: [schedule] -> prepare -> recurrence (split variant), or
+// [schedule] -> ready-flag clear -> one cooperative launch (fused variant).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -22,8 +23,11 @@ namespace kda {
 __global__ void kda_schedule_kernel(const KdaParams p);
 __global__ void kda_prepare_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps);
 __global__ void kda_recurrence_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps);
+__global__ void kda_fused_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps,
+                                 int32_t rec_ctas, int64_t prep_items);
 namespace prep { extern const uint32_t kSmemAllocBytes; }
 namespace rec { extern const uint32_t kSmemAllocBytes; extern const int kThreadsPerCta; }
+namespace fused { extern const uint32_t kSmemAllocBytes; extern const int kThreadsPerCta; }
 }  // namespace kda
 
 using namespace kda;
@@ -75,7 +79,6 @@ kda_status_t check_options(const kda_options_t* o) {
   if (o->variant < KDA_VARIANT_AUTO || o->variant > KDA_VARIANT_FUSED) return KDA_ERR_BAD_OPTION;
   if (o->flags & ~(static_cast<uint32_t>(KDA_FLAG_VALIDATE | KDA_FLAG_TEST_FORCE_TIMEOUT)))
     return KDA_ERR_BAD_OPTION;
-  if (o->variant == KDA_VARIANT_FUSED) return KDA_ERR_BAD_OPTION;  // not available yet
   return KDA_OK;
 }
 
@@ -92,10 +95,57 @@ kda_status_t check_shape(const kda_shape_t* s, bool fixed, bool ckpt) {
   return KDA_OK;
 }
 
+int sm_count();
+
+// The fused launch keeps at least this many SMs for its prepare CTAs.
+constexpr int kFusedMinPrepCtas = 16;
+
+// Per-shape variant table, from CUDA-event timings on one B200 (1965 MHz, ms per
+// call, split / fused): B1 T8192 H12 (12 chains of 128 chunks) 0.296 / 0.256;
+// B1 T512 H12 (12 chains of 8 chunks) 0.041 / 0.044; B4 T8192 H12 (48 chains)
+// 0.487 / 0.547; B6 T8192 H12 (72) 0.551 / 0.989; B8 T1024 and B8 T8192 H12
+// (96) 0.110 / 0.268 and 0.651 / 1.897.  The fused launch hides the prepare
+// work behind the recurrence chains only when few chains (one SM each) leave
+// most SMs to its prepare CTAs and the sequences are long enough to overlap.
+struct VariantRule {
+  int64_t max_chains;   // N H at most this
+  int64_t min_chunks;   // and at least this many chunks in the longest sequence
+  int variant;          // -> this variant
+};
+constexpr VariantRule kVariantTable[] = {
+    {16, 32, KDA_VARIANT_FUSED},
+    {INT64_MAX, 0, KDA_VARIANT_SPLIT},
+};
+
+bool fused_eligible(const kda_shape_t* s) {
+  const int64_t chains = static_cast<int64_t>(s->num_seqs) * s->num_heads;
+  return chains + kFusedMinPrepCtas <= sm_count();
+}
+
+int64_t max_chunks_per_seq(const kda_shape_t* s, bool fixed, bool ckpt);
+
+int choose_variant(const kda_shape_t* s, const kda_options_t* o) {
+  if (o && o->variant != KDA_VARIANT_AUTO) return o->variant;
+  const int64_t chains = static_cast<int64_t>(s->num_seqs) * s->num_heads;
+  const int64_t chunks = max_chunks_per_seq(s, false, false);
+  for (const VariantRule& rule : kVariantTable)
+    if (chains <= rule.max_chains && chunks >= rule.min_chunks) {
+      if (rule.variant == KDA_VARIANT_FUSED && !fused_eligible(s)) continue;
+      return rule.variant;
+    }
+  return KDA_VARIANT_SPLIT;
+}
+
+// Upper bound on the chunks of one sequence (the fused launch's chunk-major items).
+int64_t max_chunks_per_seq(const kda_shape_t* s, bool fixed, bool ckpt) {
+  int64_t L = fixed ? s->total_tokens / s->num_seqs
+                    : (s->max_seqlen > 0 ? s->max_seqlen : s->total_tokens);
+  return (L + kC - 1) / kC + (ckpt ? 1 : 0);
+}
+
 Resolved resolve(const kda_shape_t* s, bool fixed, bool ckpt, const kda_options_t* o) {
   Resolved r{};
-  r.variant = KDA_VARIANT_SPLIT;
-  (void)o;
+  r.variant = choose_variant(s, o);
   r.fixed = fixed;
   r.lay = make_layout(s->num_seqs, s->total_tokens, s->num_heads, fixed, true, ckpt);
   return r;
@@ -211,13 +261,21 @@ kda_status_t kda_prefill_describe(const kda_shape_t* shape, int has_ckpt,
     return st;
   }
   const Resolved r = resolve(shape, false, has_ckpt != 0, options);
-  snprintf(buf, n,
-           "variant=split chunk=%d prepare_items=%lldx%d (persistent, 2 CTAs/SM, 256 threads) "
-           "recurrence_grid=%lldx%d "
-           "workspace_bytes=%zu",
-           kC, static_cast<long long>(r.lay.slots), shape->num_heads,
-           static_cast<long long>(shape->num_seqs) * shape->num_heads, rec::kThreadsPerCta,
-           r.lay.total);
+  const long long chains = static_cast<long long>(shape->num_seqs) * shape->num_heads;
+  if (r.variant == KDA_VARIANT_FUSED) {
+    snprintf(buf, n,
+             "variant=fused chunk=%d grid=%dx%d (recurrence CTAs %lld, prepare CTAs %lld, "
+             "cooperative) workspace_bytes=%zu",
+             kC, sm_count(), fused::kThreadsPerCta, chains,
+             static_cast<long long>(sm_count()) - chains, r.lay.total);
+  } else {
+    snprintf(buf, n,
+             "variant=split chunk=%d prepare_items=%lldx%d (persistent, 2 CTAs/SM, 256 threads) "
+             "recurrence_grid=%lldx%d "
+             "workspace_bytes=%zu",
+             kC, static_cast<long long>(r.lay.slots), shape->num_heads, chains,
+             rec::kThreadsPerCta, r.lay.total);
+  }
   return KDA_OK;
 }
 
@@ -265,6 +323,8 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
   const Resolved r = resolve(shape, fixed, ckpt, options);
   const size_t need = kda_prefill_workspace_size(shape, ckpt ? 1 : 0, options);
   if (workspace_bytes < need || workspace_bytes < r.lay.total) return KDA_ERR_WORKSPACE_TOO_SMALL;
+  // the fused launch needs an SM per chain plus SMs for its prepare CTAs
+  if (r.variant == KDA_VARIANT_FUSED && !fused_eligible(shape)) return KDA_ERR_BAD_OPTION;
 
   // ---------------- device
   st = device_check();
@@ -327,7 +387,10 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
     cudaError_t e2 = cudaFuncSetAttribute(kda_recurrence_kernel,
                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           rec::kSmemAllocBytes);
-    attr_err = (e1 != cudaSuccess) ? e1 : e2;
+    cudaError_t e3 = cudaFuncSetAttribute(kda_fused_kernel,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          fused::kSmemAllocBytes);
+    attr_err = (e1 != cudaSuccess) ? e1 : (e2 != cudaSuccess ? e2 : e3);
   });
   if (attr_err != cudaSuccess) return KDA_ERR_LAUNCH_FAILED;
   (void)cudaGetLastError();
@@ -339,16 +402,41 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
     kda_schedule_kernel<<<1, 1024, 0, s>>>(p);
     mark(0);
   }
-  if (T > 0) {
-    // persistent prepare grid: two CTAs per SM walk the (chunk slot, head) items
-    const int64_t items = r.lay.slots * H;
-    const int64_t grid = std::min<int64_t>(items, 2 * static_cast<int64_t>(sm_count()));
-    kda_prepare_kernel<<<static_cast<unsigned>(grid), 256, prep::kSmemAllocBytes, s>>>(p, maps);
+  if (r.variant == KDA_VARIANT_FUSED) {
+    // one cooperative launch: CTAs 0 .. N H - 1 run the recurrences, the rest of
+    // the SMs (one CTA each) prepare the chunk records in chunk-major order
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kda_fused_kernel,
+                                                      fused::kThreadsPerCta,
+                                                      fused::kSmemAllocBytes) != cudaSuccess ||
+        per_sm < 1)
+      return KDA_ERR_LAUNCH_FAILED;
+    int32_t rec_ctas = static_cast<int32_t>(N * H);
+    const int grid = sm_count();   // one CTA per SM (checked above: chains + 16 <= SMs)
+    int64_t prep_items = max_chunks_per_seq(shape, fixed, ckpt) * static_cast<int64_t>(rec_ctas);
+    if (r.lay.slots > 0 &&
+        cudaMemsetAsync(ws + r.lay.ready, 0, static_cast<size_t>(r.lay.slots) * H * sizeof(int32_t),
+                        s) != cudaSuccess)
+      return KDA_ERR_LAUNCH_FAILED;
+    void* args[] = {&p, &maps, &rec_ctas, &prep_items};
+    if (cudaLaunchCooperativeKernel(reinterpret_cast<void*>(kda_fused_kernel), dim3(grid),
+                                    dim3(fused::kThreadsPerCta), args, fused::kSmemAllocBytes,
+                                    s) != cudaSuccess)
+      return KDA_ERR_LAUNCH_FAILED;
+    mark(1);
+    mark(2);
+  } else {
+    if (T > 0) {
+      // persistent prepare grid: two CTAs per SM walk the (chunk slot, head) items
+      const int64_t items = r.lay.slots * H;
+      const int64_t grid = std::min<int64_t>(items, 2 * static_cast<int64_t>(sm_count()));
+      kda_prepare_kernel<<<static_cast<unsigned>(grid), 256, prep::kSmemAllocBytes, s>>>(p, maps);
+    }
+    mark(1);
+    kda_recurrence_kernel<<<static_cast<unsigned>(N * H), rec::kThreadsPerCta,
+                            rec::kSmemAllocBytes, s>>>(p, maps);
+    mark(2);
   }
-  mark(1);
-  kda_recurrence_kernel<<<static_cast<unsigned>(N * H), rec::kThreadsPerCta, rec::kSmemAllocBytes, s>>>(
-      p, maps);
-  mark(2);
   if (cudaGetLastError() != cudaSuccess) return KDA_ERR_LAUNCH_FAILED;
   return KDA_OK;
 }

@@ -43,7 +43,8 @@ constexpr size_t kTileGC = 128 * 4;        // Gamma at the chunk end, f32 [128]
 struct WorkspaceLayout {
   size_t chunk_base;   // int32 [N+1]   first slot of each sequence
   size_t seq_order;    // int32 [N]     longest-first order of sequences
-  size_t wt, qg, ut, kd, aqk, gc;     // per-record tiles (split variant)
+  size_t wt, qg, ut, kd, aqk, gc;     // per-record tiles
+  size_t ready;        // int32 [recs]  per-record ready flags (fused variant)
   size_t total;
   int64_t slots;       // chunk slots (upper bound on the number of chunks)
 };
@@ -75,6 +76,7 @@ inline WorkspaceLayout make_layout(int64_t N, int64_t T, int64_t H, bool fixed, 
   L.kd = off;  off = align_up(off + recs * kTileKd, 1024);
   L.aqk = off; off = align_up(off + recs * kTileAqk, 1024);
   L.gc = off;  off = align_up(off + recs * kTileGC, 1024);
+  L.ready = off; off = align_up(off + recs * sizeof(int32_t), 1024);
   L.total = off;
   return L;
 }

@@ -1,0 +1,779 @@
+// kda_prepare.cuh — chunk-local prepare (body shared by the split prepare kernel
+// and the prepare CTAs of the fused launch).
+//
+// A persistent grid (two CTAs of 256 threads per SM in the split variant) walks
+// the records (chunk slot, head).  For each 64-token chunk it forms the decay-weighted
+// intra-chunk products, solves the unit-lower-triangular UT/WY system and
+// writes the per-chunk operands the recurrence kernel consumes:
+//   W^T [128 k][64 tok] bf16, U^T [128 v][64 tok] f16, Aqk [64][64] f16
+//   (UMMA results, staged in shared memory and written by TMA tile stores),
+//   Q*Gamma [64 tok][128 k] bf16, Kd [64 tok][128 k] f16 (token rows, written
+//   straight from the element-wise pass with 128-byte warp stores),
+//   Gamma_end [128] f32.
+// A checkpoint offset p inside a sequence is a chunk boundary of the schedule
+// (the chunks cover [0, p) and [p, len) separately), so the checkpoint state is
+// the state after a chunk and needs no extra operands here.
+// (north star subsystem (a): "a chunk-local prepare kernel that forms the
+// decay-weighted intra-chunk products, solves the unit-lower-triangular UT/WY
+// system per chunk and emits W and U"; the split into prepare and recurrence
+// launches is the "decomp" variant of FlashInfer PR #4633 "Description").
+//
+// Inputs of a chunk: q, k (bf16) and g (f32) arrive by TMA as whole [64 tok][128 ch]
+// tiles into shared memory the previous chunk no longer needs (issued as soon as
+// that chunk's second UMMA has completed, with the rows already prefetched into
+// L2 one chunk earlier); v follows by TMA straight into its UMMA operand layout.
+//
+// Thread mapping for the element-wise part: thread t owns the channel pair
+// (2p, 2p+1), p = t % 64, in sub-block b = t / 64 (tokens 16b .. 16b+15), so a
+// warp writes one full 128-byte row of one operand per store.
+//
+// Decay factorisation (log2 domain, G = cumsum(g * log2 e), B_b = G at the
+// first token of sub-block b, E = G at the chunk end):
+//   e_r   = 2^(G_r - B_b)   in [2^-116, 1]        inv_r = 2^(B_b - G_r) in [1, 2^116]
+//   K+_r  = k_r e_r,  Q+_r = q_r e_r              (left operand, row r / 64 + r)
+//   R^i_r = k_r inv_r 2^(B_i - B_b)  for i >= b   (right operand, segment i)
+//   Gamma_r = e_r 2^(B_b),  Kd_r = k_r inv_r 2^(E - B_b)
+// so the only per-element MUFU work is e_r and inv_r.  When 2^(B_i - B_b) or
+// 2^(E - B_b) underflows, the exact product is below 2^-18 (|G_r - B_b| <= 116),
+// an absolute error far under the BF16/FP16 rounding of the operands.
+//   A[r, s] = K+_r . R^{b(r)}_s for every s in sub-blocks 0..b(r): inside one
+// sub-block the exponents cancel (|.| <= 80 nats); before it both factors are
+// <= 1.  One UMMA of M = 128 ([K+; Q+]) by N = 160 (R^0..R^3, 16+32+48+64 rows)
+// yields A (strict lower part) and Aqk (lower part with the diagonal).
+//
+// UT solve: T = (I + M)^-1 with M = diag(beta) A_strict, in 16x16 blocks.  The
+// diagonal blocks X_ii are inverted in FP32 by forward substitution; then
+// Z_ik = -X_ii M_ik for all i > k in one step, and the off-diagonal blocks
+// follow level by level, X_ij = sum_{k=j}^{i-1} Z_ik X_kj, as FP16 mma.sync
+// products with FP32 accumulation.  Each block of T diag(beta), the B operand
+// of the W/U UMMA, is written from the accumulator as soon as it is final.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "kda_common.cuh"
+#include "sm100_primitives.cuh"
+
+namespace kda {
+
+namespace prep {
+constexpr int kThreads = 256;
+constexpr uint32_t kV = 0;           // 16 KB  v tile, MN-major A of U^T: 2 panels [64 tok][64 v]
+constexpr uint32_t kKG = 16384;      // 16 KB  K*Gamma tile, MN-major A of W^T
+constexpr uint32_t kL = 32768;       // 32 KB  [K+; Q+], K-major A: 2 panels [128 rows][64 ch]
+constexpr uint32_t kR = 65536;       // 40 KB  R^0..R^3, K-major B: 2 panels [160 rows][64 ch]
+constexpr uint32_t kBytes = 65536 + 40960;
+// raw input tiles of a chunk, landed before its element-wise pass (which reads
+// them into registers before anything overwrites these regions)
+constexpr uint32_t kQraw = kV;                  // q [64 tok][128 ch] bf16
+constexpr uint32_t kKraw = kKG;                 // k [64 tok][128 ch] bf16
+constexpr uint32_t kGraw = kR;                  // g [64 tok][128 ch] f32 (32 KB)
+constexpr uint32_t kRawTx = 16384 + 16384 + 32768;
+// aliases of [K+; Q+] once the first UMMA has completed: the solve scratch, and
+// after the solve the staging tiles of the W^T / U^T TMA stores
+constexpr int kLdh = 72;
+constexpr uint32_t kMf = kL;                    // f32 [4][16][17] diagonal blocks of M
+constexpr uint32_t kMh = kMf + 4 * 16 * 17 * 4; // f16 [64][72] off-diagonal blocks of M
+constexpr uint32_t kXh = kMh + 64 * kLdh * 2;   // f16 [64][72] T = (I + M)^-1
+constexpr uint32_t kZh = kXh + 64 * kLdh * 2;   // f16 [64][72] Z_ik = -X_ii M_ik
+constexpr uint32_t kWs = kL;                    // W^T staging [128 k][64 tok] bf16, 128B swizzle
+constexpr uint32_t kUs = kL + 16384;            // U^T staging [128 v][64 tok] f16, 128B swizzle
+// aliases of R once the first UMMA has completed
+constexpr uint32_t kAqs = kR;                   // Aqk staging [64 r][64 s] f16, 128B swizzle
+constexpr uint32_t kTb = 98304;                 // 8 KB T diag(beta) bf16, K-major [64 r][64 s]
+constexpr uint32_t kSmemAlloc = kBytes + 1024;
+static_assert(kZh + 64 * kLdh * 2 <= kR, "solve scratch overlaps the Aqk staging tile");
+static_assert(kAqs + 8192 <= kTb, "Aqk staging overlaps the Tb tile");
+static_assert(kUs + 16384 <= kR, "W/U staging overlaps R");
+}  // namespace prep
+
+// Packed bf16x2 product (round to nearest even), for operands that are rounded
+// to bf16 for the tensor core anyway.
+__device__ __forceinline__ uint32_t hmul2_bf16(uint32_t a, uint32_t b) {
+  __nv_bfloat162 r = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&a),
+                             *reinterpret_cast<const __nv_bfloat162*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+
+__device__ __forceinline__ void sts32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ float2 bf2_to_f2(uint32_t u) {
+  return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.x4.m8n8.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.x4.trans.m8n8.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+// D(16x8, f32) += A(16x16, f16, row) * B(16x8, f16, col)
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// (c0 | c1) += A * B for 16x16 blocks of two row-major [64][72] f16 arrays:
+// A at (ar, ac) of the array at shared address aA, B at (br, bc) of aB.
+__device__ __forceinline__ void mma_block(float (&c0)[4], float (&c1)[4], uint32_t aA, int ar,
+                                          int ac, uint32_t aB, int br, int bc, int lane) {
+  using prep::kLdh;
+  uint32_t a[4], b[4];
+  ldsm_x4(aA + ((ar + (lane & 15)) * kLdh + ac + (lane >> 4) * 8) * 2, a);
+  ldsm_x4_t(aB + ((br + (lane & 7) + ((lane >> 3) & 1) * 8) * kLdh + bc + (lane >> 4) * 8) * 2, b);
+  mma16816(c0, a, b[0], b[1]);
+  mma16816(c1, a, b[2], b[3]);
+}
+
+// Store a 16x16 f32 accumulator pair (two m16n8 fragments) as f16 into a
+// row-major tile (row stride `ld` halves), multiplied by `s`.
+__device__ __forceinline__ void store_frag16(__half* base, int ld, const float (&c0)[4],
+                                             const float (&c1)[4], float s, int lane) {
+  const int g = lane >> 2, q = lane & 3;
+  *reinterpret_cast<__half2*>(base + g * ld + 2 * q) = __floats2half2_rn(s * c0[0], s * c0[1]);
+  *reinterpret_cast<__half2*>(base + (g + 8) * ld + 2 * q) = __floats2half2_rn(s * c0[2], s * c0[3]);
+  *reinterpret_cast<__half2*>(base + g * ld + 8 + 2 * q) = __floats2half2_rn(s * c1[0], s * c1[1]);
+  *reinterpret_cast<__half2*>(base + (g + 8) * ld + 8 + 2 * q) =
+      __floats2half2_rn(s * c1[2], s * c1[3]);
+}
+
+// Store the same 16x16 block of T, scaled by beta of its column, as bf16 into the
+// 128B-swizzled K-major Tb tile (rows r0.., columns c0..).
+__device__ __forceinline__ void store_tb16(uint32_t tb, const float* beta, int r0, int c0,
+                                           const float (&x0)[4], const float (&x1)[4], int lane) {
+  const int g = lane >> 2, q = lane & 3;
+  {
+    const int s = c0 + 2 * q;
+    const float b0 = beta[s], b1 = beta[s + 1];
+    const uint32_t off = static_cast<uint32_t>((s & 7) * 2);
+    sts32(tb + sw128_offset(r0 + g, s >> 3) + off, pack_bf16(x0[0] * b0, x0[1] * b1));
+    sts32(tb + sw128_offset(r0 + g + 8, s >> 3) + off, pack_bf16(x0[2] * b0, x0[3] * b1));
+  }
+  {
+    const int s = c0 + 8 + 2 * q;
+    const float b0 = beta[s], b1 = beta[s + 1];
+    const uint32_t off = static_cast<uint32_t>((s & 7) * 2);
+    sts32(tb + sw128_offset(r0 + g, s >> 3) + off, pack_bf16(x1[0] * b0, x1[1] * b1));
+    sts32(tb + sw128_offset(r0 + g + 8, s >> 3) + off, pack_bf16(x1[2] * b0, x1[3] * b1));
+  }
+}
+
+// Write one row of the first UMMA's result.  Row rl lies in sub-block BL and
+// `val[s]` holds its products with the right-operand segment of that sub-block
+// (s = 0 .. 16 BL + 15).  Key rows feed M = diag(beta) A_strict (diagonal block in
+// FP32, earlier blocks in FP16); query rows are Aqk (s <= rl), written as FP16
+// into the swizzled staging tile of its TMA store.
+template <int BL>
+__device__ __forceinline__ void emit_rows(const uint32_t* val, bool is_q, int rl, float br,
+                                          uint8_t* sm) {
+  using namespace prep;
+  constexpr int NV = 16 * (BL + 1);
+  if (!is_q) {
+    float* Mf = reinterpret_cast<float*>(sm + kMf) + BL * (16 * 17) + (rl & 15) * 17;
+#pragma unroll
+    for (int s = 16 * BL; s < 16 * BL + 16; ++s)
+      Mf[s & 15] = (s < rl) ? br * __uint_as_float(val[s]) : 0.f;
+    __half* Mh = reinterpret_cast<__half*>(sm + kMh) + rl * kLdh;
+#pragma unroll
+    for (int s0 = 0; s0 < 16 * BL; s0 += 8) {
+      uint32_t pk[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        pk[u] = pack_f16(br * __uint_as_float(val[s0 + 2 * u]),
+                         br * __uint_as_float(val[s0 + 2 * u + 1]));
+      *reinterpret_cast<uint4*>(Mh + s0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    }
+  } else {
+#pragma unroll
+    for (int s0 = 0; s0 < kC; s0 += 8) {
+      uint32_t pk[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int s = s0 + 2 * u;
+        const float a = (s < NV && s <= rl) ? __uint_as_float(val[s < NV ? s : 0]) : 0.f;
+        const float b2 = (s + 1 < NV && s + 1 <= rl) ? __uint_as_float(val[s + 1 < NV ? s + 1 : 0]) : 0.f;
+        pk[u] = pack_f16(a, b2);
+      }
+      *reinterpret_cast<uint4*>(sm + kAqs + sw128_offset(rl, s0 >> 3)) =
+          make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    }
+  }
+}
+
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
+// Work item w of the persistent grid: chunk slot w / H, head w % H.  Returns
+// false when the slot holds no chunk (past the end of the chunk table).
+struct PrepItem {
+  int32_t h, c, t0;
+  int64_t slot, rec;
+};
+__device__ __forceinline__ bool locate_item(const KdaParams& p, int64_t w, PrepItem& it) {
+  if (w < 0x7fffffff) {   // 32-bit divisions (every realistic grid)
+    const uint32_t w32 = static_cast<uint32_t>(w), H = static_cast<uint32_t>(p.H);
+    it.slot = w32 / H;
+    it.h = static_cast<int32_t>(w32 - static_cast<uint32_t>(it.slot) * H);
+  } else {
+    it.slot = w / p.H;
+    it.h = static_cast<int32_t>(w % p.H);
+  }
+  if (it.slot >= p.slots) return false;
+  int32_t n = 0, j = 0;
+  if (p.cu_seqlens == nullptr && p.ckpt_offsets == nullptr) {
+    const uint32_t cps = static_cast<uint32_t>((p.fixed_len + kC - 1) / kC);
+    const uint32_t s32 = static_cast<uint32_t>(it.slot);   // slot < slots < 2^31 here
+    n = static_cast<int32_t>(s32 / cps);
+    j = static_cast<int32_t>(s32 - static_cast<uint32_t>(n) * cps);
+  } else {
+    const int32_t* cb = reinterpret_cast<const int32_t*>(p.ws + p.lay.chunk_base);
+    if (it.slot >= cb[p.N]) return false;
+    int32_t lo = 0, hi = p.N;  // largest n with cb[n] <= slot
+    while (hi - lo > 1) {
+      const int32_t mid = (lo + hi) >> 1;
+      if (cb[mid] <= it.slot) lo = mid; else hi = mid;
+    }
+    n = lo;
+    j = static_cast<int32_t>(it.slot - cb[n]);
+  }
+  if (n >= p.N) return false;
+  const SeqInfo si = seq_info(p, n, false);
+  if (j >= si.nch) return false;
+  chunk_span(si, j, it.t0, it.c);
+  it.t0 += si.start;
+  it.rec = it.slot * p.H + it.h;
+  return it.c > 0;
+}
+
+// Work item w in chunk-major order, used when prepare CTAs feed recurrence CTAs
+// of the same launch: chunk j = w / R of chain c = w % R (R = N H chains, in the
+// recurrence grid's order), so every chain's chunk j is prepared before any
+// chain's chunk j + 1.
+__device__ __forceinline__ bool locate_item_chunk_major(const KdaParams& p, int64_t w, PrepItem& it) {
+  const int64_t R = static_cast<int64_t>(p.N) * p.H;
+  const int64_t j = w / R, c = w - (w / R) * R;
+  int32_t n = static_cast<int32_t>(c / p.H);
+  it.h = static_cast<int32_t>(c - static_cast<int64_t>(n) * p.H);
+  if (p.cu_seqlens != nullptr) n = reinterpret_cast<const int32_t*>(p.ws + p.lay.seq_order)[n];
+  if (n < 0 || n >= p.N) return false;
+  const SeqInfo si = seq_info(p, n);
+  if (j >= si.nch) return false;
+  it.slot = si.slot0 + j;
+  if (it.slot < 0 || it.slot >= p.slots) return false;
+  chunk_span(si, static_cast<int32_t>(j), it.t0, it.c);
+  it.t0 += si.start;
+  it.rec = it.slot * p.H + it.h;
+  return it.c > 0;
+}
+
+// CTA-wide barriers of the prepare body: the whole CTA in the split kernel, the
+// first 256 threads (named barrier 1) in a prepare CTA of the fused launch.
+template <bool kFused>
+__device__ __forceinline__ void prep_sync() {
+  if constexpr (kFused) named_bar_sync(1, prep::kThreads); else __syncthreads();
+}
+template <bool kFused>
+__device__ __forceinline__ bool prep_sync_or(bool pred) {
+  if constexpr (kFused) return named_bar_or(1, prep::kThreads, pred);
+  else return __syncthreads_or(pred) != 0;
+}
+
+// Publish a finished record to the recurrence CTAs of the fused launch: its tile
+// stores (issued by this thread) are complete and every thread's plain stores
+// were ordered before the last CTA barrier.
+__device__ __forceinline__ void publish_record(const KdaParams& p, int64_t rec) {
+  bulk_wait_all();
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  int32_t* flag = reinterpret_cast<int32_t*>(p.ws + p.lay.ready) + rec;
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(flag), "r"(1) : "memory");
+}
+
+// The prepare loop.  Items first, first + stride, ... < nitems; kFused selects the
+// chunk-major item order, the 256-thread barriers and the ready flags.
+template <bool kFused>
+__device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps& maps,
+                                             uint8_t* smem_raw, int64_t first, int64_t stride,
+                                             int64_t nitems) {
+  using namespace prep;
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~static_cast<uintptr_t>(1023));
+  __shared__ uint64_t tma_bar, mma_bar, raw_bar;
+  __shared__ uint32_t tmem_slot;
+  __shared__ float s_beta[kC];
+  __shared__ float2 s_tot[4][64];     // per sub-block sums of g (log2 domain), channel pairs
+  __shared__ float2 s_first[4][64];   // running sum at the first token of the sub-block
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  if ((p.flags & kFlagValidate) && reinterpret_cast<const WsHeader*>(p.ws)->call_ok == 0) return;
+  const long long budget = p.wait_budget;
+  const long long drain_budget = 4000000000LL;
+  auto locate = [&](int64_t w, PrepItem& it) {
+    if constexpr (kFused) return locate_item_chunk_major(p, w, it);
+    else return locate_item(p, w, it);
+  };
+
+  if (tid == 0) {
+    mbar_init(&tma_bar, 1);
+    mbar_init(&mma_bar, 1);
+    mbar_init(&raw_bar, 1);
+    fence_mbar_init();
+    prefetch_tmap(&maps.v_in);
+    prefetch_tmap(&maps.q_in);
+    prefetch_tmap(&maps.k_in);
+    prefetch_tmap(&maps.g_in);
+    prefetch_tmap(&maps.wt);
+    prefetch_tmap(&maps.ut);
+    prefetch_tmap(&maps.aqk);
+  }
+  if (warp == 0) {
+    tmem_alloc(&tmem_slot, 256);
+    tmem_relinquish();
+  }
+  prep_sync<kFused>();
+  tc_fence_after();
+  const uint32_t tbase = tmem_slot;
+  const uint32_t sbase = smem_u32(sm);
+  bool ok = true;
+  int mma_commits = 0;     // UMMA commits issued so far (their mbarrier phases)
+  int tma_issued = 0;      // v tiles issued so far (tma_bar phases)
+  int raw_issued = 0;      // raw q/k/g tile sets issued so far (raw_bar phases)
+  bool raw_for_cur = false;  // the current item's raw tiles are already in flight
+  auto issue_raw = [&](const PrepItem& it) {  // thread 0 only
+    mbar_arrive_expect_tx(&raw_bar, kRawTx);
+    tma_load_3d(sm + kQraw, &maps.q_in, &raw_bar, 0, it.h, it.t0);
+    tma_load_3d(sm + kKraw, &maps.k_in, &raw_bar, 0, it.h, it.t0);
+    tma_load_3d(sm + kGraw, &maps.g_in, &raw_bar, 0, it.h, it.t0);
+  };
+
+  PrepItem cur;
+  bool cur_valid = first < nitems && locate(first, cur);
+  int64_t pending = -1;   // fused launch: record whose ready flag is still to be raised
+  for (int64_t w = first; w < nitems && ok; w += stride) {
+    PrepItem nxt;
+    const bool nxt_valid = (w + stride < nitems) && locate(w + stride, nxt);
+    if (!cur_valid) {
+      cur = nxt;
+      cur_valid = nxt_valid;
+      continue;
+    }
+    const int h = cur.h;
+    const int32_t t0 = cur.t0, c = cur.c;
+    const int64_t rec = cur.rec;
+
+    const int cp = tid & 63;         // channel pair
+    const int blk = tid >> 6;        // sub-block 0..3
+    if (!raw_for_cur) {
+      if (tid == 0) issue_raw(cur);
+      ++raw_issued;
+    }
+    raw_for_cur = false;
+    if constexpr (kFused) {
+      if (tid == 0 && pending >= 0) publish_record(p, pending);
+      pending = -1;
+    }
+    uint16_t beta_raw = 0;   // consumed only after the operand pass, so its latency hides
+    if (tid < c) beta_raw = p.beta[static_cast<int64_t>(t0 + tid) * p.H + h];
+
+    // ---- L2 prefetch of the next item's tiles (q, k, g, v) and beta rows
+    if (nxt_valid) {
+      if (tid == 0) {
+        tma_prefetch_3d(&maps.q_in, 0, nxt.h, nxt.t0);
+        tma_prefetch_3d(&maps.k_in, 0, nxt.h, nxt.t0);
+        tma_prefetch_3d(&maps.g_in, 0, nxt.h, nxt.t0);
+        tma_prefetch_3d(&maps.v_in, 0, nxt.h, nxt.t0);
+        tma_prefetch_3d(&maps.v_in, 64, nxt.h, nxt.t0);
+        // beta rows of the next chunk, all heads: 16-byte aligned and inside the tensor
+        const uintptr_t lo =
+            reinterpret_cast<uintptr_t>(p.beta + static_cast<int64_t>(nxt.t0) * p.H) & ~uintptr_t(15);
+        uintptr_t hi = (reinterpret_cast<uintptr_t>(p.beta + static_cast<int64_t>(nxt.t0 + nxt.c) * p.H) + 15) &
+                       ~uintptr_t(15);
+        const uintptr_t lim =
+            reinterpret_cast<uintptr_t>(p.beta + static_cast<int64_t>(p.T) * p.H) & ~uintptr_t(15);
+        hi = hi < lim ? hi : lim;
+        if (hi > lo) bulk_prefetch_l2(reinterpret_cast<const void*>(lo), static_cast<uint32_t>(hi - lo));
+      }
+    }
+
+    // ---- raw tiles -> registers: g (float2), k, q (bf16x2) for 16 tokens x 2 channels
+    ok = mbar_wait(&raw_bar, static_cast<uint32_t>((raw_issued - 1) & 1), budget);
+    float2 G[16];
+    uint32_t kw[16], qw[16];
+    {
+      const float2* gs = reinterpret_cast<const float2*>(sm + kGraw) + blk * 16 * 64 + cp;
+      const uint32_t* ks = reinterpret_cast<const uint32_t*>(sm + kKraw) + blk * 16 * 64 + cp;
+      const uint32_t* qs = reinterpret_cast<const uint32_t*>(sm + kQraw) + blk * 16 * 64 + cp;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const bool in = ok && blk * 16 + i < c;   // rows past the chunk read as zero
+        G[i] = in ? gs[i * 64] : make_float2(0.f, 0.f);
+        kw[i] = in ? ks[i * 64] : 0u;
+        qw[i] = in ? qs[i * 64] : 0u;
+      }
+    }
+    // ---- gate scan within the sub-block; one exchange gives every sub-block start
+    {
+      float2 run = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        run.x = fmaf(G[i].x, kLog2e, run.x);
+        run.y = fmaf(G[i].y, kLog2e, run.y);
+        G[i] = run;
+      }
+      s_first[blk][cp] = G[0];
+      s_tot[blk][cp] = run;
+    }
+    // the previous item's TMA stores have finished reading their staging tiles
+    if (tid == 0) bulk_wait_read();
+    ok = !prep_sync_or<kFused>(!ok);
+    if (!ok) break;
+    // ---- TMA: v tile straight into the MN-major A operand of U^T (the raw q tile
+    // in that region has been read by every thread)
+    if (tid == 0) {
+      mbar_arrive_expect_tx(&tma_bar, 16384);
+      tma_load_3d(sm + kV, &maps.v_in, &tma_bar, 0, h, t0);
+      tma_load_3d(sm + kV + 8192, &maps.v_in, &tma_bar, 64, h, t0);
+    }
+    const uint32_t tma_parity = static_cast<uint32_t>(tma_issued & 1);
+    ++tma_issued;
+    float2 Bs[4];   // B_i: G at the first token of sub-block i
+    float2 E;       // G at the chunk end
+    {
+      float2 acc = make_float2(0.f, 0.f), pre = acc;
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const float2 f = s_first[b][cp], t = s_tot[b][cp];
+        Bs[b] = make_float2(acc.x + f.x, acc.y + f.y);
+        if (b == blk) pre = acc;
+        acc.x += t.x;
+        acc.y += t.y;
+      }
+      E = acc;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        G[i].x += pre.x;
+        G[i].y += pre.y;
+      }
+    }
+
+    // ---- operands
+    {
+      const float2 B = G[0];
+      const float2 cB = make_float2(ex2(B.x), ex2(B.y));                    // 2^B_b
+      const float2 cE = make_float2(ex2(E.x - B.x), ex2(E.y - B.y));        // 2^(E - B_b)
+      // 2^(B_i - B_b) for the later sub-blocks i = 1, 2, 3 (unused entries never read)
+      float2 c1 = make_float2(0.f, 0.f), c2 = c1, c3 = c1;
+      if (blk < 1) c1 = make_float2(ex2(Bs[1].x - B.x), ex2(Bs[1].y - B.y));
+      if (blk < 2) c2 = make_float2(ex2(Bs[2].x - B.x), ex2(Bs[2].y - B.y));
+      if (blk < 3) c3 = make_float2(ex2(Bs[3].x - B.x), ex2(Bs[3].y - B.y));
+      const int seg_own = (blk == 0) ? 0 : (blk == 1) ? 16 : (blk == 2) ? 48 : 96;
+      // Store addresses.  Row r = 16 blk + i has (r & 7) == (i & 7), so the 128-byte
+      // swizzle of every operand row reduces to a per-thread base plus one of eight
+      // per-thread XOR terms and a compile-time row offset.
+      const uint32_t panel = static_cast<uint32_t>(cp >> 5);
+      const uint32_t chunk = static_cast<uint32_t>((cp & 31) >> 2);
+      const uint32_t inner = static_cast<uint32_t>((cp & 3) * 4 + blk * 2048);
+      const uint32_t bL = sbase + kL + panel * 16384u + inner;
+      const uint32_t bR = sbase + kR + panel * 20480u + inner;
+      const uint32_t bRo = bR + static_cast<uint32_t>(seg_own) * 128u;
+      const uint32_t bKG = sbase + kKG + panel * 8192u + inner;
+      const uint32_t cB2 = pack_bf16(cB.x, cB.y);
+      const uint32_t c1b = pack_bf16(c1.x, c1.y), c2b = pack_bf16(c2.x, c2.y),
+                     c3b = pack_bf16(c3.x, c3.y);
+      // Q Gamma and Kd token rows: this thread's channel pair of rows 16 blk + i
+      uint32_t* qg_out = reinterpret_cast<uint32_t*>(p.ws + p.lay.qg + rec * kTileQG) + blk * 16 * 64 + cp;
+      uint32_t* kd_out = reinterpret_cast<uint32_t*>(p.ws + p.lay.kd + rec * kTileKd) + blk * 16 * 64 + cp;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const uint32_t xo = ((chunk ^ static_cast<uint32_t>(i & 7)) << 4) + static_cast<uint32_t>(i) * 128u;
+        const float2 g2 = G[i];
+        const float e0 = ex2(g2.x - B.x), e1 = ex2(g2.y - B.y);
+        const float i0 = ex2(B.x - g2.x), i1 = ex2(B.y - g2.y);
+        // bf16 operands: factors rounded to bf16, products in packed bf16 math
+        const uint32_t e2 = pack_bf16(e0, e1), inv2 = pack_bf16(i0, i1);
+        sts32(bL + xo, hmul2_bf16(kw[i], e2));
+        sts32(bL + xo + 64u * 128u, hmul2_bf16(qw[i], e2));
+        const uint32_t rd2 = hmul2_bf16(kw[i], inv2);
+        sts32(bRo + xo, rd2);
+        if (blk < 1) sts32(bR + xo + 16u * 128u, hmul2_bf16(rd2, c1b));
+        if (blk < 2) sts32(bR + xo + 48u * 128u, hmul2_bf16(rd2, c2b));
+        if (blk < 3) sts32(bR + xo + 96u * 128u, hmul2_bf16(rd2, c3b));
+        const uint32_t gm2 = hmul2_bf16(e2, cB2);
+        sts32(bKG + xo, hmul2_bf16(kw[i], gm2));
+        qg_out[i * 64] = hmul2_bf16(qw[i], gm2);
+        // Kd feeds the FP16 state update: FP32 products, one rounding
+        const float2 kf = bf2_to_f2(kw[i]);
+        kd_out[i * 64] = pack_f16(kf.x * i0 * cE.x, kf.y * i1 * cE.y);
+      }
+      if (blk == 0)
+        reinterpret_cast<float2*>(p.ws + p.lay.gc + rec * kTileGC)[cp] =
+            make_float2(ex2(E.x), ex2(E.y));
+    }
+    if (tid < kC) s_beta[tid] = bf16_to_f32(beta_raw);
+
+    // ---- UMMA 1: D[0:128, 0:160] = [K+; Q+] . R^T   (bf16 -> f32)
+    fence_proxy_async_smem();
+    tc_fence_before();
+    prep_sync<kFused>();
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t idesc = idesc_f16(128, 160, kFmtBF16, kKMajor, kKMajor);
+      const uint32_t aL = sbase + kL, aR = sbase + kR;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint64_t ad = sdesc_sw128(aL + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+        const uint64_t bd = sdesc_sw128(aR + (kk >> 2) * 20480 + (kk & 3) * 32, 16, 1024);
+        umma_f16(tbase, ad, bd, idesc, kk > 0);
+      }
+      umma_commit(&mma_bar);
+    }
+    ++mma_commits;
+    ok = mbar_wait(&mma_bar, static_cast<uint32_t>((mma_commits - 1) & 1), budget);
+    ok = !prep_sync_or<kFused>(!ok);
+    if (ok) {
+      tc_fence_after();
+      // ---- extract A (lane quarters 0,1) and Aqk (quarters 2,3): row rl, sub-block bl.
+      // Warps w and w + 4 share a lane quarter; warp w reads the column segment of
+      // the first sub-block its rows hold, warp w + 4 that of the second, so at most
+      // 64 accumulator values are live per thread and all eight warps take part.
+      const int qw4 = warp & 3, phase = warp >> 2;
+      const int rl = (qw4 & 1) * 32 + lane;
+      const int bl = rl >> 4;
+      const bool is_q = qw4 >= 2;
+      const uint32_t lane_base = static_cast<uint32_t>(qw4 * 32);
+      const float br = s_beta[rl];
+      if ((qw4 & 1) == 0) {
+        if (phase == 0) {
+          uint32_t v[16];
+          tmem_ld16(tmem_addr(tbase, lane_base, 0), v);
+          tmem_wait_ld();
+          if (bl == 0) emit_rows<0>(v, is_q, rl, br, sm);
+        } else {
+          uint32_t v[32];
+          tmem_ld32(tmem_addr(tbase, lane_base, 16), v);
+          tmem_wait_ld();
+          if (bl == 1) emit_rows<1>(v, is_q, rl, br, sm);
+        }
+      } else {
+        if (phase == 0) {
+          uint32_t v[48], t32[32], t16[16];
+          tmem_ld32(tmem_addr(tbase, lane_base, 48), t32);
+          tmem_ld16(tmem_addr(tbase, lane_base, 80), t16);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = t32[i];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[32 + i] = t16[i];
+          if (bl == 2) emit_rows<2>(v, is_q, rl, br, sm);
+        } else {
+          uint32_t v[64], ta[32], tb[32];
+          tmem_ld32(tmem_addr(tbase, lane_base, 96), ta);
+          tmem_ld32(tmem_addr(tbase, lane_base, 128), tb);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            v[i] = ta[i];
+            v[32 + i] = tb[i];
+          }
+          if (bl == 3) emit_rows<3>(v, is_q, rl, br, sm);
+        }
+      }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    prep_sync<kFused>();
+    if (ok && tid == 0) {
+      tma_store_2d(&maps.aqk, sm + kAqs, 0, static_cast<int32_t>(rec * 64));
+      bulk_commit();
+    }
+
+    if (ok) {
+      __half* Xh = reinterpret_cast<__half*>(sm + kXh);
+      __half* Zh = reinterpret_cast<__half*>(sm + kZh);
+      const uint32_t aMh = sbase + kMh, aXh = sbase + kXh, aZh = sbase + kZh, aTb = sbase + kTb;
+      if (tid < 64) {
+        // ---- diagonal blocks: forward substitution in FP32, one column per thread
+        const int bi = tid >> 4, jj = tid & 15;
+        const float* Mf = reinterpret_cast<const float*>(sm + kMf) + bi * (16 * 17);
+        float x[16];
+#pragma unroll
+        for (int rr = 0; rr < 16; ++rr) {
+          float acc0 = 0.f, acc1 = 0.f;  // two partial sums halve the dependent chain
+#pragma unroll
+          for (int ss = 0; ss < rr; ss += 2) {
+            acc0 = fmaf(Mf[rr * 17 + ss], x[ss], acc0);
+            if (ss + 1 < rr) acc1 = fmaf(Mf[rr * 17 + ss + 1], x[ss + 1], acc1);
+          }
+          x[rr] = (rr < jj) ? 0.f : (rr == jj ? 1.f : -(acc0 + acc1));
+        }
+        const int col = bi * 16 + jj;
+        const float bcol = s_beta[col];
+        __nv_bfloat16* tbp = reinterpret_cast<__nv_bfloat16*>(sm + kTb + (col & 7) * 2);
+#pragma unroll
+        for (int rr = 0; rr < 16; ++rr) {
+          Xh[(bi * 16 + rr) * kLdh + col] = __float2half_rn(x[rr]);
+          tbp[sw128_offset(bi * 16 + rr, col >> 3) >> 1] = __float2bfloat16_rn(x[rr] * bcol);
+        }
+      } else {
+        // ---- strictly upper blocks of Tb are zero
+        for (int slot = tid - 64; slot < 64 * 8; slot += kThreads - 64) {
+          const int r = slot >> 3, ch = slot & 7;
+          if (ch >= 2 * ((r >> 4) + 1))
+            *reinterpret_cast<uint4*>(sm + kTb + sw128_offset(r, ch)) = make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+      prep_sync<kFused>();
+      // ---- Z_ik = -X_ii M_ik for the six blocks below the diagonal (one warp each)
+      if (warp < 6) {
+        const int zi = (warp < 3) ? warp + 1 : (warp < 5 ? warp - 1 : 3);
+        const int zk = (warp < 3) ? warp : (warp < 5 ? warp - 3 : 0);
+        float z0[4] = {0.f, 0.f, 0.f, 0.f}, z1[4] = {0.f, 0.f, 0.f, 0.f};
+        mma_block(z0, z1, aXh, zi * 16, zi * 16, aMh, zi * 16, zk * 16, lane);
+        store_frag16(Zh + (zi * 16) * kLdh + zk * 16, kLdh, z0, z1, -1.f, lane);
+      }
+      prep_sync<kFused>();
+      // ---- level 1: X_{i,i-1} = Z_{i,i-1} X_{i-1,i-1}
+      if (warp < 3) {
+        const int i = warp + 1, j = warp;
+        float x0[4] = {0.f, 0.f, 0.f, 0.f}, x1[4] = {0.f, 0.f, 0.f, 0.f};
+        mma_block(x0, x1, aZh, i * 16, j * 16, aXh, j * 16, j * 16, lane);
+        store_frag16(Xh + (i * 16) * kLdh + j * 16, kLdh, x0, x1, 1.f, lane);
+        store_tb16(aTb, s_beta, i * 16, j * 16, x0, x1, lane);
+      }
+      prep_sync<kFused>();
+      // ---- level 2: X_20 = Z_20 X_00 + Z_21 X_10, X_31 = Z_31 X_11 + Z_32 X_21,
+      // and the first two terms of X_30 (kept in warp 2's registers)
+      float y0[4] = {0.f, 0.f, 0.f, 0.f}, y1[4] = {0.f, 0.f, 0.f, 0.f};
+      if (warp < 3) {
+        const int i = (warp == 1) ? 3 : 2 + (warp == 2), j = (warp == 1) ? 1 : 0;
+        mma_block(y0, y1, aZh, i * 16, j * 16, aXh, j * 16, j * 16, lane);
+        mma_block(y0, y1, aZh, i * 16, (j + 1) * 16, aXh, (j + 1) * 16, j * 16, lane);
+        if (warp < 2) {
+          store_frag16(Xh + (i * 16) * kLdh + j * 16, kLdh, y0, y1, 1.f, lane);
+          store_tb16(aTb, s_beta, i * 16, j * 16, y0, y1, lane);
+        }
+      }
+      prep_sync<kFused>();
+      // ---- level 3: X_30 += Z_32 X_20
+      if (warp == 2) {
+        mma_block(y0, y1, aZh, 48, 32, aXh, 32, 0, lane);
+        store_tb16(aTb, s_beta, 48, 0, y0, y1, lane);
+      }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    ok = !prep_sync_or<kFused>(!ok);
+
+    // ---- UMMA 2: W^T = (K Gamma)^T (T diag beta)^T -> cols [0,64); U^T = V^T (T diag beta)^T -> [64,128)
+    bool tma_seen = false;
+    if (ok && tid == 0) {
+      tma_seen = mbar_wait(&tma_bar, tma_parity, budget);
+      if (tma_seen) {
+        tc_fence_after();
+        const uint32_t idesc = idesc_f16(128, 64, kFmtBF16, kMNMajor, kKMajor);
+        const uint32_t aKG = sbase + kKG, aV = sbase + kV, bT = sbase + kTb;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t bd = sdesc_sw128(bT + kk * 32, 16, 1024);
+          umma_f16(tbase + 0, sdesc_sw128(aKG + kk * 2048, 8192, 1024), bd, idesc, kk > 0);
+          umma_f16(tbase + 64, sdesc_sw128(aV + kk * 2048, 8192, 1024), bd, idesc, kk > 0);
+        }
+        umma_commit(&mma_bar);
+      }
+    }
+    if (tid == 0 && !tma_seen) ok = false;
+    ok = !prep_sync_or<kFused>(!ok);
+    if (ok) {
+      ++mma_commits;
+      ok = mbar_wait(&mma_bar, static_cast<uint32_t>((mma_commits - 1) & 1), budget);
+    }
+    ok = !prep_sync_or<kFused>(!ok);
+    // the next item's raw tiles go into v / K Gamma / R, all free now that the
+    // second UMMA has completed (the Aqk staging tile in R has been read once
+    // the bulk group is drained)
+    if (ok && nxt_valid) {
+      if (tid == 0) {
+        bulk_wait_read();
+        issue_raw(nxt);
+      }
+      ++raw_issued;
+      raw_for_cur = true;
+    }
+    if (ok) {
+      tc_fence_after();
+      // warps 0-3: W^T rows (lane = k); warps 4-7: U^T rows (lane = v), into the
+      // swizzled staging tiles of the TMA stores
+      const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32);
+      const int row = (warp & 3) * 32 + lane;
+      const bool is_u = warp >= 4;
+      uint8_t* dst = sm + (is_u ? kUs : kWs);
+      const uint32_t col0 = is_u ? 64u : 0u;
+      uint32_t a[32];
+#pragma unroll
+      for (int part = 0; part < 2; ++part) {
+        tmem_ld32(tmem_addr(tbase, lane_base, col0 + part * 32), a);
+        tmem_wait_ld();
+#pragma unroll
+        for (int q8 = 0; q8 < 4; ++q8) {
+          uint4 o;
+          const float* f = reinterpret_cast<const float*>(a) + q8 * 8;
+          if (is_u) {
+            o = make_uint4(pack_f16(f[0], f[1]), pack_f16(f[2], f[3]), pack_f16(f[4], f[5]),
+                           pack_f16(f[6], f[7]));
+          } else {
+            o = make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
+                           pack_bf16(f[6], f[7]));
+          }
+          *reinterpret_cast<uint4*>(dst + sw128_offset(row, part * 4 + q8)) = o;
+        }
+      }
+    }
+
+    // next item: every thread is done with this item's TMEM and shared tiles
+    fence_proxy_async_smem();
+    tc_fence_before();
+    ok = !prep_sync_or<kFused>(!ok);
+    if (ok && tid == 0) {
+      tma_store_2d(&maps.wt, sm + kWs, 0, static_cast<int32_t>(rec * 128));
+      tma_store_2d(&maps.ut, sm + kUs, 0, static_cast<int32_t>(rec * 128));
+      bulk_commit();
+    }
+    if (ok) pending = rec;
+    cur = nxt;
+    cur_valid = nxt_valid;
+  }
+
+  // ---- teardown: on any failure record it, drain what was issued, free TMEM
+  if (tid == 0) {
+    if (!ok) {
+      record_status(p.ws, kStatusTimeout);
+      // copies and commits complete in issue order: waiting for the last drains all
+      if (tma_issued > 0)
+        mbar_wait(&tma_bar, static_cast<uint32_t>((tma_issued - 1) & 1), drain_budget);
+      if (mma_commits > 0)
+        mbar_wait(&mma_bar, static_cast<uint32_t>((mma_commits - 1) & 1), drain_budget);
+      if (raw_issued > 0)
+        mbar_wait(&raw_bar, static_cast<uint32_t>((raw_issued - 1) & 1), drain_budget);
+    }
+    bulk_wait_all();   // the tile stores this thread issued are complete
+    if constexpr (kFused) {
+      if (ok && pending >= 0) publish_record(p, pending);
+    }
+  }
+  tc_fence_before();
+  prep_sync<kFused>();
+  if (warp == 0) tmem_dealloc(tbase, 256);
+}
+
+}  // namespace kda

@@ -139,3 +139,23 @@ def test_valid_arguments_reach_the_device_check_without_gpu():
         pytest.skip("would launch on fake pointers")
     assert call(fake_args()) == capi.KDA_ERR_UNSUPPORTED_DEVICE
     assert call(fake_args(ht=BASE + 6 * MB)) == capi.KDA_ERR_UNSUPPORTED_DEVICE  # exact alias ok
+
+
+def test_auto_variant_follows_the_table():
+    # few (sequence, head) chains: the fused launch; chains filling the GPU: split
+    few = capi.kda_prefill_describe(capi.make_shape(1, 8192, 12), False)
+    short = capi.kda_prefill_describe(capi.make_shape(1, 512, 12), False)
+    many = capi.kda_prefill_describe(capi.make_shape(8, 65536, 12), False)
+    assert "variant=fused" in few and "recurrence CTAs 12" in few, few
+    assert "variant=split" in short, short
+    assert "variant=split" in many, many
+
+
+def test_fused_variant_needs_free_sms():
+    torch = pytest.importorskip("torch")
+    o = capi.kda_options_t()
+    o.variant = 2
+    # 140 chains leave fewer than 16 SMs of the 148 for prepare CTAs
+    assert call(fake_args(T=1, H=140, h0=None, ht=None, opts=o)) == capi.KDA_ERR_BAD_OPTION
+    if not torch.cuda.is_available():
+        assert call(fake_args(H=4, opts=o)) == capi.KDA_ERR_UNSUPPORTED_DEVICE
