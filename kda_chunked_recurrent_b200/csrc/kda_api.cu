@@ -1,10 +1,10 @@
 // kda_api.cu — host side of the C ABI declared in include/kda_prefill.h.
 //
 // Validation (pointers, sizes, alignment, aliasing, workspace) happens before
-// any launch or write, as the pages require of the native prefill path
-// ("validate paired checkpoint arguments ... before cache mutation", lmdeploy
-// PR #5050 "Motivation"; partial h0/ht overlap rejected, FlashInfer PR #4262
-// "Physical schedules and true in-place state update").  Device metadata
+// any launch or write: lmdeploy PR #5050 ("Motivation") checks the paired
+// checkpoint arguments before anything is mutated, and FlashInfer PR #4262
+// ("Physical schedules and true in-place state update") rejects a partial
+// h0/ht overlap.  Device metadata
 // (cu_seqlens, ckpt_offsets) is never read on the host.  Launch order on the
 // caller's stream: [schedule] -> prepare -> recurrence (split variant), or
 // [schedule] -> ready-flag clear -> one cooperative launch (fused variant).

@@ -11,10 +11,9 @@
 //   Ud       = U - W S0
 //   O        = scale [ (Q * Gamma) S0 + Aqk Ud ]
 //   S1       = Diag(Gamma_63) S0 + (K * exp(G_63 - G))^T Ud
-// This is the chunk-wise factorisation the pages name for the prepare /
-// recurrence split ("decomp runs prepare and recurrence as two launches",
-// FlashInfer PR #4633 "Description"); the algebra is derived from the per-token
-// recurrence.  exp(G_r - G_s) is formed from 16-token sub-blocks so that no FP32
+// The split of this factorisation into a prepare launch and a recurrence launch
+// is the two-launch design FlashInfer PR #4633 calls decomp ("Description");
+// the algebra itself is derived here from the per-token recurrence.  exp(G_r - G_s) is formed from 16-token sub-blocks so that no FP32
 // factor leaves [e^-80, e^80] when every g lies in [-5, 0] (the gate bound of
 // lmdeploy PR #5050 "Motivation").
 #pragma once

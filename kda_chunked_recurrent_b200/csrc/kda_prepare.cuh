@@ -13,10 +13,10 @@
 // A checkpoint offset p inside a sequence is a chunk boundary of the schedule
 // (the chunks cover [0, p) and [p, len) separately), so the checkpoint state is
 // the state after a chunk and needs no extra operands here.
-// (north star subsystem (a): "a chunk-local prepare kernel that forms the
-// decay-weighted intra-chunk products, solves the unit-lower-triangular UT/WY
-// system per chunk and emits W and U"; the split into prepare and recurrence
-// launches is the "decomp" variant of FlashInfer PR #4633 "Description").
+// This is the chunk-local step of the method: decay-weighted intra-chunk key
+// products, the unit-lower-triangular UT/WY solve and W, U per chunk.  Running it
+// as its own launch before the recurrence is the two-launch design FlashInfer PR
+// #4633 calls decomp ("Description").
 //
 // Inputs of a chunk: q, k (bf16) and g (f32) arrive by TMA as whole [64 tok][128 ch]
 // tiles into shared memory the previous chunk no longer needs (issued as soon as

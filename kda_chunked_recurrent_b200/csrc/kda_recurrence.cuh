@@ -1,10 +1,10 @@
 // kda_recurrence.cuh — inter-chunk recurrence with the fused output (body shared
 // by the split recurrence kernel and the recurrence CTAs of the fused launch).
 //
-// One CTA per (sequence, head); the chunks of the sequence are walked in order
-// (north star subsystems (b) "an inter-chunk recurrence kernel that carries S
-// in TMEM/registers across chunks via tcgen05 GEMMs fed by TMA" and (c) "an
-// output kernel fusing the intra-chunk causal term with q.S").  The state is
+// One CTA per (sequence, head); the chunks of the sequence are walked in order,
+// the state S stays in tensor memory from chunk to chunk, tcgen05 UMMAs fed by
+// TMA carry it, and the output (intra-chunk causal term plus the read of S by
+// q) is formed in the same CTA.  The state is
 // kept transposed, S^T[v][k], in TMEM lanes v = 0..127, so every UMMA has M = 128:
 //   P_W^T = S0^T W^T                            (N=64, K=128; bf16; B = W^T, MN-major)
 //   P_Q^T = S0^T (Q Gamma)^T                    (N=64, K=128; bf16; B = Q Gamma rows, K-major)

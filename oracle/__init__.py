@@ -9,11 +9,11 @@ Two independent implementations of the same definition live here:
 * ``prefill``  — the per-token FP64 recurrence in plain C (kda_oracle.c), the
   reference every GPU result is compared against;
 * ``chunked_prefill`` — the chunked (UT/WY) form in NumPy FP64, derived by hand
-  from the per-token recurrence and used only to pin the recurrence
-  ("chunked and unchunked forms agree").
+  from the per-token recurrence and used only to pin it: the chunked and the
+  per-token forms must agree.
 
-Both follow the method statement for Kimi Delta Attention quoted in the
-module header of kda_oracle.c.
+Both compute the Kimi Delta Attention recurrence written out in the module
+header of kda_oracle.c.
 """
 from .kda_oracle import (build_oracle, oracle_library_path, prefill, prefill_f64,
                          max_threads)

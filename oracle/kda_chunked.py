@@ -1,10 +1,10 @@
 """Chunked (UT/WY) form of the KDA recurrence in NumPy FP64 (test infrastructure).
 
 Derived by hand from the per-token recurrence of kda_oracle.c and used only as
-an independent check of it ("chunked and unchunked CPU forms agree").  The
-chunk-wise factorisation is the one the pages name for their prepare /
-recurrence split (FlashInfer PR #4633 "Description": decomp runs prepare and
-recurrence as two launches); the algebra below is ours.
+an independent check of it: the chunked and the per-token forms must agree.
+Splitting a chunk-wise form into a prepare pass and a recurrence pass is what
+FlashInfer PR #4633 ("Description") does in its two-launch design; the algebra
+below is derived here.
 
 For one (sequence, head), one chunk of c tokens (local r = 0..c-1), state S0
 (K x V) entering the chunk, G_r = sum_{s<=r} g_s (per key channel),
