@@ -19,9 +19,11 @@
 // #4633 calls decomp ("Description").
 //
 // Inputs of a chunk: q, k (bf16) and g (f32) arrive by TMA as whole [64 tok][128 ch]
-// tiles into shared memory the previous chunk no longer needs (issued as soon as
-// that chunk's second UMMA has completed, with the rows already prefetched into
-// L2 one chunk earlier); v follows by TMA straight into its UMMA operand layout.
+// tiles into shared memory the previous chunk no longer needs: g into R as soon
+// as that chunk's first UMMA and its Aqk store are done with R (the start of its
+// solve), q and k once its second UMMA has completed; all of them were
+// prefetched into L2 one chunk earlier.  v follows by TMA straight into its
+// UMMA operand layout.
 //
 // Thread mapping for the element-wise part: thread t owns the channel pair
 // (2p, 2p+1), p = t % 64, in sub-block b = t / 64 (tokens 16b .. 16b+15), so a
@@ -68,7 +70,11 @@ constexpr uint32_t kBytes = 65536 + 40960;
 constexpr uint32_t kQraw = kV;                  // q [64 tok][128 ch] bf16
 constexpr uint32_t kKraw = kKG;                 // k [64 tok][128 ch] bf16
 constexpr uint32_t kGraw = kR;                  // g [64 tok][128 ch] f32 (32 KB)
-constexpr uint32_t kRawTx = 16384 + 16384 + 32768;
+constexpr uint32_t kRawQKTx = 16384 + 16384;
+constexpr uint32_t kRawGTx = 32768;
+// the thread that stores Aqk and requests the next g tile (warp 7, idle in the
+// diagonal solve); thread 0 issues every other copy and UMMA
+constexpr int kGThread = 224;
 // aliases of [K+; Q+] once the first UMMA has completed: the solve scratch, and
 // after the solve the staging tiles of the W^T / U^T TMA stores
 constexpr int kLdh = 72;
@@ -308,7 +314,7 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
   using namespace prep;
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
-  __shared__ uint64_t tma_bar, mma_bar, raw_bar;
+  __shared__ uint64_t tma_bar, mma_bar, raw_qk_bar, raw_g_bar;
   __shared__ uint32_t tmem_slot;
   __shared__ float s_beta[kC];
   __shared__ float2 s_tot[4][64];     // per sub-block sums of g (log2 domain), channel pairs
@@ -327,7 +333,8 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
   if (tid == 0) {
     mbar_init(&tma_bar, 1);
     mbar_init(&mma_bar, 1);
-    mbar_init(&raw_bar, 1);
+    mbar_init(&raw_qk_bar, 1);
+    mbar_init(&raw_g_bar, 1);
     fence_mbar_init();
     prefetch_tmap(&maps.v_in);
     prefetch_tmap(&maps.q_in);
@@ -348,13 +355,17 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
   bool ok = true;
   int mma_commits = 0;     // UMMA commits issued so far (their mbarrier phases)
   int tma_issued = 0;      // v tiles issued so far (tma_bar phases)
-  int raw_issued = 0;      // raw q/k/g tile sets issued so far (raw_bar phases)
-  bool raw_for_cur = false;  // the current item's raw tiles are already in flight
-  auto issue_raw = [&](const PrepItem& it) {  // thread 0 only
-    mbar_arrive_expect_tx(&raw_bar, kRawTx);
-    tma_load_3d(sm + kQraw, &maps.q_in, &raw_bar, 0, it.h, it.t0);
-    tma_load_3d(sm + kKraw, &maps.k_in, &raw_bar, 0, it.h, it.t0);
-    tma_load_3d(sm + kGraw, &maps.g_in, &raw_bar, 0, it.h, it.t0);
+  int raw_qk_issued = 0;   // raw q/k tile pairs issued so far (raw_qk_bar phases)
+  int raw_g_issued = 0;    // raw g tiles issued so far (raw_g_bar phases)
+  bool qk_for_cur = false, g_for_cur = false;  // the current item's tiles are in flight
+  auto issue_qk = [&](const PrepItem& it) {  // thread 0 only
+    mbar_arrive_expect_tx(&raw_qk_bar, kRawQKTx);
+    tma_load_3d(sm + kQraw, &maps.q_in, &raw_qk_bar, 0, it.h, it.t0);
+    tma_load_3d(sm + kKraw, &maps.k_in, &raw_qk_bar, 0, it.h, it.t0);
+  };
+  auto issue_g = [&](const PrepItem& it) {  // thread kGThread only, its Aqk stores read
+    mbar_arrive_expect_tx(&raw_g_bar, kRawGTx);
+    tma_load_3d(sm + kGraw, &maps.g_in, &raw_g_bar, 0, it.h, it.t0);
   };
 
   PrepItem cur;
@@ -374,11 +385,18 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
 
     const int cp = tid & 63;         // channel pair
     const int blk = tid >> 6;        // sub-block 0..3
-    if (!raw_for_cur) {
-      if (tid == 0) issue_raw(cur);
-      ++raw_issued;
+    if (!qk_for_cur) {
+      if (tid == 0) issue_qk(cur);
+      ++raw_qk_issued;
     }
-    raw_for_cur = false;
+    if (!g_for_cur) {
+      if (tid == kGThread) {
+        bulk_wait_read();
+        issue_g(cur);
+      }
+      ++raw_g_issued;
+    }
+    qk_for_cur = g_for_cur = false;
     if constexpr (kFused) {
       if (tid == 0 && pending >= 0) publish_record(p, pending);
       pending = -1;
@@ -407,7 +425,8 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
     }
 
     // ---- raw tiles -> registers: g (float2), k, q (bf16x2) for 16 tokens x 2 channels
-    ok = mbar_wait(&raw_bar, static_cast<uint32_t>((raw_issued - 1) & 1), budget);
+    ok = mbar_wait(&raw_g_bar, static_cast<uint32_t>((raw_g_issued - 1) & 1), budget);
+    ok = ok && mbar_wait(&raw_qk_bar, static_cast<uint32_t>((raw_qk_issued - 1) & 1), budget);
     float2 G[16];
     uint32_t kw[16], qw[16];
     {
@@ -593,9 +612,19 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
     fence_proxy_async_smem();
     tc_fence_before();
     prep_sync<kFused>();
-    if (ok && tid == 0) {
+    if (ok && tid == kGThread) {
       tma_store_2d(&maps.aqk, sm + kAqs, 0, static_cast<int32_t>(rec * 64));
       bulk_commit();
+      // R (UMMA1's operand, then the Aqk staging tile) is free once the store has
+      // read it: the next item's g tile goes there now, a whole solve early
+      if (nxt_valid) {
+        bulk_wait_read();
+        issue_g(nxt);
+      }
+    }
+    if (ok && nxt_valid) {
+      ++raw_g_issued;
+      g_for_cur = true;   // (for the next iteration)
     }
 
     if (ok) {
@@ -699,16 +728,12 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
       ok = mbar_wait(&mma_bar, static_cast<uint32_t>((mma_commits - 1) & 1), budget);
     }
     ok = !prep_sync_or<kFused>(!ok);
-    // the next item's raw tiles go into v / K Gamma / R, all free now that the
-    // second UMMA has completed (the Aqk staging tile in R has been read once
-    // the bulk group is drained)
+    // the next item's q and k tiles go into v / K Gamma, free now that the second
+    // UMMA has completed
     if (ok && nxt_valid) {
-      if (tid == 0) {
-        bulk_wait_read();
-        issue_raw(nxt);
-      }
-      ++raw_issued;
-      raw_for_cur = true;
+      if (tid == 0) issue_qk(nxt);
+      ++raw_qk_issued;
+      qk_for_cur = true;
     }
     if (ok) {
       tc_fence_after();
@@ -741,6 +766,14 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
     }
 
     // next item: every thread is done with this item's TMEM and shared tiles
+    if constexpr (kFused) {
+      // the record is published by thread 0 after this barrier: the Aqk store of
+      // kGThread has to be complete by then
+      if (tid == kGThread) {
+        bulk_wait_all();
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+      }
+    }
     fence_proxy_async_smem();
     tc_fence_before();
     ok = !prep_sync_or<kFused>(!ok);
@@ -763,13 +796,18 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
         mbar_wait(&tma_bar, static_cast<uint32_t>((tma_issued - 1) & 1), drain_budget);
       if (mma_commits > 0)
         mbar_wait(&mma_bar, static_cast<uint32_t>((mma_commits - 1) & 1), drain_budget);
-      if (raw_issued > 0)
-        mbar_wait(&raw_bar, static_cast<uint32_t>((raw_issued - 1) & 1), drain_budget);
+      if (raw_qk_issued > 0)
+        mbar_wait(&raw_qk_bar, static_cast<uint32_t>((raw_qk_issued - 1) & 1), drain_budget);
     }
     bulk_wait_all();   // the tile stores this thread issued are complete
     if constexpr (kFused) {
       if (ok && pending >= 0) publish_record(p, pending);
     }
+  }
+  if (tid == kGThread) {
+    if (!ok && raw_g_issued > 0)
+      mbar_wait(&raw_g_bar, static_cast<uint32_t>((raw_g_issued - 1) & 1), drain_budget);
+    bulk_wait_all();
   }
   tc_fence_before();
   prep_sync<kFused>();
