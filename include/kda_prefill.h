@@ -96,6 +96,8 @@ typedef enum {
 
 enum {
   KDA_FLAG_VALIDATE = 1u << 0,       /* kernels check cu_seqlens / ckpt_offsets values  */
+  KDA_FLAG_CU_SEQLENS_I64 = 1u << 2, /* cu_seqlens holds INT64 entries (8-byte aligned);
+                                        the metadata kernel converts them on the device  */
   KDA_FLAG_TEST_FORCE_TIMEOUT = 1u << 1 /* test hook: every bounded wait gives up at once;
                                           exercises the error path, never for production */
 };
@@ -142,8 +144,11 @@ kda_status_t kda_workspace_init(void* workspace, size_t workspace_bytes, void* s
  *   scale     output scale (e.g. 1/sqrt(128)).
  *   h0        [N, H, 128, 128] FP32 initial state S[k][v] (row index = key
  *             channel), contiguous, 16-byte aligned; NULL = zero state.
- *   cu_seqlens [N+1] INT32 device array of sequence starts, or NULL for the
- *             fixed layout (N sequences of T_total / N tokens each).
+ *   cu_seqlens [N+1] INT32 device array of sequence starts (4-byte aligned), or
+ *             NULL for the fixed layout (N sequences of T_total / N tokens each).
+ *             With KDA_FLAG_CU_SEQLENS_I64 the array holds INT64 entries (pass its
+ *             address cast to const int32_t*; 8-byte aligned): a device kernel
+ *             checks and narrows it into the workspace, the host never reads it.
  *   shape     host struct, see kda_shape_t.
  *   out       [T_total, H, 128] BF16 output o (round-to-nearest-even from FP32).
  *   ht        [N, H, 128, 128] FP32 final state, or NULL.  May be exactly h0

@@ -19,7 +19,7 @@ _CAPI_NAMES = {"kda_prefill", "kda_prefill_describe", "kda_prefill_status",
                "kda_workspace_init", "make_shape"}
 KDA_OK = 0
 KDA_VARIANT_AUTO, KDA_VARIANT_SPLIT, KDA_VARIANT_FUSED = 0, 1, 2
-KDA_FLAG_VALIDATE, KDA_FLAG_TEST_FORCE_TIMEOUT = 1, 2
+KDA_FLAG_VALIDATE, KDA_FLAG_TEST_FORCE_TIMEOUT, KDA_FLAG_CU_SEQLENS_I64 = 1, 2, 4
 
 
 def __getattr__(name):
@@ -77,7 +77,8 @@ def prefill(q, k, v, g, beta, scale: float, *, h0=None, cu_seqlens=None, num_seq
     """Launch KDA prefill on device tensors.
 
     q, k, v: [T, H, 128] bf16; g: [T, H, 128] fp32; beta: [T, H] bf16;
-    h0/ht/ckpt_state: [N, H, 128, 128] fp32; cu_seqlens/ckpt_offsets: int32.
+    h0/ht/ckpt_state: [N, H, 128, 128] fp32; cu_seqlens: int32 or int64;
+    ckpt_offsets: int32.
     Without cu_seqlens, ``num_seqs`` (default 1) equal-length sequences are assumed.
     Returns (out, ht, ckpt_state).
     """
@@ -93,6 +94,8 @@ def prefill(q, k, v, g, beta, scale: float, *, h0=None, cu_seqlens=None, num_seq
     if ckpt_offsets is not None and ckpt_state is None:
         ckpt_state = torch.empty(N, H, 128, 128, dtype=torch.float32, device=dev)
     shape = capi.make_shape(N, T, H, max_seqlen)
+    if cu_seqlens is not None and cu_seqlens.dtype == torch.int64:
+        flags |= KDA_FLAG_CU_SEQLENS_I64   # INT64 offsets, narrowed on the device
     opts = {"variant": variant, "flags": flags}
     s = stream if stream is not None else torch.cuda.current_stream(dev)
     need = capi.kda_prefill_workspace_size(shape, ckpt_offsets is not None, opts)

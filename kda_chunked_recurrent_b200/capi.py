@@ -33,6 +33,7 @@ KDA_VARIANT_SPLIT = 1
 KDA_VARIANT_FUSED = 2
 KDA_FLAG_VALIDATE = 1
 KDA_FLAG_TEST_FORCE_TIMEOUT = 2
+KDA_FLAG_CU_SEQLENS_I64 = 4
 
 
 class kda_shape_t(ctypes.Structure):

@@ -77,7 +77,8 @@ struct Resolved {
 kda_status_t check_options(const kda_options_t* o) {
   if (!o) return KDA_OK;
   if (o->variant < KDA_VARIANT_AUTO || o->variant > KDA_VARIANT_FUSED) return KDA_ERR_BAD_OPTION;
-  if (o->flags & ~(static_cast<uint32_t>(KDA_FLAG_VALIDATE | KDA_FLAG_TEST_FORCE_TIMEOUT)))
+  if (o->flags & ~(static_cast<uint32_t>(KDA_FLAG_VALIDATE | KDA_FLAG_TEST_FORCE_TIMEOUT |
+                                         KDA_FLAG_CU_SEQLENS_I64)))
     return KDA_ERR_BAD_OPTION;
   return KDA_OK;
 }
@@ -289,6 +290,9 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
   kda_status_t st = check_options(options);
   if (st != KDA_OK) return st;
   const bool fixed = (cu_seqlens == nullptr);
+  const bool cu64 = options && (options->flags & KDA_FLAG_CU_SEQLENS_I64);
+  if (cu64 && fixed) return KDA_ERR_BAD_OPTION;   // the flag describes a cu_seqlens array
+  const size_t cu_elem = cu64 ? 8 : 4;
   if (!shape) return KDA_ERR_NULL_ARG;
   st = check_shape(shape, fixed, ckpt_state != nullptr);
   if (st != KDA_OK) return st;
@@ -298,7 +302,7 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
   if ((ckpt_state == nullptr) != (ckpt_offsets == nullptr)) return KDA_ERR_UNPAIRED_CKPT;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(g, 16) ||
       !aligned(out, 16) || !aligned(beta, 2) || !aligned(h0, 16) || !aligned(ht, 16) ||
-      !aligned(ckpt_state, 16) || !aligned(cu_seqlens, 4) || !aligned(ckpt_offsets, 4) ||
+      !aligned(ckpt_state, 16) || !aligned(cu_seqlens, cu_elem) || !aligned(ckpt_offsets, 4) ||
       !aligned(workspace, 256))
     return KDA_ERR_MISALIGNED;
   const size_t tok16 = static_cast<size_t>(T * H * 128 * 2);
@@ -306,7 +310,7 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
   const Range rq = rng(q, tok16), rk = rng(k, tok16), rv = rng(v, tok16),
               rg = rng(g, tok16 * 2), rb = rng(beta, static_cast<size_t>(T * H * 2)),
               rh0 = rng(h0, state), rht = rng(ht, state), rck = rng(ckpt_state, state),
-              rcu = rng(cu_seqlens, static_cast<size_t>((N + 1) * 4)),
+              rcu = rng(cu_seqlens, static_cast<size_t>(N + 1) * cu_elem),
               rco = rng(ckpt_offsets, static_cast<size_t>(N * 4)),
               rws = rng(workspace, workspace_bytes), ro = rng(out, tok16);
   if (overlap(rh0, rht) && h0 != ht) return KDA_ERR_PARTIAL_ALIAS;
@@ -341,6 +345,7 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
   p.scale = scale;
   p.h0 = h0;
   p.cu_seqlens = cu_seqlens;
+  p.cu_seqlens64 = nullptr;
   p.ckpt_offsets = ckpt_offsets;
   p.out = static_cast<uint16_t*>(out);
   p.ht = ht;
@@ -352,6 +357,11 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
   p.fixed_len = fixed ? static_cast<int32_t>(T / N) : 0;
   p.ws = static_cast<uint8_t*>(workspace);
   p.lay = r.lay;
+  if (cu64) {
+    // kernels read the INT32 copy the schedule kernel writes into the workspace
+    p.cu_seqlens64 = reinterpret_cast<const int64_t*>(cu_seqlens);
+    p.cu_seqlens = reinterpret_cast<const int32_t*>(p.ws + r.lay.cu32);
+  }
   p.slots = r.lay.slots;
   p.flags = flags;
   p.wait_budget = (flags & KDA_FLAG_TEST_FORCE_TIMEOUT) ? -1 : kDefaultWaitBudget;

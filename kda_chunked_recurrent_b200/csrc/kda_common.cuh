@@ -40,6 +40,7 @@ constexpr size_t kTileAqk = 64 * 64 * 2;   // Aqk   [64 r][64 s]  f16
 constexpr size_t kTileGC = 128 * 4;        // Gamma at the chunk end, f32 [128]
 
 struct WorkspaceLayout {
+  size_t cu32;         // int32 [N+1]   narrowed copy of INT64 cu_seqlens
   size_t chunk_base;   // int32 [N+1]   first slot of each sequence
   size_t seq_order;    // int32 [N]     longest-first order of sequences
   size_t wt, qg, ut, kd, aqk, gc;     // per-record tiles
@@ -63,6 +64,8 @@ inline WorkspaceLayout make_layout(int64_t N, int64_t T, int64_t H, bool fixed, 
                                    bool ckpt) {
   WorkspaceLayout L{};
   size_t off = kHeaderBytes;
+  L.cu32 = off;
+  off = align_up(off + sizeof(int32_t) * (N + 1), 256);
   L.chunk_base = off;
   off = align_up(off + sizeof(int32_t) * (N + 1), 256);
   L.seq_order = off;
@@ -97,7 +100,9 @@ struct KdaParams {
   const uint16_t* beta;
   float scale;
   const float* h0;
-  const int32_t* cu_seqlens;     // NULL: fixed layout
+  const int32_t* cu_seqlens;     // NULL: fixed layout (an INT32 view; see cu_seqlens64)
+  const int64_t* cu_seqlens64;   // INT64 caller array, narrowed into the workspace by the
+                                 // schedule kernel (cu_seqlens then points at the copy)
   const int32_t* ckpt_offsets;   // NULL: no checkpoint
   // outputs
   uint16_t* out;
@@ -135,7 +140,7 @@ enum : int32_t {
   kStatusTimeout = 18,
 };
 
-enum : uint32_t { kFlagValidate = 1u, kFlagForceTimeout = 2u };
+enum : uint32_t { kFlagValidate = 1u, kFlagForceTimeout = 2u, kFlagCu64 = 4u };
 
 __device__ __forceinline__ void record_status(uint8_t* ws, int32_t code) {
   atomicCAS(reinterpret_cast<int32_t*>(ws), 0, code);

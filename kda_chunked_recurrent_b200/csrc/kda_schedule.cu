@@ -32,6 +32,22 @@ __global__ void __launch_bounds__(kSchedThreads) kda_schedule_kernel(const KdaPa
     bad_cu = 0;
     bad_ck = 0;
   }
+  // INT64 cu_seqlens: check (validate mode) and narrow into the workspace copy that
+  // every kernel of this call reads (values clamped to [0, T]; T < 2^31)
+  if (p.cu_seqlens64 != nullptr) {
+    int32_t* cu32 = const_cast<int32_t*>(p.cu_seqlens);
+    for (int n = tid; n <= p.N; n += kSchedThreads) {
+      const int64_t a = p.cu_seqlens64[n];
+      if (validate) {
+        const int64_t prev = n > 0 ? p.cu_seqlens64[n - 1] : 0;
+        if (a < 0 || a > p.T || a < prev || (n == 0 && a != 0) || (n == p.N && a != p.T) ||
+            (n > 0 && p.max_len > 0 && a - prev > p.max_len))
+          atomicExch(&bad_cu, 1);
+      }
+      cu32[n] = static_cast<int32_t>(a < 0 ? 0 : (a > p.T ? p.T : a));
+    }
+    __threadfence_block();
+  }
   __syncthreads();
   for (int base = 0; base < p.N; base += kSchedThreads) {
     const int n = base + tid;

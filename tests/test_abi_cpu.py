@@ -159,3 +159,16 @@ def test_fused_variant_needs_free_sms():
     assert call(fake_args(T=1, H=140, h0=None, ht=None, opts=o)) == capi.KDA_ERR_BAD_OPTION
     if not torch.cuda.is_available():
         assert call(fake_args(H=4, opts=o)) == capi.KDA_ERR_UNSUPPORTED_DEVICE
+
+
+def test_int64_cu_seqlens_validation():
+    torch = pytest.importorskip("torch")
+    o = capi.kda_options_t()
+    o.flags = capi.KDA_FLAG_CU_SEQLENS_I64
+    # the flag describes a cu_seqlens array: meaningless without one
+    assert call(fake_args(opts=o)) == capi.KDA_ERR_BAD_OPTION
+    wsb = capi.kda_prefill_workspace_size(capi.make_shape(2, 128, 2), False)
+    a = fake_args(N=2, cu=BASE + 20 * MB + 4, shape=capi.make_shape(2, 128, 2), wsb=wsb, opts=o)
+    assert call(a) == capi.KDA_ERR_MISALIGNED        # INT64 entries need 8-byte alignment
+    if not torch.cuda.is_available():
+        assert call(dict(a, cu=BASE + 20 * MB)) == capi.KDA_ERR_UNSUPPORTED_DEVICE
