@@ -91,7 +91,7 @@ typedef enum {
                             head) on its own SM, the other SMs prepare the chunk records
                             and hand each one over through a ready flag in the workspace.
                             Needs N*H + 16 <= SM count, else KDA_ERR_BAD_OPTION.  AUTO
-                            picks it for at most 16 chains of at least 32 chunks.      */
+                            picks it for at most 56 chains of at least 32 chunks.      */
 } kda_variant_t;
 
 enum {

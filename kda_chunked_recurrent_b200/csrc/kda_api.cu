@@ -24,7 +24,7 @@ __global__ void kda_schedule_kernel(const KdaParams p);
 __global__ void kda_prepare_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps);
 __global__ void kda_recurrence_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps);
 __global__ void kda_fused_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps,
-                                 int32_t rec_ctas, int64_t prep_items);
+                                 int32_t rec_ctas, int64_t prep_items, int32_t prep_groups);
 namespace prep { extern const uint32_t kSmemAllocBytes; }
 namespace rec { extern const uint32_t kSmemAllocBytes; extern const int kThreadsPerCta; }
 namespace fused { extern const uint32_t kSmemAllocBytes; extern const int kThreadsPerCta; }
@@ -98,23 +98,26 @@ kda_status_t check_shape(const kda_shape_t* s, bool fixed, bool ckpt) {
 
 int sm_count();
 
-// The fused launch keeps at least this many SMs for its prepare CTAs.
+// The fused launch keeps at least this many SMs for its prepare CTAs, which run
+// one prepare group each up to kFusedOneGroupMaxChains chains and two above.
 constexpr int kFusedMinPrepCtas = 16;
+constexpr int kFusedOneGroupMaxChains = 16;
 
 // Per-shape variant table, from CUDA-event timings on one B200 (1965 MHz, ms per
-// call, split / fused): B1 T8192 H12 (12 chains of 128 chunks) 0.296 / 0.256;
-// B1 T512 H12 (12 chains of 8 chunks) 0.041 / 0.044; B4 T8192 H12 (48 chains)
-// 0.487 / 0.547; B6 T8192 H12 (72) 0.551 / 0.989; B8 T1024 and B8 T8192 H12
-// (96) 0.110 / 0.268 and 0.651 / 1.897.  The fused launch hides the prepare
-// work behind the recurrence chains only when few chains (one SM each) leave
-// most SMs to its prepare CTAs and the sequences are long enough to overlap.
+// call, split / fused): B1 T8192 H12 (12 chains of 128 chunks) 0.294 / 0.254;
+// B1 T512 H12 (12 chains of 8 chunks) 0.040 / 0.047; B4 T8192 H12 with
+// checkpoints (48 chains) 0.485 / 0.380; B6 T8192 H12 (72) 0.543 / 0.652;
+// B8 T1024 and B8 T8192 H12 (96) 0.110 / 0.186 and 0.639 / 1.228.  The fused
+// launch hides the prepare work behind the recurrence chains while the chains
+// (one SM each) leave enough SMs to its prepare groups and the sequences are
+// long enough to overlap.
 struct VariantRule {
   int64_t max_chains;   // N H at most this
   int64_t min_chunks;   // and at least this many chunks in the longest sequence
   int variant;          // -> this variant
 };
 constexpr VariantRule kVariantTable[] = {
-    {16, 32, KDA_VARIANT_FUSED},
+    {56, 32, KDA_VARIANT_FUSED},
     {INT64_MAX, 0, KDA_VARIANT_SPLIT},
 };
 
@@ -428,7 +431,8 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
         cudaMemsetAsync(ws + r.lay.ready, 0, static_cast<size_t>(r.lay.slots) * H * sizeof(int32_t),
                         s) != cudaSuccess)
       return KDA_ERR_LAUNCH_FAILED;
-    void* args[] = {&p, &maps, &rec_ctas, &prep_items};
+    int32_t prep_groups = rec_ctas <= kFusedOneGroupMaxChains ? 1 : 2;
+    void* args[] = {&p, &maps, &rec_ctas, &prep_items, &prep_groups};
     if (cudaLaunchCooperativeKernel(reinterpret_cast<void*>(kda_fused_kernel), dim3(grid),
                                     dim3(fused::kThreadsPerCta), args, fused::kSmemAllocBytes,
                                     s) != cudaSuccess)

@@ -13,19 +13,30 @@
 
 namespace kda {
 namespace fused {
-extern const int kThreadsPerCta = rec::kThreads;
-extern const uint32_t kSmemAllocBytes = rec::kSmemAlloc > prep::kSmemAlloc ? rec::kSmemAlloc : prep::kSmemAlloc;
+// two prepare groups of 256 threads per prepare CTA (the recurrence CTAs leave
+// their last two warps idle)
+constexpr int kThreads = 2 * prep::kThreads;
+constexpr uint32_t kPrepBytes = 2 * prep::kGroupBytes + 1024;
+extern const int kThreadsPerCta = kThreads;
+extern const uint32_t kSmemAllocBytes = rec::kSmemAlloc > kPrepBytes ? rec::kSmemAlloc : kPrepBytes;
+static_assert(rec::kThreads <= kThreads, "recurrence warps fit the CTA");
 }
 
-__global__ void __launch_bounds__(rec::kThreads, 1)
+// prep_groups: prepare groups per prepare CTA (1 or 2).  Few chains need little
+// prepare throughput, and one group then leaves more memory bandwidth to them.
+__global__ void __launch_bounds__(fused::kThreads, 1)
 kda_fused_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps, int32_t rec_ctas,
-                 int64_t prep_items) {
+                 int64_t prep_items, int32_t prep_groups) {
   extern __shared__ uint8_t smem_raw[];
   if (static_cast<int32_t>(blockIdx.x) < rec_ctas) {
     recurrence_body<true>(p, maps, smem_raw, blockIdx.x);
   } else {
-    if (threadIdx.x >= prep::kThreads) return;   // the prepare body uses 256 threads
-    prepare_body<true>(p, maps, smem_raw, blockIdx.x - rec_ctas, gridDim.x - rec_ctas, prep_items);
+    const int grp = threadIdx.x / prep::kThreads;
+    if (grp >= prep_groups) return;
+    const int64_t groups = prep_groups * static_cast<int64_t>(gridDim.x - rec_ctas);
+    prepare_body<true>(p, maps, smem_raw, grp,
+                       prep_groups * static_cast<int64_t>(blockIdx.x - rec_ctas) + grp, groups,
+                       prep_items);
   }
 }
 

@@ -10,7 +10,7 @@ extern const uint32_t kSmemAllocBytes = kSmemAlloc;
 __global__ void __launch_bounds__(prep::kThreads, 2)
 kda_prepare_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps) {
   extern __shared__ uint8_t smem_raw[];
-  prepare_body<false>(p, maps, smem_raw, blockIdx.x, gridDim.x, p.slots * p.H);
+  prepare_body<false>(p, maps, smem_raw, 0, blockIdx.x, gridDim.x, p.slots * p.H);
 }
 
 }  // namespace kda

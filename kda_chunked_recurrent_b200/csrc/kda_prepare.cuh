@@ -87,7 +87,15 @@ constexpr uint32_t kUs = kL + 16384;            // U^T staging [128 v][64 tok] f
 // aliases of R once the first UMMA has completed
 constexpr uint32_t kAqs = kR;                   // Aqk staging [64 r][64 s] f16, 128B swizzle
 constexpr uint32_t kTb = 98304;                 // 8 KB T diag(beta) bf16, K-major [64 r][64 s]
-constexpr uint32_t kSmemAlloc = kBytes + 1024;
+// small per-group state after the tiles: mbarriers, TMEM slot, beta, gate sums
+constexpr uint32_t kAux = kBytes;
+constexpr uint32_t kAuxBars = kAux;              // 4 x u64 mbarriers
+constexpr uint32_t kAuxTmem = kAux + 32;         // u32 TMEM base
+constexpr uint32_t kAuxBeta = kAux + 64;         // f32 [64]
+constexpr uint32_t kAuxTot = kAuxBeta + 256;     // float2 [4][64]
+constexpr uint32_t kAuxFirst = kAuxTot + 2048;   // float2 [4][64]
+constexpr uint32_t kGroupBytes = (kAuxFirst + 2048 + 1023) / 1024 * 1024;   // one prepare group
+constexpr uint32_t kSmemAlloc = kGroupBytes + 1024;
 static_assert(kZh + 64 * kLdh * 2 <= kR, "solve scratch overlaps the Aqk staging tile");
 static_assert(kAqs + 8192 <= kTb, "Aqk staging overlaps the Tb tile");
 static_assert(kUs + 16384 <= kR, "W/U staging overlaps R");
@@ -283,15 +291,16 @@ __device__ __forceinline__ bool locate_item_chunk_major(const KdaParams& p, int6
   return it.c > 0;
 }
 
-// CTA-wide barriers of the prepare body: the whole CTA in the split kernel, the
-// first 256 threads (named barrier 1) in a prepare CTA of the fused launch.
+// Group-wide barriers of the prepare body: the whole CTA in the split kernel; in a
+// prepare CTA of the fused launch, which runs two independent 256-thread groups,
+// named barrier 1 + grp over the group's threads.
 template <bool kFused>
-__device__ __forceinline__ void prep_sync() {
-  if constexpr (kFused) named_bar_sync(1, prep::kThreads); else __syncthreads();
+__device__ __forceinline__ void prep_sync(int grp) {
+  if constexpr (kFused) named_bar_sync(1 + grp, prep::kThreads); else __syncthreads();
 }
 template <bool kFused>
-__device__ __forceinline__ bool prep_sync_or(bool pred) {
-  if constexpr (kFused) return named_bar_or(1, prep::kThreads, pred);
+__device__ __forceinline__ bool prep_sync_or(int grp, bool pred) {
+  if constexpr (kFused) return named_bar_or(1 + grp, prep::kThreads, pred);
   else return __syncthreads_or(pred) != 0;
 }
 
@@ -305,22 +314,29 @@ __device__ __forceinline__ void publish_record(const KdaParams& p, int64_t rec) 
   asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(flag), "r"(1) : "memory");
 }
 
-// The prepare loop.  Items first, first + stride, ... < nitems; kFused selects the
-// chunk-major item order, the 256-thread barriers and the ready flags.
+// The prepare loop of one 256-thread group (grp: its index in the CTA; its shared
+// memory is the grp-th kGroupBytes slice).  Items first, first + stride, ... <
+// nitems; kFused selects the chunk-major item order, the named barriers and the
+// ready flags.
 template <bool kFused>
 __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps& maps,
-                                             uint8_t* smem_raw, int64_t first, int64_t stride,
-                                             int64_t nitems) {
+                                             uint8_t* smem_raw, int grp, int64_t first,
+                                             int64_t stride, int64_t nitems) {
   using namespace prep;
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                           ~static_cast<uintptr_t>(1023));
-  __shared__ uint64_t tma_bar, mma_bar, raw_qk_bar, raw_g_bar;
-  __shared__ uint32_t tmem_slot;
-  __shared__ float s_beta[kC];
-  __shared__ float2 s_tot[4][64];     // per sub-block sums of g (log2 domain), channel pairs
-  __shared__ float2 s_first[4][64];   // running sum at the first token of the sub-block
+                                           ~static_cast<uintptr_t>(1023)) +
+                static_cast<size_t>(grp) * kGroupBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kAuxBars);
+  uint64_t& tma_bar = bars[0];
+  uint64_t& mma_bar = bars[1];
+  uint64_t& raw_qk_bar = bars[2];
+  uint64_t& raw_g_bar = bars[3];
+  uint32_t& tmem_slot = *reinterpret_cast<uint32_t*>(sm + kAuxTmem);
+  float* s_beta = reinterpret_cast<float*>(sm + kAuxBeta);
+  float2 (*s_tot)[64] = reinterpret_cast<float2 (*)[64]>(sm + kAuxTot);     // per sub-block sums of g
+  float2 (*s_first)[64] = reinterpret_cast<float2 (*)[64]>(sm + kAuxFirst); // first token's running sum
 
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x - grp * kThreads;
   const int warp = tid >> 5, lane = tid & 31;
   if ((p.flags & kFlagValidate) && reinterpret_cast<const WsHeader*>(p.ws)->call_ok == 0) return;
   const long long budget = p.wait_budget;
@@ -348,7 +364,7 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
     tmem_alloc(&tmem_slot, 256);
     tmem_relinquish();
   }
-  prep_sync<kFused>();
+  prep_sync<kFused>(grp);
   tc_fence_after();
   const uint32_t tbase = tmem_slot;
   const uint32_t sbase = smem_u32(sm);
@@ -455,7 +471,7 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
     }
     // the previous item's TMA stores have finished reading their staging tiles
     if (tid == 0) bulk_wait_read();
-    ok = !prep_sync_or<kFused>(!ok);
+    ok = !prep_sync_or<kFused>(grp, !ok);
     if (!ok) break;
     // ---- TMA: v tile straight into the MN-major A operand of U^T (the raw q tile
     // in that region has been read by every thread)
@@ -544,7 +560,7 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
     // ---- UMMA 1: D[0:128, 0:160] = [K+; Q+] . R^T   (bf16 -> f32)
     fence_proxy_async_smem();
     tc_fence_before();
-    prep_sync<kFused>();
+    prep_sync<kFused>(grp);
     if (tid == 0) {
       tc_fence_after();
       const uint32_t idesc = idesc_f16(128, 160, kFmtBF16, kKMajor, kKMajor);
@@ -559,7 +575,7 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
     }
     ++mma_commits;
     ok = mbar_wait(&mma_bar, static_cast<uint32_t>((mma_commits - 1) & 1), budget);
-    ok = !prep_sync_or<kFused>(!ok);
+    ok = !prep_sync_or<kFused>(grp, !ok);
     if (ok) {
       tc_fence_after();
       // ---- extract A (lane quarters 0,1) and Aqk (quarters 2,3): row rl, sub-block bl.
@@ -611,7 +627,7 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
     }
     fence_proxy_async_smem();
     tc_fence_before();
-    prep_sync<kFused>();
+    prep_sync<kFused>(grp);
     if (ok && tid == kGThread) {
       tma_store_2d(&maps.aqk, sm + kAqs, 0, static_cast<int32_t>(rec * 64));
       bulk_commit();
@@ -662,7 +678,7 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
             *reinterpret_cast<uint4*>(sm + kTb + sw128_offset(r, ch)) = make_uint4(0u, 0u, 0u, 0u);
         }
       }
-      prep_sync<kFused>();
+      prep_sync<kFused>(grp);
       // ---- Z_ik = -X_ii M_ik for the six blocks below the diagonal (one warp each)
       if (warp < 6) {
         const int zi = (warp < 3) ? warp + 1 : (warp < 5 ? warp - 1 : 3);
@@ -671,7 +687,7 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
         mma_block(z0, z1, aXh, zi * 16, zi * 16, aMh, zi * 16, zk * 16, lane);
         store_frag16(Zh + (zi * 16) * kLdh + zk * 16, kLdh, z0, z1, -1.f, lane);
       }
-      prep_sync<kFused>();
+      prep_sync<kFused>(grp);
       // ---- level 1: X_{i,i-1} = Z_{i,i-1} X_{i-1,i-1}
       if (warp < 3) {
         const int i = warp + 1, j = warp;
@@ -680,7 +696,7 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
         store_frag16(Xh + (i * 16) * kLdh + j * 16, kLdh, x0, x1, 1.f, lane);
         store_tb16(aTb, s_beta, i * 16, j * 16, x0, x1, lane);
       }
-      prep_sync<kFused>();
+      prep_sync<kFused>(grp);
       // ---- level 2: X_20 = Z_20 X_00 + Z_21 X_10, X_31 = Z_31 X_11 + Z_32 X_21,
       // and the first two terms of X_30 (kept in warp 2's registers)
       float y0[4] = {0.f, 0.f, 0.f, 0.f}, y1[4] = {0.f, 0.f, 0.f, 0.f};
@@ -693,7 +709,7 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
           store_tb16(aTb, s_beta, i * 16, j * 16, y0, y1, lane);
         }
       }
-      prep_sync<kFused>();
+      prep_sync<kFused>(grp);
       // ---- level 3: X_30 += Z_32 X_20
       if (warp == 2) {
         mma_block(y0, y1, aZh, 48, 32, aXh, 32, 0, lane);
@@ -702,7 +718,7 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
     }
     fence_proxy_async_smem();
     tc_fence_before();
-    ok = !prep_sync_or<kFused>(!ok);
+    ok = !prep_sync_or<kFused>(grp, !ok);
 
     // ---- UMMA 2: W^T = (K Gamma)^T (T diag beta)^T -> cols [0,64); U^T = V^T (T diag beta)^T -> [64,128)
     bool tma_seen = false;
@@ -722,12 +738,12 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
       }
     }
     if (tid == 0 && !tma_seen) ok = false;
-    ok = !prep_sync_or<kFused>(!ok);
+    ok = !prep_sync_or<kFused>(grp, !ok);
     if (ok) {
       ++mma_commits;
       ok = mbar_wait(&mma_bar, static_cast<uint32_t>((mma_commits - 1) & 1), budget);
     }
-    ok = !prep_sync_or<kFused>(!ok);
+    ok = !prep_sync_or<kFused>(grp, !ok);
     // the next item's q and k tiles go into v / K Gamma, free now that the second
     // UMMA has completed
     if (ok && nxt_valid) {
@@ -776,7 +792,7 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
     }
     fence_proxy_async_smem();
     tc_fence_before();
-    ok = !prep_sync_or<kFused>(!ok);
+    ok = !prep_sync_or<kFused>(grp, !ok);
     if (ok && tid == 0) {
       tma_store_2d(&maps.wt, sm + kWs, 0, static_cast<int32_t>(rec * 128));
       tma_store_2d(&maps.ut, sm + kUs, 0, static_cast<int32_t>(rec * 128));
@@ -810,7 +826,7 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
     bulk_wait_all();
   }
   tc_fence_before();
-  prep_sync<kFused>();
+  prep_sync<kFused>(grp);
   if (warp == 0) tmem_dealloc(tbase, 256);
 }
 

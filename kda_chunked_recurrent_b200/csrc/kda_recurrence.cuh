@@ -154,7 +154,9 @@ __device__ __forceinline__ void recurrence_body(const KdaParams& p, const SplitM
   tc_fence_after();
   const uint32_t tbase = tmem_slot;
 
-  if (warp == kTmaWarp) {
+  if (warp >= kThreads / 32) {
+    // no role (the fused launch gives every CTA two more warps than the recurrence uses)
+  } else if (warp == kTmaWarp) {
     // =========================== TMA producer ====================================
     if ((tid & 31) == 0) {
       int issued[kStages] = {0, 0, 0};

@@ -149,6 +149,9 @@ def test_auto_variant_follows_the_table():
     assert "variant=fused" in few and "recurrence CTAs 12" in few, few
     assert "variant=split" in short, short
     assert "variant=split" in many, many
+    mid = capi.kda_prefill_describe(capi.make_shape(4, 32768, 12), False)    # 48 chains
+    wide = capi.kda_prefill_describe(capi.make_shape(6, 49152, 12), False)   # 72 chains
+    assert "variant=fused" in mid and "variant=split" in wide, (mid, wide)
 
 
 def test_fused_variant_needs_free_sms():
