@@ -307,7 +307,11 @@ def main():
     opts = {"variant": args.variant}
     ws = K.Workspace(capi.kda_prefill_workspace_size(shape, cko is not None, opts), dev)
     desc = capi.kda_prefill_describe(shape, cko is not None, opts)
-    variant = "fused" if "variant=fused" in desc else "split"
+    variant = desc.split()[0].split("=")[1] if desc.startswith("variant=") else "split"
+    hybrid_frac = 0.0   # share of the chunks the hybrid's separate prepare launch makes
+    if variant == "hybrid":
+        a, b = desc.split("prepare_chunks=")[1].split()[0].split("/")
+        hybrid_frac = int(a) / int(b)
     stream = torch.cuda.current_stream(dev)
     P = lambda t: None if t is None else t.data_ptr()
 
@@ -324,7 +328,7 @@ def main():
     # schedule (packed layout or checkpoints), then prepare + recurrence (split) or
     # the single cooperative launch (fused)
     launches_per_step = (0 if fixed and cko is None else 1) + \
-        (1 if variant == "fused" else (1 if T > 0 else 0) + 1)
+        {"fused": 1, "hybrid": 2}.get(variant, (1 if T > 0 else 0) + 1)
     in_bytes = sum(x.numel() * x.element_size() for x in (q, k, v, g, beta))
     flush = None
     if in_bytes < 2 * L2_BYTES:
@@ -379,7 +383,18 @@ def main():
     # ---- roofline of the dominant kernel
     peaks, peak_src = load_peaks()
     state_io = N * H * STATE_BYTES * ((1 if h0 is not None else 0) + 1 + (1 if ck is not None else 0))
-    if variant == "fused":
+    if variant == "hybrid":
+        kernels = {
+            "kda_prepare_kernel": (prep_ms, hybrid_frac * PREP_BYTES_PER_TOKHEAD * units,
+                                   ["kda_prepare.cu", "kda_prepare.cuh", "kda_common.cuh",
+                                    "sm100_primitives.cuh"]),
+            "kda_fused_kernel": (rec_ms,
+                                 ((1 - hybrid_frac) * PREP_BYTES_PER_TOKHEAD + REC_BYTES_PER_TOKHEAD)
+                                 * units + state_io,
+                                 ["kda_fused.cu", "kda_prepare.cuh", "kda_recurrence.cuh",
+                                  "kda_common.cuh", "sm100_primitives.cuh"]),
+        }
+    elif variant == "fused":
         # one launch moves both halves' bytes (the records still go through HBM/L2)
         kernels = {
             "kda_fused_kernel": (prep_ms + rec_ms,

@@ -87,11 +87,15 @@ typedef struct {
 typedef enum {
   KDA_VARIANT_AUTO = 0,  /* per-shape choice from the measured table                   */
   KDA_VARIANT_SPLIT = 1, /* prepare kernel over all chunks, then the recurrence kernel */
-  KDA_VARIANT_FUSED = 2  /* one cooperative launch: one recurrence CTA per (sequence,
+  KDA_VARIANT_FUSED = 2, /* one cooperative launch: one recurrence CTA per (sequence,
                             head) on its own SM, the other SMs prepare the chunk records
                             and hand each one over through a ready flag in the workspace.
                             Needs N*H + 16 <= SM count, else KDA_ERR_BAD_OPTION.  AUTO
                             picks it for at most 56 chains of at least 32 chunks.      */
+  KDA_VARIANT_HYBRID = 3 /* the prepare launch for the first chunks of every sequence, then
+                            the fused launch, whose prepare CTAs make the last chunks while
+                            its recurrence CTAs already run.  Same SM condition as FUSED;
+                            AUTO picks it above 56 chains of at least 64 chunks.          */
 } kda_variant_t;
 
 enum {

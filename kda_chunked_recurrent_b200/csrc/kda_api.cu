@@ -76,7 +76,7 @@ struct Resolved {
 
 kda_status_t check_options(const kda_options_t* o) {
   if (!o) return KDA_OK;
-  if (o->variant < KDA_VARIANT_AUTO || o->variant > KDA_VARIANT_FUSED) return KDA_ERR_BAD_OPTION;
+  if (o->variant < KDA_VARIANT_AUTO || o->variant > KDA_VARIANT_HYBRID) return KDA_ERR_BAD_OPTION;
   if (o->flags & ~(static_cast<uint32_t>(KDA_FLAG_VALIDATE | KDA_FLAG_TEST_FORCE_TIMEOUT |
                                          KDA_FLAG_CU_SEQLENS_I64)))
     return KDA_ERR_BAD_OPTION;
@@ -104,13 +104,14 @@ constexpr int kFusedMinPrepCtas = 16;
 constexpr int kFusedOneGroupMaxChains = 16;
 
 // Per-shape variant table, from CUDA-event timings on one B200 (1965 MHz, ms per
-// call, split / fused): B1 T8192 H12 (12 chains of 128 chunks) 0.294 / 0.254;
-// B1 T512 H12 (12 chains of 8 chunks) 0.040 / 0.047; B4 T8192 H12 with
-// checkpoints (48 chains) 0.485 / 0.380; B6 T8192 H12 (72) 0.543 / 0.652;
-// B8 T1024 and B8 T8192 H12 (96) 0.110 / 0.186 and 0.639 / 1.228.  The fused
-// launch hides the prepare work behind the recurrence chains while the chains
-// (one SM each) leave enough SMs to its prepare groups and the sequences are
-// long enough to overlap.
+// call, split / fused / hybrid): B1 T8192 H12 (12 chains of 128 chunks) 0.294 /
+// 0.254 / -; B1 T512 H12 (12 chains of 8 chunks) 0.040 / 0.047 / -; B4 T8192 H12
+// with checkpoints (48 chains) 0.485 / 0.380 / -; B6 T8192 H12 (72) 0.546 /
+// 0.652 / 0.497; B8 T8192 H12 (96) 0.642 / 1.228 / 0.615; B8 T1024 H12 (96 chains
+// of 16 chunks) 0.110 / 0.186 / 0.140.  The fused launch hides the prepare work
+// behind the recurrence chains while the chains (one SM each) leave enough SMs to
+// its prepare groups; the hybrid runs most of the prepare work first on every SM
+// and hides only the last chunks; both need sequences long enough to overlap.
 struct VariantRule {
   int64_t max_chains;   // N H at most this
   int64_t min_chunks;   // and at least this many chunks in the longest sequence
@@ -118,6 +119,7 @@ struct VariantRule {
 };
 constexpr VariantRule kVariantTable[] = {
     {56, 32, KDA_VARIANT_FUSED},
+    {INT64_MAX, 64, KDA_VARIANT_HYBRID},
     {INT64_MAX, 0, KDA_VARIANT_SPLIT},
 };
 
@@ -134,10 +136,26 @@ int choose_variant(const kda_shape_t* s, const kda_options_t* o) {
   const int64_t chunks = max_chunks_per_seq(s, false, false);
   for (const VariantRule& rule : kVariantTable)
     if (chains <= rule.max_chains && chunks >= rule.min_chunks) {
-      if (rule.variant == KDA_VARIANT_FUSED && !fused_eligible(s)) continue;
+      if ((rule.variant == KDA_VARIANT_FUSED || rule.variant == KDA_VARIANT_HYBRID) &&
+          !fused_eligible(s))
+        continue;
       return rule.variant;
     }
   return KDA_VARIANT_SPLIT;
+}
+
+// Hybrid variant: how many of the last chunks of every sequence the fused launch's
+// prepare groups make while its recurrence CTAs run.  The recurrence takes about
+// 1.8 us per chunk; a prepare group inside the fused launch about 13.5 us per
+// record (measured: B6 T8192 H12 with a 47-chunk tail), so the free SMs (2
+// groups each) keep up with jmax * f * 41 / R rows of R records, f = free SM
+// share; 0.9 of that keeps the producer ahead.
+int64_t hybrid_tail_chunks(int64_t jmax, int64_t chains) {
+  const double sms = static_cast<double>(sm_count());
+  const double f = (sms - static_cast<double>(chains)) / sms;
+  int64_t tail = static_cast<int64_t>(0.9 * static_cast<double>(jmax) * f * 41.0 /
+                                      static_cast<double>(chains));
+  return std::max<int64_t>(1, std::min<int64_t>(tail, jmax - 1));
 }
 
 // Upper bound on the chunks of one sequence (the fused launch's chunk-major items).
@@ -266,7 +284,16 @@ kda_status_t kda_prefill_describe(const kda_shape_t* shape, int has_ckpt,
   }
   const Resolved r = resolve(shape, false, has_ckpt != 0, options);
   const long long chains = static_cast<long long>(shape->num_seqs) * shape->num_heads;
-  if (r.variant == KDA_VARIANT_FUSED) {
+  if (r.variant == KDA_VARIANT_HYBRID) {
+    const int64_t jmax = max_chunks_per_seq(shape, false, has_ckpt != 0);
+    const int64_t tail = hybrid_tail_chunks(jmax, chains);
+    snprintf(buf, n,
+             "variant=hybrid chunk=%d prepare_chunks=%lld/%lld (split prepare launch) then "
+             "grid=%dx%d (recurrence CTAs %lld, prepare CTAs %lld, cooperative) workspace_bytes=%zu",
+             kC, static_cast<long long>(jmax - tail), static_cast<long long>(jmax), sm_count(),
+             fused::kThreadsPerCta, chains, static_cast<long long>(sm_count()) - chains,
+             r.lay.total);
+  } else if (r.variant == KDA_VARIANT_FUSED) {
     snprintf(buf, n,
              "variant=fused chunk=%d grid=%dx%d (recurrence CTAs %lld, prepare CTAs %lld, "
              "cooperative) workspace_bytes=%zu",
@@ -331,7 +358,8 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
   const size_t need = kda_prefill_workspace_size(shape, ckpt ? 1 : 0, options);
   if (workspace_bytes < need || workspace_bytes < r.lay.total) return KDA_ERR_WORKSPACE_TOO_SMALL;
   // the fused launch needs an SM per chain plus SMs for its prepare CTAs
-  if (r.variant == KDA_VARIANT_FUSED && !fused_eligible(shape)) return KDA_ERR_BAD_OPTION;
+  if ((r.variant == KDA_VARIANT_FUSED || r.variant == KDA_VARIANT_HYBRID) && !fused_eligible(shape))
+    return KDA_ERR_BAD_OPTION;
 
   // ---------------- device
   st = device_check();
@@ -358,6 +386,8 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
   p.H = static_cast<int32_t>(H);
   p.max_len = shape->max_seqlen;
   p.fixed_len = fixed ? static_cast<int32_t>(T / N) : 0;
+  p.split_jmax = INT32_MAX;
+  p.fused_j0 = 0;
   p.ws = static_cast<uint8_t*>(workspace);
   p.lay = r.lay;
   if (cu64) {
@@ -415,7 +445,20 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
     kda_schedule_kernel<<<1, 1024, 0, s>>>(p);
     mark(0);
   }
-  if (r.variant == KDA_VARIANT_FUSED) {
+  if (r.variant == KDA_VARIANT_FUSED || r.variant == KDA_VARIANT_HYBRID) {
+    const int64_t jmax = max_chunks_per_seq(shape, fixed, ckpt);
+    int64_t j0 = 0;
+    if (r.variant == KDA_VARIANT_HYBRID && T > 0) {
+      // the prepare launch makes chunks [0, j0) of every sequence first
+      j0 = jmax - hybrid_tail_chunks(jmax, N * H);
+      p.split_jmax = static_cast<int32_t>(j0);
+      const int64_t items = r.lay.slots * H;
+      const int64_t pgrid = std::min<int64_t>(items, 2 * static_cast<int64_t>(sm_count()));
+      kda_prepare_kernel<<<static_cast<unsigned>(pgrid), 256, prep::kSmemAllocBytes, s>>>(p, maps);
+      p.split_jmax = INT32_MAX;
+    }
+    p.fused_j0 = static_cast<int32_t>(j0);
+    mark(1);
     // one cooperative launch: CTAs 0 .. N H - 1 run the recurrences, the rest of
     // the SMs (one CTA each) prepare the chunk records in chunk-major order
     int per_sm = 0;
@@ -426,7 +469,7 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
       return KDA_ERR_LAUNCH_FAILED;
     int32_t rec_ctas = static_cast<int32_t>(N * H);
     const int grid = sm_count();   // one CTA per SM (checked above: chains + 16 <= SMs)
-    int64_t prep_items = max_chunks_per_seq(shape, fixed, ckpt) * static_cast<int64_t>(rec_ctas);
+    int64_t prep_items = (jmax - j0) * static_cast<int64_t>(rec_ctas);
     if (r.lay.slots > 0 &&
         cudaMemsetAsync(ws + r.lay.ready, 0, static_cast<size_t>(r.lay.slots) * H * sizeof(int32_t),
                         s) != cudaSuccess)
@@ -437,7 +480,6 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
                                     dim3(fused::kThreadsPerCta), args, fused::kSmemAllocBytes,
                                     s) != cudaSuccess)
       return KDA_ERR_LAUNCH_FAILED;
-    mark(1);
     mark(2);
   } else {
     if (T > 0) {

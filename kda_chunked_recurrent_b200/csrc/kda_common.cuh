@@ -111,6 +111,9 @@ struct KdaParams {
   // sizes
   int32_t N, T, H, max_len;
   int32_t fixed_len;             // sequence length in the fixed layout
+  int32_t split_jmax;            // prepare launch: only chunks j < split_jmax of a sequence
+  int32_t fused_j0;              // fused launch: its prepare groups make chunks j >= fused_j0;
+                                 // chunks below come from a preceding prepare launch
   int64_t slots;
   // workspace
   uint8_t* ws;

@@ -263,7 +263,7 @@ __device__ __forceinline__ bool locate_item(const KdaParams& p, int64_t w, PrepI
   }
   if (n >= p.N) return false;
   const SeqInfo si = seq_info(p, n, false);
-  if (j >= si.nch) return false;
+  if (j >= si.nch || j >= p.split_jmax) return false;
   chunk_span(si, j, it.t0, it.c);
   it.t0 += si.start;
   it.rec = it.slot * p.H + it.h;
@@ -271,12 +271,12 @@ __device__ __forceinline__ bool locate_item(const KdaParams& p, int64_t w, PrepI
 }
 
 // Work item w in chunk-major order, used when prepare CTAs feed recurrence CTAs
-// of the same launch: chunk j = w / R of chain c = w % R (R = N H chains, in the
-// recurrence grid's order), so every chain's chunk j is prepared before any
-// chain's chunk j + 1.
+// of the same launch: chunk j = fused_j0 + w / R of chain c = w % R (R = N H
+// chains, in the recurrence grid's order), so every chain's chunk j is prepared
+// before any chain's chunk j + 1.
 __device__ __forceinline__ bool locate_item_chunk_major(const KdaParams& p, int64_t w, PrepItem& it) {
   const int64_t R = static_cast<int64_t>(p.N) * p.H;
-  const int64_t j = w / R, c = w - (w / R) * R;
+  const int64_t j = p.fused_j0 + w / R, c = w - (w / R) * R;
   int32_t n = static_cast<int32_t>(c / p.H);
   it.h = static_cast<int32_t>(c - static_cast<int64_t>(n) * p.H);
   if (p.cu_seqlens != nullptr) n = reinterpret_cast<const int32_t*>(p.ws + p.lay.seq_order)[n];

@@ -167,7 +167,7 @@ __device__ __forceinline__ void recurrence_body(const KdaParams& p, const SplitM
         if (slot < 0 || slot >= p.slots) return;  // corrupt metadata: nothing to load
         const int32_t recr = static_cast<int32_t>(slot * p.H + h);
         if constexpr (kFused) {
-          if (!wait_record(p, recr, budget)) {
+          if (j >= p.fused_j0 && !wait_record(p, recr, budget)) {
             ok = false;
             return;
           }

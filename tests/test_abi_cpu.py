@@ -49,8 +49,10 @@ def test_workspace_size_grows_with_work():
 
 
 def test_describe_reports_grid_and_variant():
-    d = capi.kda_prefill_describe(capi.make_shape(8, 65536, 12, 8192), False)
+    d = capi.kda_prefill_describe(capi.make_shape(8, 65536, 12, 8192), False, {"variant": 1})
     assert "variant=split" in d and "chunk=64" in d and "recurrence_grid=96x448" in d
+    h = capi.kda_prefill_describe(capi.make_shape(8, 65536, 12, 8192), False, {"variant": 3})
+    assert "variant=hybrid" in h and "prepare_chunks=" in h and "recurrence CTAs 96" in h
 
 
 # --- host-side validation with fake, never-dereferenced device addresses ----------
@@ -148,10 +150,12 @@ def test_auto_variant_follows_the_table():
     many = capi.kda_prefill_describe(capi.make_shape(8, 65536, 12), False)
     assert "variant=fused" in few and "recurrence CTAs 12" in few, few
     assert "variant=split" in short, short
-    assert "variant=split" in many, many
+    assert "variant=hybrid" in many, many
     mid = capi.kda_prefill_describe(capi.make_shape(4, 32768, 12), False)    # 48 chains
     wide = capi.kda_prefill_describe(capi.make_shape(6, 49152, 12), False)   # 72 chains
-    assert "variant=fused" in mid and "variant=split" in wide, (mid, wide)
+    huge = capi.kda_prefill_describe(capi.make_shape(32, 16384, 12), False)  # 384 chains
+    assert "variant=fused" in mid and "variant=hybrid" in wide, (mid, wide)
+    assert "variant=split" in huge, huge
 
 
 def test_fused_variant_needs_free_sms():

@@ -84,3 +84,32 @@ def test_fused_full_size_sampled(name):
     res = run_gpu(inp, variant=FUSED)
     m = compare(inp, res, seqs=[0], heads=[0, inp.num_heads // 2, inp.num_heads - 1])
     assert_parity(m)
+
+
+HYBRID = 3
+
+
+@pytest.mark.parametrize("lens,H", [([700, 333, 64], 4), ([4100, 64, 2000, 1], 3)])
+def test_hybrid_equals_split_bitwise(lens, H):
+    inp = make_inputs(lens, H, seed=320 + H, with_h0=True)
+    a = run_gpu(inp, variant=HYBRID)
+    b = run_gpu(inp, variant=SPLIT)
+    assert torch.equal(a["o"], b["o"])
+    assert torch.equal(a["ht"], b["ht"])
+    assert_parity(compare(inp, a))
+
+
+def test_hybrid_checkpoints_and_fixed_layout():
+    inp = make_inputs([2500] * 3, 4, seed=330, with_h0=True, with_ckpt=True, fixed_layout=True)
+    assert_parity(compare(inp, run_gpu(inp, variant=HYBRID)))
+
+
+def test_hybrid_forced_timeout_reports_status_and_context_survives():
+    import kda_chunked_recurrent_b200 as K
+    inp = make_inputs([3000], 2, seed=331, fixed_layout=True)
+    d = to_dev(inp)
+    ws = K.Workspace(K.capi.kda_prefill_workspace_size(K.capi.make_shape(1, 3000, 2), False))
+    K.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], inp.scale, workspace=ws,
+              variant=HYBRID, flags=K.KDA_FLAG_TEST_FORCE_TIMEOUT)
+    assert ws.status() == K.capi.KDA_ERR_TIMEOUT
+    assert_parity(compare(inp, run_gpu(inp, variant=HYBRID)))
