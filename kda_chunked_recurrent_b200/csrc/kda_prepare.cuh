@@ -413,10 +413,6 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
       ++raw_g_issued;
     }
     qk_for_cur = g_for_cur = false;
-    if constexpr (kFused) {
-      if (tid == 0 && pending >= 0) publish_record(p, pending);
-      pending = -1;
-    }
     uint16_t beta_raw = 0;   // consumed only after the operand pass, so its latency hides
     if (tid < c) beta_raw = p.beta[static_cast<int64_t>(t0 + tid) * p.H + h];
 
@@ -572,7 +568,13 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
         umma_f16(tbase, ad, bd, idesc, kk > 0);
       }
       umma_commit(&mma_bar);
+      if constexpr (kFused) {
+        // the previous record's tile stores were issued a whole element-wise pass
+        // ago and are long complete: publish it while this UMMA runs
+        if (pending >= 0) publish_record(p, pending);
+      }
     }
+    if constexpr (kFused) pending = -1;
     ++mma_commits;
     ok = mbar_wait(&mma_bar, static_cast<uint32_t>((mma_commits - 1) & 1), budget);
     ok = !prep_sync_or<kFused>(grp, !ok);
