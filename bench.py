@@ -60,11 +60,12 @@ def kernel_source_sha(files):
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(kernel, units):
-    """DRAM bytes per launch from the committed ncu summary, if the kernel is unchanged."""
+def ncu_traffic(kernel, variant, units):
+    """DRAM bytes per launch from the committed ncu summary (kernel@variant), if the
+    kernel sources are unchanged since it was taken."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     try:
-        d = json.load(open(p))[kernel]
+        d = json.load(open(p))[f"{kernel}@{variant}"]
     except Exception:
         return None
     if d.get("source_sha") != kernel_source_sha(d.get("sources", [])):
@@ -416,7 +417,7 @@ def main():
     achieved = dbytes / (dms / 1e3) / 1e9
     roof = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1),
             "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-            "traffic": ncu_traffic(dom, units), "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
+            "traffic": ncu_traffic(dom, variant, units), "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
             if peak_src == "measured" else "fallback 6650 GB/s",
             "kernel_ms": round(dms, 4),
             "algorithmic_bytes": int(dbytes),
