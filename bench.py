@@ -11,6 +11,7 @@ last kernel of each step.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
   python bench.py --impl reference ...   # the FP64 CPU oracle on the host cores
+  python bench.py --op decode [--decode N,T,H]  # kda_decode over a state pool
 
 Multi-GPU (torchrun, one rank per GPU): every rank runs the same per-GPU
 workload on its own seeded data (weak scaling, no collective on the data path);
@@ -265,6 +266,156 @@ def run_reference(args, rank, world):
     return 0
 
 
+DECODE_METRIC = "KDA decode Mtokens·heads/s at 1 B200 (state pool, one launch per step)"
+
+
+def run_decode(args):
+    """kda_decode over a pool of N states: N sequences of T new tokens, H heads, each
+    sequence on a random slot of the pool.  A step is one kda_decode call; the pool is
+    updated in place (the recurrence continues from step to step)."""
+    import torch
+    rank, world, local = dist_setup("nccl")
+    torch.cuda.set_device(local)
+    import kda_chunked_recurrent_b200 as K
+    from kda_chunked_recurrent_b200 import capi
+    from kda_chunked_recurrent_b200.inputs import make_decode_inputs
+    N, T, H = (int(x) for x in args.decode.split(","))
+    dinp = make_decode_inputs(N, T, H, N, rank_seed(1010, rank), indices=True)
+    dev = torch.device("cuda", local)
+    q, k, v, g, beta, idx = (x.to(dev) for x in (dinp.q, dinp.k, dinp.v, dinp.g, dinp.beta,
+                                                  dinp.state_indices))
+    pool = dinp.pool.to(dev)
+    out = torch.empty(N, T, H, 128, dtype=torch.bfloat16, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    shape = capi.make_decode_shape(N, T, H, N)
+    stream = torch.cuda.current_stream(dev)
+    Pt = lambda t: t.data_ptr()
+
+    def step():
+        rc = capi.kda_decode(Pt(q), Pt(k), Pt(v), Pt(g), Pt(beta), dinp.scale, Pt(pool), Pt(idx),
+                             shape, Pt(out), None, Pt(status), 0, stream.cuda_stream)
+        if rc != 0:
+            raise K.KDAError(rc, "kda_decode")
+
+    units = N * T * H
+    # bytes a decode step must move: the state slice read and written once, the token rows
+    algo_bytes = N * H * 2 * STATE_BYTES + units * PATH_BYTES_PER_TOKHEAD
+    flush = None
+    if algo_bytes < 2 * L2_BYTES:
+        flush = torch.empty(256 * 2**20, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+    ev_a = [mk() for _ in range(args.steps)]
+    ev_b = [mk() for _ in range(args.steps)]
+    clk = ClockSampler(local if world > 1 else int(os.environ.get("CUDA_VISIBLE_DEVICES", "0").split(",")[0] or 0))
+    clk.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    clk.mark_on()
+    t0, t1 = mk(), mk()
+    t0.record(stream)
+    for i in range(args.steps):
+        if flush is not None:
+            flush.zero_()
+        ev_a[i].record(stream)
+        step()
+        ev_b[i].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clk.mark_off()
+    barrier(world)
+    clk.stop()
+    kern_ms = statistics.mean(ev_a[i].elapsed_time(ev_b[i]) for i in range(args.steps))
+    ms_local = kern_ms if flush is not None else t0.elapsed_time(t1) / args.steps
+    ms = max_over_ranks(ms_local, world)
+    if int(status.item()) != 0:
+        raise K.KDAError(int(status.item()), "decode device status")
+    value = units * world / (ms / 1e3) / 1e6
+    peaks, peak_src = load_peaks()
+    achieved = algo_bytes / (kern_ms / 1e3) / 1e9
+    roof = {"kernel": "kda_token_kernel", "bound": "hbm", "achieved": round(achieved, 1),
+            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+            "traffic": ncu_traffic("kda_token_kernel", f"decode_{N}_{T}_{H}", units),
+            "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
+            else "fallback 6650 GB/s", "kernel_ms": round(kern_ms, 4),
+            "algorithmic_bytes": int(algo_bytes)}
+
+    # end to end: the step's token rows and slots from pinned host memory, o back;
+    # the pool stays resident on the device as in a serving engine
+    e2e = None
+    if args.e2e_steps > 0:
+        hq, hk, hv, hg, hb, hi = (x.pin_memory() for x in (dinp.q, dinp.k, dinp.v, dinp.g,
+                                                           dinp.beta, dinp.state_indices))
+        ho = torch.empty(N, T, H, 128, dtype=torch.bfloat16).pin_memory()
+        h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hg, hb, hi))
+
+        def e2e_step():
+            for dst, src in ((q, hq), (k, hk), (v, hv), (g, hg), (beta, hb), (idx, hi)):
+                dst.copy_(src, non_blocking=True)
+            step()
+            ho.copy_(out, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        a, b = mk(), mk()
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = max_over_ranks(a.elapsed_time(b) / args.e2e_steps, world)
+        e2e = {"value": units * world / (e_ms / 1e3) / 1e6, "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(ho.numel() * 2),
+               "ms_per_step": round(e_ms, 4)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import numpy as np
+        import oracle
+        oracle.build_oracle()
+        ns = min(N, 64)
+        sel = lambda x: np.ascontiguousarray(x[:ns].double().numpy().reshape(ns * T, H, -1))
+        qs, ks, vs, gs = sel(dinp.q), sel(dinp.k), sel(dinp.v), sel(dinp.g)
+        bs = np.ascontiguousarray(dinp.beta[:ns].double().numpy().reshape(ns * T, H))
+        h0 = np.ascontiguousarray(dinp.pool.double().numpy()[dinp.state_indices[:ns].long().numpy()])
+        cu = np.arange(ns + 1, dtype=np.int64) * T
+        cores = min(os.cpu_count() or 1, ns * H)
+        reps, dt = 0, 0.0
+        while reps == 0 or (dt < 2.0 and reps < 200):
+            t = time.perf_counter()
+            oracle.prefill_f64(qs, ks, vs, gs, bs, dinp.scale, cu, h0, threads=cores)
+            dt += time.perf_counter() - t
+            reps += 1
+        cpu = {"value": ns * T * H * reps / dt / 1e6, "unit": UNIT, "cores": cores,
+               "kind": "oracle",
+               "sample": f"first {ns} of {N} sequences x {T} token(s) x {H} heads from their pool "
+                         f"slots, x {reps} run(s), FP64 per-token recurrence"}
+
+    if rank == 0:
+        line = {"metric": DECODE_METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+                "data": "synthetic",
+                "config": {"workload": f"decode_N{N}_T{T}_H{H}", "num_seqs": N, "tokens_per_seq": T,
+                           "heads": H, "pool_slots": N, "head_dim": 128,
+                           "parallelism": f"dp{world}" if world > 1 else "single",
+                           "l2": "state and rows (%.3f GB) larger than 2x L2, no flush" %
+                           (algo_bytes / 1e9) if flush is None else
+                           "state and rows (%.3f GB) smaller than 2x L2: 256 MB written before "
+                           "every step, each step timed alone" % (algo_bytes / 1e9)},
+                "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": args.steps, "clocks": clk.summary()}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -275,8 +426,13 @@ def main():
     ap.add_argument("--variant", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--op", default="prefill", choices=["prefill", "decode"])
+    ap.add_argument("--decode", default="256,1,12",
+                    help="N,T,H of the decode workload: N sequences of T new tokens, H heads")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.op == "decode":
+        return run_decode(args)
 
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))
@@ -328,8 +484,11 @@ def main():
 
     # schedule (packed layout or checkpoints), then prepare + recurrence (split) or
     # the single cooperative launch (fused)
-    launches_per_step = (0 if fixed and cko is None else 1) + \
-        {"fused": 1, "hybrid": 2}.get(variant, (1 if T > 0 else 0) + 1)
+    if variant == "token":
+        launches_per_step = 1   # no metadata kernel for INT32 offsets without validation
+    else:
+        launches_per_step = (0 if fixed and cko is None else 1) + \
+            {"fused": 1, "hybrid": 2}.get(variant, (1 if T > 0 else 0) + 1)
     in_bytes = sum(x.numel() * x.element_size() for x in (q, k, v, g, beta))
     flush = None
     if in_bytes < 2 * L2_BYTES:
@@ -394,6 +553,11 @@ def main():
                                  * units + state_io,
                                  ["kda_fused.cu", "kda_prepare.cuh", "kda_recurrence.cuh",
                                   "kda_common.cuh", "sm100_primitives.cuh"]),
+        }
+    elif variant == "token":
+        kernels = {
+            "kda_token_kernel": (prep_ms + rec_ms, PATH_BYTES_PER_TOKHEAD * units + state_io,
+                                 ["kda_token.cu", "kda_common.cuh", "sm100_primitives.cuh"]),
         }
     elif variant == "fused":
         # one launch moves both halves' bytes (the records still go through HBM/L2)
@@ -479,7 +643,8 @@ def main():
                 "config": {"workload": args.workload, "num_seqs": N, "seq_lens": "x".join(
                     map(str, sorted(set(lens)))) if len(set(lens)) < 4 else "ragged",
                     "total_tokens": T, "heads": H, "head_dim": 128, "h0": h0 is not None,
-                    "checkpoint": ck is not None, "variant": variant, "chunk": 64,
+                    "checkpoint": ck is not None, "variant": variant,
+                    "chunk": None if variant == "token" else 64,
                     "parallelism": f"dp{world}" if world > 1 else "single",
                     "l2": ("inputs (%.2f GB) larger than L2, no flush" % (in_bytes / 1e9))
                     if flush is None else

@@ -72,8 +72,9 @@ typedef enum {
   KDA_ERR_BAD_CU_SEQLENS = 16,     /* cu_seqlens[0] != 0, decreasing, or last != T,
                                       or a length above max_seqlen (validate mode)   */
   KDA_ERR_BAD_CKPT_OFFSET = 17,    /* an offset outside [0, len] (validate mode)     */
-  KDA_ERR_TIMEOUT = 18             /* a bounded on-chip wait gave up (the kernel
+  KDA_ERR_TIMEOUT = 18,            /* a bounded on-chip wait gave up (the kernel
                                       returned without finishing its work)          */
+  KDA_ERR_BAD_STATE_INDEX = 19     /* kda_decode: a state index >= pool_size          */
 } kda_status_t;
 
 /* Sizes known on the host.  No device memory is read to obtain them. */
@@ -92,11 +93,16 @@ typedef enum {
                             and hand each one over through a ready flag in the workspace.
                             Needs N*H + 16 <= SM count, else KDA_ERR_BAD_OPTION.  AUTO
                             picks it for at most 56 chains of at least 32 chunks.      */
-  KDA_VARIANT_HYBRID = 3 /* the prepare launch for the first chunks of every sequence, then
+  KDA_VARIANT_HYBRID = 3, /* the prepare launch for the first chunks of every sequence, then
                             the fused launch, whose prepare CTAs make the last chunks while
                             its recurrence CTAs already run.  Same SM condition as FUSED;
                             AUTO picks it above 56 chains of at least 64 chunks.          */
+  KDA_VARIANT_TOKEN = 4   /* the recurrence one token at a time: 4 CTAs per (sequence,
+                            head), each holding 32 value columns of the state in registers;
+                            no chunk records, workspace = header only.  AUTO picks it when
+                            max_seqlen (else T_total) is at most KDA_TOKEN_AUTO_MAX_LEN.  */
 } kda_variant_t;
+#define KDA_TOKEN_AUTO_MAX_LEN 64
 
 enum {
   KDA_FLAG_VALIDATE = 1u << 0,       /* kernels check cu_seqlens / ckpt_offsets values  */
@@ -230,6 +236,62 @@ kda_status_t kda_prefill_noalloc(const void* q, const void* k, const void* v, co
                                  void* out, float* ht, float* ckpt_state,
                                  const int32_t* ckpt_offsets, const kda_options_t* options,
                                  void* stream);
+
+/*
+ * Decode and draft verification over a pool of states (one launch on `stream`).
+ *
+ * The same recurrence as kda_prefill, for N sequences of exactly T new tokens
+ * each (T = 1: decode of one token; T = 1 + d: verification of d draft tokens),
+ * each continuing from a state held in a caller-owned pool.  Serving engines keep
+ * the per-(sequence, head) recurrent states of many requests in one pool and pass
+ * the slot of every request (SGLang kda_flashinfer.py "FlashInferKDAKernel":
+ * decode and target-verify over a state pool with per-request state indices).
+ * The pages define no separate verify arithmetic; here verification is the plain
+ * recurrence over the T tokens with the state after every token exported, so
+ * that the caller can keep the state of the accepted prefix.
+ *
+ *   q, k, v   [N, T, H, 128] BF16, contiguous, 16-byte aligned.
+ *   g         [N, T, H, 128] FP32 log-decay, contiguous, 16-byte aligned.
+ *   beta      [N, T, H] BF16, 2-byte aligned.
+ *   scale     output scale.
+ *   state     [P, H, 128, 128] FP32 pool, S[k][v] per (slot, head), 16-byte
+ *             aligned.  Slot i of sequence n is read before its first token and,
+ *             unless KDA_DECODE_KEEP_STATE, overwritten with the state after its
+ *             last token (in place).
+ *   state_indices [N] INT32 device array, 4-byte aligned, or NULL (sequence n uses
+ *             slot n; then P >= N).  A negative entry marks a padding row: its
+ *             slot is neither read nor written and its out rows are set to zero.
+ *             An entry >= P is handled like a padding row and recorded as
+ *             KDA_ERR_BAD_STATE_INDEX in *device_status.  Two sequences sharing a
+ *             slot race (undefined result).  Values are never read on the host.
+ *   shape     host struct, see kda_decode_shape_t.
+ *   out       [N, T, H, 128] BF16 output o.
+ *   step_states [N, T, H, 128, 128] FP32, 16-byte aligned, or NULL: the state
+ *             after each token (step_states[n][t] = state after token t).
+ *   device_status  INT32 device word, 4-byte aligned, or NULL: the first device
+ *             error is stored there with atomicCAS from KDA_OK (the caller clears
+ *             it); without it device errors are not reported.
+ *   flags     KDA_DECODE_KEEP_STATE: the pool is read only.
+ *   stream    cudaStream_t.
+ *
+ * Outputs (state, out, step_states, device_status) must not overlap the inputs
+ * or each other (KDA_ERR_OUT_ALIAS).  Returns KDA_OK when the launch was
+ * enqueued.  No workspace and no allocation; CUDA-graph capturable.
+ */
+typedef struct {
+  int32_t num_seqs;       /* N >= 1                                               */
+  int32_t tokens_per_seq; /* T >= 1 new tokens of every sequence                  */
+  int32_t num_heads;      /* H >= 1                                               */
+  int32_t pool_size;      /* P >= 1 state slots in `state`                        */
+} kda_decode_shape_t;
+
+enum { KDA_DECODE_KEEP_STATE = 1u << 0 };
+
+kda_status_t kda_decode(const void* q, const void* k, const void* v, const float* g,
+                        const void* beta, float scale, float* state,
+                        const int32_t* state_indices, const kda_decode_shape_t* shape,
+                        void* out, float* step_states, int32_t* device_status, uint32_t flags,
+                        void* stream);
 
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
 int kda_version(void);

@@ -16,9 +16,11 @@ from typing import Optional
 # any use of the CUDA path without the built library raises ImportError.
 _CAPI_NAMES = {"kda_prefill", "kda_prefill_describe", "kda_prefill_status",
                "kda_prefill_workspace_size", "kda_status_string", "kda_version",
-               "kda_workspace_init", "make_shape"}
+               "kda_workspace_init", "make_shape", "kda_decode", "make_decode_shape"}
 KDA_OK = 0
 KDA_VARIANT_AUTO, KDA_VARIANT_SPLIT, KDA_VARIANT_FUSED = 0, 1, 2
+KDA_VARIANT_HYBRID, KDA_VARIANT_TOKEN = 3, 4
+KDA_DECODE_KEEP_STATE = 1
 KDA_FLAG_VALIDATE, KDA_FLAG_TEST_FORCE_TIMEOUT, KDA_FLAG_CU_SEQLENS_I64 = 1, 2, 4
 
 
@@ -29,9 +31,10 @@ def __getattr__(name):
         return getattr(importlib.import_module(".capi", __name__), name)
     raise AttributeError(name)
 
-__all__ = ["capi", "prefill", "Workspace", "KDAError", "kda_prefill", "kda_prefill_describe",
-           "kda_prefill_status", "kda_prefill_workspace_size", "kda_status_string",
-           "kda_version", "kda_workspace_init", "make_shape"]
+__all__ = ["capi", "prefill", "decode", "Workspace", "KDAError", "kda_prefill",
+           "kda_prefill_describe", "kda_prefill_status", "kda_prefill_workspace_size",
+           "kda_status_string", "kda_version", "kda_workspace_init", "make_shape", "kda_decode",
+           "make_decode_shape"]
 
 
 class KDAError(RuntimeError):
@@ -110,3 +113,33 @@ def prefill(q, k, v, g, beta, scale: float, *, h0=None, cu_seqlens=None, num_seq
     if rc != KDA_OK:
         raise KDAError(rc)
     return out, ht, ckpt_state
+
+
+def decode(q, k, v, g, beta, scale: float, state, *, state_indices=None, out=None,
+           step_states=None, return_step_states: bool = False, keep_state: bool = False,
+           device_status=None, stream=None):
+    """Decode / draft verification over a state pool (kda_decode).
+
+    q, k, v: [N, T, H, 128] bf16; g: [N, T, H, 128] fp32; beta: [N, T, H] bf16;
+    state: [P, H, 128, 128] fp32 pool, updated in place unless ``keep_state``;
+    state_indices: [N] int32 slots (negative = padding row) or None (slot n).
+    Returns (out, step_states); step_states [N, T, H, 128, 128] when requested.
+    """
+    import torch
+    from . import capi
+    N, T, H = int(q.shape[0]), int(q.shape[1]), int(q.shape[2])
+    P = int(state.shape[0])
+    dev = q.device
+    if out is None:
+        out = torch.empty(N, T, H, 128, dtype=torch.bfloat16, device=dev)
+    if step_states is None and return_step_states:
+        step_states = torch.empty(N, T, H, 128, 128, dtype=torch.float32, device=dev)
+    shape = capi.make_decode_shape(N, T, H, P)
+    s = stream if stream is not None else torch.cuda.current_stream(dev)
+    rc = capi.kda_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale),
+                         _ptr(state), _ptr(state_indices), shape, _ptr(out), _ptr(step_states),
+                         _ptr(device_status), KDA_DECODE_KEEP_STATE if keep_state else 0,
+                         s.cuda_stream)
+    if rc != KDA_OK:
+        raise KDAError(rc, "kda_decode")
+    return out, step_states

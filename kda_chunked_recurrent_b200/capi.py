@@ -27,10 +27,15 @@ KDA_ERR_BAD_OPTION = 10
 KDA_ERR_BAD_CU_SEQLENS = 16
 KDA_ERR_BAD_CKPT_OFFSET = 17
 KDA_ERR_TIMEOUT = 18
+KDA_ERR_BAD_STATE_INDEX = 19
 
 KDA_VARIANT_AUTO = 0
 KDA_VARIANT_SPLIT = 1
 KDA_VARIANT_FUSED = 2
+KDA_VARIANT_HYBRID = 3
+KDA_VARIANT_TOKEN = 4
+KDA_TOKEN_AUTO_MAX_LEN = 64
+KDA_DECODE_KEEP_STATE = 1
 KDA_FLAG_VALIDATE = 1
 KDA_FLAG_TEST_FORCE_TIMEOUT = 2
 KDA_FLAG_CU_SEQLENS_I64 = 4
@@ -39,6 +44,11 @@ KDA_FLAG_CU_SEQLENS_I64 = 4
 class kda_shape_t(ctypes.Structure):
     _fields_ = [("num_seqs", ctypes.c_int32), ("total_tokens", ctypes.c_int32),
                 ("num_heads", ctypes.c_int32), ("max_seqlen", ctypes.c_int32)]
+
+
+class kda_decode_shape_t(ctypes.Structure):
+    _fields_ = [("num_seqs", ctypes.c_int32), ("tokens_per_seq", ctypes.c_int32),
+                ("num_heads", ctypes.c_int32), ("pool_size", ctypes.c_int32)]
 
 
 class kda_options_t(ctypes.Structure):
@@ -70,6 +80,9 @@ def _load():
     lib.kda_prefill_describe.argtypes = [ctypes.POINTER(kda_shape_t), ctypes.c_int,
                                          ctypes.POINTER(kda_options_t), ctypes.c_char_p,
                                          ctypes.c_size_t]
+    lib.kda_decode.restype = ctypes.c_int
+    lib.kda_decode.argtypes = [P, P, P, P, P, ctypes.c_float, P, P,
+                               ctypes.POINTER(kda_decode_shape_t), P, P, P, ctypes.c_uint32, P]
     return lib
 
 
@@ -128,3 +141,15 @@ def kda_prefill_describe(shape: kda_shape_t, has_ckpt: bool, options=None) -> st
     buf = ctypes.create_string_buffer(512)
     lib.kda_prefill_describe(ctypes.byref(shape), int(bool(has_ckpt)), _opt(options), buf, 512)
     return buf.value.decode()
+
+
+def make_decode_shape(num_seqs, tokens_per_seq, num_heads, pool_size) -> kda_decode_shape_t:
+    return kda_decode_shape_t(int(num_seqs), int(tokens_per_seq), int(num_heads), int(pool_size))
+
+
+def kda_decode(q, k, v, g, beta, scale, state, state_indices, shape, out, step_states,
+               device_status, flags, stream) -> int:
+    """All pointer arguments are integers (device addresses) or None."""
+    return int(lib.kda_decode(q, k, v, g, beta, ctypes.c_float(scale), state, state_indices,
+                              ctypes.byref(shape), out, step_states, device_status,
+                              int(flags), stream))

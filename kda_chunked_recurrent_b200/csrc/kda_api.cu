@@ -28,6 +28,12 @@ __global__ void kda_fused_kernel(const KdaParams p, const __grid_constant__ Spli
 namespace prep { extern const uint32_t kSmemAllocBytes; }
 namespace rec { extern const uint32_t kSmemAllocBytes; extern const int kThreadsPerCta; }
 namespace fused { extern const uint32_t kSmemAllocBytes; extern const int kThreadsPerCta; }
+__global__ void kda_token_kernel(const TokenParams p);
+namespace tok {
+extern const uint32_t kSmemAllocBytes;
+extern const int kThreadsPerCta;
+extern const int kCtasPerUnit;
+}
 }  // namespace kda
 
 using namespace kda;
@@ -76,7 +82,7 @@ struct Resolved {
 
 kda_status_t check_options(const kda_options_t* o) {
   if (!o) return KDA_OK;
-  if (o->variant < KDA_VARIANT_AUTO || o->variant > KDA_VARIANT_HYBRID) return KDA_ERR_BAD_OPTION;
+  if (o->variant < KDA_VARIANT_AUTO || o->variant > KDA_VARIANT_TOKEN) return KDA_ERR_BAD_OPTION;
   if (o->flags & ~(static_cast<uint32_t>(KDA_FLAG_VALIDATE | KDA_FLAG_TEST_FORCE_TIMEOUT |
                                          KDA_FLAG_CU_SEQLENS_I64)))
     return KDA_ERR_BAD_OPTION;
@@ -101,6 +107,8 @@ int sm_count();
 // The fused launch keeps at least this many SMs for its prepare CTAs, which run
 // one prepare group each up to kFusedOneGroupMaxChains chains and two above.
 constexpr int kFusedMinPrepCtas = 16;
+// AUTO takes the token variant when no sequence is longer than this
+constexpr int64_t kTokenMaxLen = KDA_TOKEN_AUTO_MAX_LEN;
 constexpr int kFusedOneGroupMaxChains = 16;
 
 // Per-shape variant table, from CUDA-event timings on one B200 (1965 MHz, ms per
@@ -112,15 +120,19 @@ constexpr int kFusedOneGroupMaxChains = 16;
 // behind the recurrence chains while the chains (one SM each) leave enough SMs to
 // its prepare groups; the hybrid runs most of the prepare work first on every SM
 // and hides only the last chunks; both need sequences long enough to overlap.
+// The token variant (one token at a time, state slice in registers) wins while
+// every sequence is short: TOKEN_TABLE_NOTE.
 struct VariantRule {
   int64_t max_chains;   // N H at most this
   int64_t min_chunks;   // and at least this many chunks in the longest sequence
+  int64_t max_len;      // and no sequence longer than this
   int variant;          // -> this variant
 };
 constexpr VariantRule kVariantTable[] = {
-    {56, 32, KDA_VARIANT_FUSED},
-    {INT64_MAX, 64, KDA_VARIANT_HYBRID},
-    {INT64_MAX, 0, KDA_VARIANT_SPLIT},
+    {INT64_MAX, 0, kTokenMaxLen, KDA_VARIANT_TOKEN},
+    {56, 32, INT64_MAX, KDA_VARIANT_FUSED},
+    {INT64_MAX, 64, INT64_MAX, KDA_VARIANT_HYBRID},
+    {INT64_MAX, 0, INT64_MAX, KDA_VARIANT_SPLIT},
 };
 
 bool fused_eligible(const kda_shape_t* s) {
@@ -134,8 +146,9 @@ int choose_variant(const kda_shape_t* s, const kda_options_t* o) {
   if (o && o->variant != KDA_VARIANT_AUTO) return o->variant;
   const int64_t chains = static_cast<int64_t>(s->num_seqs) * s->num_heads;
   const int64_t chunks = max_chunks_per_seq(s, false, false);
+  const int64_t len = s->max_seqlen > 0 ? s->max_seqlen : s->total_tokens;
   for (const VariantRule& rule : kVariantTable)
-    if (chains <= rule.max_chains && chunks >= rule.min_chunks) {
+    if (chains <= rule.max_chains && chunks >= rule.min_chunks && len <= rule.max_len) {
       if ((rule.variant == KDA_VARIANT_FUSED || rule.variant == KDA_VARIANT_HYBRID) &&
           !fused_eligible(s))
         continue;
@@ -169,7 +182,10 @@ Resolved resolve(const kda_shape_t* s, bool fixed, bool ckpt, const kda_options_
   Resolved r{};
   r.variant = choose_variant(s, o);
   r.fixed = fixed;
-  r.lay = make_layout(s->num_seqs, s->total_tokens, s->num_heads, fixed, true, ckpt);
+  // the token variant needs no per-record tiles; AUTO sizes for the largest variant
+  // so that one workspace serves whatever the table picks
+  const bool tiles = !(o && o->variant == KDA_VARIANT_TOKEN);
+  r.lay = make_layout(s->num_seqs, s->total_tokens, s->num_heads, fixed, tiles, ckpt);
   return r;
 }
 
@@ -249,6 +265,7 @@ const char* kda_status_string(int s) {
     case KDA_ERR_BAD_CU_SEQLENS: return "cu_seqlens invalid (validate mode)";
     case KDA_ERR_BAD_CKPT_OFFSET: return "checkpoint offset outside its sequence (validate mode)";
     case KDA_ERR_TIMEOUT: return "a bounded on-device wait timed out";
+    case KDA_ERR_BAD_STATE_INDEX: return "a state index at or above the pool size";
     default: return "unknown status";
   }
 }
@@ -284,7 +301,12 @@ kda_status_t kda_prefill_describe(const kda_shape_t* shape, int has_ckpt,
   }
   const Resolved r = resolve(shape, false, has_ckpt != 0, options);
   const long long chains = static_cast<long long>(shape->num_seqs) * shape->num_heads;
-  if (r.variant == KDA_VARIANT_HYBRID) {
+  if (r.variant == KDA_VARIANT_TOKEN) {
+    snprintf(buf, n,
+             "variant=token grid=%lldx%d (%d CTAs per (sequence, head), 32 value columns "
+             "each) workspace_bytes=%zu",
+             chains * tok::kCtasPerUnit, tok::kThreadsPerCta, tok::kCtasPerUnit, r.lay.total);
+  } else if (r.variant == KDA_VARIANT_HYBRID) {
     const int64_t jmax = max_chunks_per_seq(shape, false, has_ckpt != 0);
     const int64_t tail = hybrid_tail_chunks(jmax, chains);
     snprintf(buf, n,
@@ -441,11 +463,41 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
   auto mark = [&](int i) {
     if (ev && ev[i]) cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), s);
   };
-  if (!fixed || ckpt || (flags & KDA_FLAG_VALIDATE)) {
+  // metadata kernel: INT64 narrowing, validation, and (chunked variants) the chunk table
+  const bool sched = (r.variant == KDA_VARIANT_TOKEN)
+                         ? (cu64 || (flags & KDA_FLAG_VALIDATE))
+                         : (!fixed || ckpt || (flags & KDA_FLAG_VALIDATE));
+  if (sched) {
     kda_schedule_kernel<<<1, 1024, 0, s>>>(p);
     mark(0);
   }
-  if (r.variant == KDA_VARIANT_FUSED || r.variant == KDA_VARIANT_HYBRID) {
+  if (r.variant == KDA_VARIANT_TOKEN) {
+    mark(1);
+    TokenParams tp{};
+    tp.q = p.q;
+    tp.k = p.k;
+    tp.v = p.v;
+    tp.g = p.g;
+    tp.beta = p.beta;
+    tp.scale = scale;
+    tp.src = h0;
+    tp.dst = ht;
+    tp.cu_seqlens = p.cu_seqlens;
+    tp.fixed_len = p.fixed_len;
+    tp.ckpt_offsets = ckpt_offsets;
+    tp.ckpt = ckpt_state;
+    tp.out = p.out;
+    tp.N = p.N;
+    tp.T = p.T;
+    tp.H = p.H;
+    tp.ws = p.ws;
+    tp.status = reinterpret_cast<int32_t*>(p.ws);
+    tp.flags = flags;
+    tp.wait_budget = p.wait_budget;
+    kda_token_kernel<<<static_cast<unsigned>(N * H * tok::kCtasPerUnit), tok::kThreadsPerCta,
+                       tok::kSmemAllocBytes, s>>>(tp);
+    mark(2);
+  } else if (r.variant == KDA_VARIANT_FUSED || r.variant == KDA_VARIANT_HYBRID) {
     const int64_t jmax = max_chunks_per_seq(shape, fixed, ckpt);
     int64_t j0 = 0;
     if (r.variant == KDA_VARIANT_HYBRID && T > 0) {
@@ -493,6 +545,73 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
                             rec::kSmemAllocBytes, s>>>(p, maps);
     mark(2);
   }
+  if (cudaGetLastError() != cudaSuccess) return KDA_ERR_LAUNCH_FAILED;
+  return KDA_OK;
+}
+
+kda_status_t kda_decode(const void* q, const void* k, const void* v, const float* g,
+                        const void* beta, float scale, float* state,
+                        const int32_t* state_indices, const kda_decode_shape_t* shape,
+                        void* out, float* step_states, int32_t* device_status, uint32_t flags,
+                        void* stream) {
+  if (!shape) return KDA_ERR_NULL_ARG;
+  if (flags & ~static_cast<uint32_t>(KDA_DECODE_KEEP_STATE)) return KDA_ERR_BAD_OPTION;
+  const int64_t N = shape->num_seqs, T = shape->tokens_per_seq, H = shape->num_heads,
+                P = shape->pool_size;
+  if (N < 1 || T < 1 || H < 1 || P < 1) return KDA_ERR_BAD_SHAPE;
+  if (!state_indices && P < N) return KDA_ERR_BAD_SHAPE;
+  // 32-bit token rows and grid
+  if (N * T * H * 128 >= (int64_t(1) << 31) || N * H * tok::kCtasPerUnit >= (int64_t(1) << 31))
+    return KDA_ERR_BAD_SHAPE;
+  if (!q || !k || !v || !g || !beta || !state || !out) return KDA_ERR_NULL_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(g, 16) ||
+      !aligned(out, 16) || !aligned(beta, 2) || !aligned(state, 16) ||
+      !aligned(step_states, 16) || !aligned(state_indices, 4) || !aligned(device_status, 4))
+    return KDA_ERR_MISALIGNED;
+  const size_t tok16 = static_cast<size_t>(N * T * H * 128 * 2);
+  const size_t st1 = static_cast<size_t>(H * 128 * 128 * 4);   // one slot, all heads
+  const Range rq = rng(q, tok16), rk = rng(k, tok16), rv = rng(v, tok16),
+              rg = rng(g, tok16 * 2), rb = rng(beta, static_cast<size_t>(N * T * H * 2)),
+              ri = rng(state_indices, static_cast<size_t>(N * 4)),
+              rs = rng(state, st1 * static_cast<size_t>(P)), ro = rng(out, tok16),
+              rst = rng(step_states, st1 * static_cast<size_t>(N * T)),
+              rds = rng(device_status, 4);
+  const Range inputs[] = {rq, rk, rv, rg, rb, ri};
+  const Range outputs[] = {rs, ro, rst, rds};
+  for (const Range& o : outputs)
+    for (const Range& in : inputs)
+      if (overlap(o, in)) return KDA_ERR_OUT_ALIAS;
+  for (int i = 0; i < 4; ++i)
+    for (int j = i + 1; j < 4; ++j)
+      if (overlap(outputs[i], outputs[j])) return KDA_ERR_OUT_ALIAS;
+  kda_status_t st = device_check();
+  if (st != KDA_OK) return st;
+
+  TokenParams tp{};
+  tp.q = static_cast<const uint16_t*>(q);
+  tp.k = static_cast<const uint16_t*>(k);
+  tp.v = static_cast<const uint16_t*>(v);
+  tp.g = g;
+  tp.beta = static_cast<const uint16_t*>(beta);
+  tp.scale = scale;
+  tp.src = state;
+  tp.dst = (flags & KDA_DECODE_KEEP_STATE) ? nullptr : state;
+  tp.slot = state_indices;
+  tp.pool = static_cast<int32_t>(P);
+  tp.cu_seqlens = nullptr;
+  tp.fixed_len = static_cast<int32_t>(T);
+  tp.steps = step_states;
+  tp.out = static_cast<uint16_t*>(out);
+  tp.N = static_cast<int32_t>(N);
+  tp.T = static_cast<int32_t>(N * T);
+  tp.H = static_cast<int32_t>(H);
+  tp.status = device_status;
+  tp.flags = 0;
+  tp.wait_budget = kDefaultWaitBudget;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  (void)cudaGetLastError();
+  kda_token_kernel<<<static_cast<unsigned>(N * H * tok::kCtasPerUnit), tok::kThreadsPerCta,
+                     tok::kSmemAllocBytes, s>>>(tp);
   if (cudaGetLastError() != cudaSuccess) return KDA_ERR_LAUNCH_FAILED;
   return KDA_OK;
 }

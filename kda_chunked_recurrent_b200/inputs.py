@@ -121,3 +121,37 @@ def workload(name: str) -> KDAInputs:
     lens = w["seqlens"] if w.get("seqlens") is not None else ragged_lengths(w["ragged"])
     return make_inputs(lens, w["H"], w["seed"], with_h0=w.get("h0", False),
                        with_ckpt=w.get("ckpt", False), fixed_layout=w.get("fixed", False))
+
+
+@dataclass
+class DecodeInputs:
+    """N sequences of T new tokens each over a pool of P states."""
+    q: torch.Tensor              # [N, T, H, 128] bf16
+    k: torch.Tensor              # [N, T, H, 128] bf16
+    v: torch.Tensor              # [N, T, H, 128] bf16
+    g: torch.Tensor              # [N, T, H, 128] fp32
+    beta: torch.Tensor           # [N, T, H] bf16
+    scale: float
+    pool: torch.Tensor           # [P, H, 128, 128] fp32
+    state_indices: Optional[torch.Tensor]   # [N] int32 (negative = padding) or None
+
+
+def make_decode_inputs(num_seqs: int, tokens: int, num_heads: int, pool_size: int, seed: int, *,
+                       indices: bool = True, pad_every: int = 0, pool_std: float = 0.1
+                       ) -> DecodeInputs:
+    """Token rows as in make_inputs; a pool of N(0, pool_std) states; the slots of the
+    sequences a random injective map into the pool (every ``pad_every``-th entry -1)."""
+    base = make_inputs([tokens] * num_seqs, num_heads, seed, fixed_layout=True)
+    N, T, H = int(num_seqs), int(tokens), int(num_heads)
+    gen = torch.Generator().manual_seed(int(seed) + 7)
+    pool = pool_std * torch.randn(int(pool_size), H, DK, DV, generator=gen, dtype=torch.float32)
+    idx = None
+    if indices:
+        assert pool_size >= N
+        idx = torch.randperm(int(pool_size), generator=gen)[:N].to(torch.int32)
+        if pad_every > 0:
+            idx[::pad_every] = -1
+    shp = (N, T, H)
+    return DecodeInputs(q=base.q.view(*shp, DK), k=base.k.view(*shp, DK), v=base.v.view(*shp, DV),
+                        g=base.g.view(*shp, DK), beta=base.beta.view(*shp), scale=base.scale,
+                        pool=pool, state_indices=idx)

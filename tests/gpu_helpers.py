@@ -82,3 +82,34 @@ def assert_parity(m):
         assert m["ht_rel"] <= S_TOL, m
     if "ckpt_rel" in m:
         assert m["ckpt_rel"] <= S_TOL, m
+
+
+def decode_oracle(dinp, steps: bool = False):
+    """FP64 oracle for kda_decode: every live sequence (slot in [0, P)) is a prefill
+    of T tokens from its pool slot.  Returns dict with "live" (sequence indices),
+    "o" [L, T, H, V], "ht" [L, H, K, V] and, with ``steps``, "steps" [L, T, H, K, V]
+    (the oracle's checkpoint at every prefix length 1..T)."""
+    N, T, H = (int(x) for x in dinp.q.shape[:3])
+    P = int(dinp.pool.shape[0])
+    idx = list(range(N)) if dinp.state_indices is None else dinp.state_indices.tolist()
+    live = [n for n in range(N) if 0 <= idx[n] < P]
+    L = len(live)
+    res = {"live": live}
+    if L == 0:
+        return res
+    sel = lambda x: np.ascontiguousarray(x.double().numpy()[live].reshape(L * T, H, -1))
+    q, k, v, g = sel(dinp.q), sel(dinp.k), sel(dinp.v), sel(dinp.g)
+    beta = np.ascontiguousarray(dinp.beta.double().numpy()[live].reshape(L * T, H))
+    h0 = np.ascontiguousarray(dinp.pool.double().numpy()[[idx[n] for n in live]])
+    cu = np.arange(L + 1, dtype=np.int64) * T
+    o, ht, _ = oracle.prefill_f64(q, k, v, g, beta, dinp.scale, cu, h0)
+    res["o"] = o.reshape(L, T, H, -1)
+    res["ht"] = ht
+    if steps:
+        st = np.zeros((L, T, H, 128, 128))
+        for tau in range(1, T + 1):
+            _, _, ck = oracle.prefill_f64(q, k, v, g, beta, dinp.scale, cu, h0,
+                                          np.full(L, tau, np.int64))
+            st[:, tau - 1] = ck
+        res["steps"] = st
+    return res

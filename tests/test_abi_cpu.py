@@ -32,7 +32,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_status_strings_cover_all_codes():
-    for code in (0, 1, 2, 3, 4, 5, 6, 7, 8, 9, 10, 16, 17, 18):
+    for code in (0, 1, 2, 3, 4, 5, 6, 7, 8, 9, 10, 16, 17, 18, 19):
         s = capi.kda_status_string(code)
         assert s and s != "unknown status"
     assert capi.kda_status_string(12345) == "unknown status"
