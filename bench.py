@@ -266,6 +266,15 @@ def run_reference(args, rank, world):
     return 0
 
 
+TOKEN_SOURCES = ["kda_token.cu", "kda_token.cuh", "kda_common.cuh", "sm100_primitives.cuh"]
+
+
+def token_kernel_name(capi, N, H):
+    """Which per-token kernel the library launches for N x H units (its describe line)."""
+    d = capi.kda_prefill_describe(capi.make_shape(N, N, H, 1), False, {"variant": 4})
+    return "kda_token_wide_kernel" if "(wide" in d else "kda_token_narrow_kernel"
+
+
 DECODE_METRIC = "KDA decode Mtokens·heads/s at 1 B200 (state pool, one launch per step)"
 
 
@@ -336,9 +345,10 @@ def run_decode(args):
     value = units * world / (ms / 1e3) / 1e6
     peaks, peak_src = load_peaks()
     achieved = algo_bytes / (kern_ms / 1e3) / 1e9
-    roof = {"kernel": "kda_token_kernel", "bound": "hbm", "achieved": round(achieved, 1),
+    kname = token_kernel_name(capi, N, H)
+    roof = {"kernel": kname, "bound": "hbm", "achieved": round(achieved, 1),
             "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-            "traffic": ncu_traffic("kda_token_kernel", f"decode_{N}_{T}_{H}", units),
+            "traffic": ncu_traffic(kname, f"decode_N{N}_T{T}_H{H}", units),
             "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
             else "fallback 6650 GB/s", "kernel_ms": round(kern_ms, 4),
             "algorithmic_bytes": int(algo_bytes)}
@@ -556,8 +566,9 @@ def main():
         }
     elif variant == "token":
         kernels = {
-            "kda_token_kernel": (prep_ms + rec_ms, PATH_BYTES_PER_TOKHEAD * units + state_io,
-                                 ["kda_token.cu", "kda_common.cuh", "sm100_primitives.cuh"]),
+            token_kernel_name(capi, N, H): (prep_ms + rec_ms,
+                                            PATH_BYTES_PER_TOKHEAD * units + state_io,
+                                            TOKEN_SOURCES),
         }
     elif variant == "fused":
         # one launch moves both halves' bytes (the records still go through HBM/L2)

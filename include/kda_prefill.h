@@ -97,12 +97,13 @@ typedef enum {
                             the fused launch, whose prepare CTAs make the last chunks while
                             its recurrence CTAs already run.  Same SM condition as FUSED;
                             AUTO picks it above 56 chains of at least 64 chunks.          */
-  KDA_VARIANT_TOKEN = 4   /* the recurrence one token at a time: 4 CTAs per (sequence,
-                            head), each holding 32 value columns of the state in registers;
+  KDA_VARIANT_TOKEN = 4   /* the recurrence one token at a time with the state in
+                            registers: 4 CTAs of 32 value columns per (sequence, head)
+                            below 128 units, one CTA of 128 columns per unit from 128 on;
                             no chunk records, workspace = header only.  AUTO picks it when
-                            max_seqlen (else T_total) is at most KDA_TOKEN_AUTO_MAX_LEN.  */
+                            max_seqlen (else T_total) is at most 16, or at most 32 with
+                            N*H <= 16.                                                   */
 } kda_variant_t;
-#define KDA_TOKEN_AUTO_MAX_LEN 64
 
 enum {
   KDA_FLAG_VALIDATE = 1u << 0,       /* kernels check cu_seqlens / ckpt_offsets values  */
@@ -271,7 +272,9 @@ kda_status_t kda_prefill_noalloc(const void* q, const void* k, const void* v, co
  *   device_status  INT32 device word, 4-byte aligned, or NULL: the first device
  *             error is stored there with atomicCAS from KDA_OK (the caller clears
  *             it); without it device errors are not reported.
- *   flags     KDA_DECODE_KEEP_STATE: the pool is read only.
+ *   flags     KDA_DECODE_KEEP_STATE: the pool is read only.  KDA_DECODE_NARROW /
+ *             KDA_DECODE_WIDE force the kernel shape (timing aid; the default
+ *             picks by the number of (sequence, head) units).
  *   stream    cudaStream_t.
  *
  * Outputs (state, out, step_states, device_status) must not overlap the inputs
@@ -285,7 +288,13 @@ typedef struct {
   int32_t pool_size;      /* P >= 1 state slots in `state`                        */
 } kda_decode_shape_t;
 
-enum { KDA_DECODE_KEEP_STATE = 1u << 0 };
+enum {
+  KDA_DECODE_KEEP_STATE = 1u << 0, /* the pool is read only                              */
+  KDA_DECODE_NARROW = 1u << 1,     /* force 4 CTAs of 32 value columns per (sequence,
+                                      head) (default below 128 units)                   */
+  KDA_DECODE_WIDE = 1u << 2        /* force 1 CTA of 128 value columns per unit (default
+                                      from 128 units); not together with NARROW         */
+};
 
 kda_status_t kda_decode(const void* q, const void* k, const void* v, const float* g,
                         const void* beta, float scale, float* state,

@@ -16,7 +16,8 @@ CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libkda_prefill.so")
 SOURCES = ["kda_api.cu", "kda_schedule.cu", "kda_prepare.cu", "kda_recurrence.cu",
            "kda_fused.cu", "kda_token.cu", "kda_noalloc.cu"]
-HEADERS = ["kda_common.cuh", "sm100_primitives.cuh", "kda_prepare.cuh", "kda_recurrence.cuh"]
+HEADERS = ["kda_common.cuh", "sm100_primitives.cuh", "kda_prepare.cuh", "kda_recurrence.cuh",
+           "kda_token.cuh"]
 
 
 def nvcc_path() -> str:

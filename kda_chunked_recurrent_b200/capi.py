@@ -34,8 +34,9 @@ KDA_VARIANT_SPLIT = 1
 KDA_VARIANT_FUSED = 2
 KDA_VARIANT_HYBRID = 3
 KDA_VARIANT_TOKEN = 4
-KDA_TOKEN_AUTO_MAX_LEN = 64
 KDA_DECODE_KEEP_STATE = 1
+KDA_DECODE_NARROW = 2
+KDA_DECODE_WIDE = 4
 KDA_FLAG_VALIDATE = 1
 KDA_FLAG_TEST_FORCE_TIMEOUT = 2
 KDA_FLAG_CU_SEQLENS_I64 = 4

@@ -18,6 +18,7 @@
 
 #include "../../include/kda_prefill.h"
 #include "kda_common.cuh"
+#include "kda_token.cuh"
 
 namespace kda {
 __global__ void kda_schedule_kernel(const KdaParams p);
@@ -28,11 +29,12 @@ __global__ void kda_fused_kernel(const KdaParams p, const __grid_constant__ Spli
 namespace prep { extern const uint32_t kSmemAllocBytes; }
 namespace rec { extern const uint32_t kSmemAllocBytes; extern const int kThreadsPerCta; }
 namespace fused { extern const uint32_t kSmemAllocBytes; extern const int kThreadsPerCta; }
-__global__ void kda_token_kernel(const TokenParams p);
+__global__ void kda_token_narrow_kernel(const TokenParams p);
+__global__ void kda_token_wide_kernel(const TokenParams p);
 namespace tok {
-extern const uint32_t kSmemAllocBytes;
+extern const uint32_t kSmemNarrow;
+extern const uint32_t kSmemWide;
 extern const int kThreadsPerCta;
-extern const int kCtasPerUnit;
 }
 }  // namespace kda
 
@@ -107,8 +109,41 @@ int sm_count();
 // The fused launch keeps at least this many SMs for its prepare CTAs, which run
 // one prepare group each up to kFusedOneGroupMaxChains chains and two above.
 constexpr int kFusedMinPrepCtas = 16;
-// AUTO takes the token variant when no sequence is longer than this
-constexpr int64_t kTokenMaxLen = KDA_TOKEN_AUTO_MAX_LEN;
+// Token kernel shape: 4 narrow CTAs (32 value columns each) per (sequence, head)
+// below this many units, one wide CTA (all 128 columns) per unit from it on.
+// Measured (kda_decode, T = 1, H = 12, ms narrow / wide): 48 units 0.0097 / 0.0104,
+// 96 units 0.0103 / 0.0105, 144 units 0.0128 / 0.0116, 768 units 0.0311 / 0.0272,
+// 3072 units 0.0956 / 0.0744.
+constexpr int64_t kTokenWideMinUnits = 128;
+
+bool token_wide(int64_t units, uint32_t force) {
+  if (force & KDA_DECODE_NARROW) return false;
+  if (force & KDA_DECODE_WIDE) return true;
+  return units >= kTokenWideMinUnits;
+}
+
+// Launch the per-token kernel for `units` (sequence, head) pairs.
+kda_status_t launch_token(const TokenParams& tp, int64_t units, bool wide, cudaStream_t s) {
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    cudaError_t e1 = cudaFuncSetAttribute(kda_token_narrow_kernel,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          tok::kSmemNarrow);
+    cudaError_t e2 = cudaFuncSetAttribute(kda_token_wide_kernel,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          tok::kSmemWide);
+    attr_err = e1 != cudaSuccess ? e1 : e2;
+  });
+  if (attr_err != cudaSuccess) return KDA_ERR_LAUNCH_FAILED;
+  if (wide)
+    kda_token_wide_kernel<<<static_cast<unsigned>(units), tok::kThreadsPerCta, tok::kSmemWide,
+                            s>>>(tp);
+  else
+    kda_token_narrow_kernel<<<static_cast<unsigned>(units * 4), tok::kThreadsPerCta,
+                              tok::kSmemNarrow, s>>>(tp);
+  return KDA_OK;
+}
 constexpr int kFusedOneGroupMaxChains = 16;
 
 // Per-shape variant table, from CUDA-event timings on one B200 (1965 MHz, ms per
@@ -121,7 +156,10 @@ constexpr int kFusedOneGroupMaxChains = 16;
 // its prepare groups; the hybrid runs most of the prepare work first on every SM
 // and hides only the last chunks; both need sequences long enough to overlap.
 // The token variant (one token at a time, state slice in registers) wins while
-// every sequence is short: TOKEN_TABLE_NOTE.
+// every sequence is short.  Measured ms per call, split / token, H = 12: N = 1 T = 16
+// 0.025 / 0.015, T = 32 0.024 / 0.022, T = 64 0.024 / 0.037; N = 8 T = 16 0.026 /
+// 0.022, T = 32 0.027 / 0.037; N = 32 T = 8 0.048 / 0.031, T = 16 0.048 / 0.049;
+// N = 256 T = 8 0.258 / 0.156, T = 16 0.261 / 0.276.
 struct VariantRule {
   int64_t max_chains;   // N H at most this
   int64_t min_chunks;   // and at least this many chunks in the longest sequence
@@ -129,7 +167,8 @@ struct VariantRule {
   int variant;          // -> this variant
 };
 constexpr VariantRule kVariantTable[] = {
-    {INT64_MAX, 0, kTokenMaxLen, KDA_VARIANT_TOKEN},
+    {16, 0, 32, KDA_VARIANT_TOKEN},
+    {INT64_MAX, 0, 16, KDA_VARIANT_TOKEN},
     {56, 32, INT64_MAX, KDA_VARIANT_FUSED},
     {INT64_MAX, 64, INT64_MAX, KDA_VARIANT_HYBRID},
     {INT64_MAX, 0, INT64_MAX, KDA_VARIANT_SPLIT},
@@ -302,10 +341,12 @@ kda_status_t kda_prefill_describe(const kda_shape_t* shape, int has_ckpt,
   const Resolved r = resolve(shape, false, has_ckpt != 0, options);
   const long long chains = static_cast<long long>(shape->num_seqs) * shape->num_heads;
   if (r.variant == KDA_VARIANT_TOKEN) {
+    const bool wide = token_wide(chains, 0);
     snprintf(buf, n,
-             "variant=token grid=%lldx%d (%d CTAs per (sequence, head), 32 value columns "
+             "variant=token grid=%lldx%d (%s: %d CTA(s) per (sequence, head), %d value columns "
              "each) workspace_bytes=%zu",
-             chains * tok::kCtasPerUnit, tok::kThreadsPerCta, tok::kCtasPerUnit, r.lay.total);
+             chains * (wide ? 1 : 4), tok::kThreadsPerCta, wide ? "wide" : "narrow",
+             wide ? 1 : 4, wide ? 128 : 32, r.lay.total);
   } else if (r.variant == KDA_VARIANT_HYBRID) {
     const int64_t jmax = max_chunks_per_seq(shape, false, has_ckpt != 0);
     const int64_t tail = hybrid_tail_chunks(jmax, chains);
@@ -494,8 +535,8 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
     tp.status = reinterpret_cast<int32_t*>(p.ws);
     tp.flags = flags;
     tp.wait_budget = p.wait_budget;
-    kda_token_kernel<<<static_cast<unsigned>(N * H * tok::kCtasPerUnit), tok::kThreadsPerCta,
-                       tok::kSmemAllocBytes, s>>>(tp);
+    st = launch_token(tp, N * H, token_wide(N * H, 0), s);
+    if (st != KDA_OK) return st;
     mark(2);
   } else if (r.variant == KDA_VARIANT_FUSED || r.variant == KDA_VARIANT_HYBRID) {
     const int64_t jmax = max_chunks_per_seq(shape, fixed, ckpt);
@@ -555,13 +596,16 @@ kda_status_t kda_decode(const void* q, const void* k, const void* v, const float
                         void* out, float* step_states, int32_t* device_status, uint32_t flags,
                         void* stream) {
   if (!shape) return KDA_ERR_NULL_ARG;
-  if (flags & ~static_cast<uint32_t>(KDA_DECODE_KEEP_STATE)) return KDA_ERR_BAD_OPTION;
+  if (flags & ~static_cast<uint32_t>(KDA_DECODE_KEEP_STATE | KDA_DECODE_NARROW |
+                                     KDA_DECODE_WIDE))
+    return KDA_ERR_BAD_OPTION;
+  if ((flags & KDA_DECODE_NARROW) && (flags & KDA_DECODE_WIDE)) return KDA_ERR_BAD_OPTION;
   const int64_t N = shape->num_seqs, T = shape->tokens_per_seq, H = shape->num_heads,
                 P = shape->pool_size;
   if (N < 1 || T < 1 || H < 1 || P < 1) return KDA_ERR_BAD_SHAPE;
   if (!state_indices && P < N) return KDA_ERR_BAD_SHAPE;
   // 32-bit token rows and grid
-  if (N * T * H * 128 >= (int64_t(1) << 31) || N * H * tok::kCtasPerUnit >= (int64_t(1) << 31))
+  if (N * T * H * 128 >= (int64_t(1) << 31) || N * H * 4 >= (int64_t(1) << 31))
     return KDA_ERR_BAD_SHAPE;
   if (!q || !k || !v || !g || !beta || !state || !out) return KDA_ERR_NULL_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(g, 16) ||
@@ -610,8 +654,8 @@ kda_status_t kda_decode(const void* q, const void* k, const void* v, const float
   tp.wait_budget = kDefaultWaitBudget;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   (void)cudaGetLastError();
-  kda_token_kernel<<<static_cast<unsigned>(N * H * tok::kCtasPerUnit), tok::kThreadsPerCta,
-                     tok::kSmemAllocBytes, s>>>(tp);
+  st = launch_token(tp, N * H, token_wide(N * H, flags), s);
+  if (st != KDA_OK) return st;
   if (cudaGetLastError() != cudaSuccess) return KDA_ERR_LAUNCH_FAILED;
   return KDA_OK;
 }

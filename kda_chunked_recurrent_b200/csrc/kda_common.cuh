@@ -141,33 +141,6 @@ enum : int32_t {
   kStatusBadCuSeqlens = 16,
   kStatusBadCkptOffset = 17,
   kStatusTimeout = 18,
-  kStatusBadStateIndex = 19,
-};
-
-// Parameters of the per-token kernel (short sequences through kda_prefill, and
-// kda_decode).  A CTA owns 32 value columns of one (sequence, head).
-struct TokenParams {
-  const uint16_t* q;
-  const uint16_t* k;
-  const uint16_t* v;
-  const float* g;
-  const uint16_t* beta;
-  float scale;
-  const float* src;              // state read first, [slots][H][128][128]; NULL = zero state
-  float* dst;                    // state written last (same indexing as src); NULL = none
-  const int32_t* slot;           // state slot of each sequence; NULL = the sequence index
-  int32_t pool;                  // number of slots when slot != NULL
-  const int32_t* cu_seqlens;     // NULL: fixed layout of fixed_len tokens per sequence
-  int32_t fixed_len;
-  const int32_t* ckpt_offsets;   // NULL: no checkpoint
-  float* ckpt;                   // [N][H][128][128]
-  float* steps;                  // [N][fixed_len][H][128][128] state after every token, or NULL
-  uint16_t* out;
-  int32_t N, T, H;
-  uint8_t* ws;                   // prefill workspace (metadata check of validate mode) or NULL
-  int32_t* status;               // sticky status word, or NULL
-  uint32_t flags;
-  long long wait_budget;         // clock cycles per bounded wait; < 0 forces a timeout
 };
 
 enum : uint32_t { kFlagValidate = 1u, kFlagForceTimeout = 2u, kFlagCu64 = 4u };

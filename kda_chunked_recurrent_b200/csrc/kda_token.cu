@@ -7,15 +7,21 @@
 //   S  = S' + k_t u^T
 //   o_t = scale S^T q_t = scale (S'^T q_t + u (k_t . q_t))
 // Every value column of S evolves on its own given (k_t, q_t, g_t, beta_t), so a
-// CTA owns 32 columns of one (sequence, head) and keeps that 128 x 32 slice in
+// CTA owns a slice of the columns of one (sequence, head) and keeps it in
 // registers for the whole sequence: warp w holds key rows [16 w, 16 w + 16), lane
-// l holds column l of the slice.  Per token a thread folds its 16 rows into two
-// partial column sums (S'^T k and S'^T q) and one partial k.q; one barrier makes
-// the eight warps' partials visible, after which every thread has u and o_t for
-// its column and applies the rank-1 update to its rows.  The state is read from
-// HBM once and written once; tokens are staged 16 at a time into shared memory by
-// the copy engine (cp.async.bulk per token row, completion on an mbarrier), one
-// block ahead of the arithmetic, and exp(g) is taken once per staged element.
+// l holds kCPT adjacent columns.  Two shapes are instantiated:
+//   kCPT = 1  32 columns per CTA, 4 CTAs per (sequence, head): shortest chain per
+//             token, for few (sequence, head) units;
+//   kCPT = 4  128 columns per CTA (float4 state rows), 1 CTA per unit: fewer
+//             instructions per column and 64 KB of state in flight per CTA, for
+//             many units (decode of large batches).
+// Per token a thread folds its 16 rows into partial column sums of S'^T k and
+// S'^T q; one barrier makes the eight warps' partials visible, after which every
+// thread has u and o_t for its columns and applies the rank-1 update.  The state
+// is read from HBM once and written once.  Tokens are staged 16 at a time into
+// shared memory by the copy engine (cp.async.bulk per token row, completion on an
+// mbarrier), one block ahead of the arithmetic; once a block lands, exp(g), the
+// FP32 k and q rows and k.q are formed once per block and shared by all columns.
 //
 // Decode over a slot-indexed state pool and per-token state export follow the
 // FlashInfer KDA decode entry (SGLang kda_flashinfer.py "FlashInferKDAKernel":
@@ -23,68 +29,108 @@
 #include <cstdint>
 
 #include "kda_common.cuh"
+#include "kda_token.cuh"
 #include "sm100_primitives.cuh"
 
 namespace kda {
 namespace tok {
 
-constexpr int kCols = 32;                  // value columns per CTA (one per lane)
-constexpr int kSlices = kD / kCols;        // CTAs per (sequence, head)
 constexpr int kWarps = 8;
 constexpr int kRows = kD / kWarps;         // key rows per warp
 constexpr int kThreads = kWarps * 32;
 constexpr int kBlk = 16;                   // tokens per staged block
-// one staged block: k, q [16][128] bf16; g -> exp(g) [16][128] f32; this CTA's
-// v columns [16][32] bf16; beta [16] f32
-constexpr uint32_t kOffK = 0;
-constexpr uint32_t kOffQ = kOffK + kBlk * kD * 2;
-constexpr uint32_t kOffE = kOffQ + kBlk * kD * 2;
-constexpr uint32_t kOffV = kOffE + kBlk * kD * 4;
-constexpr uint32_t kOffB = kOffV + kBlk * kCols * 2;
-constexpr uint32_t kBufBytes = (kOffB + kBlk * 4 + 127) / 128 * 128;
-constexpr uint32_t kTokBytes = kD * 2 + kD * 2 + kD * 4 + kCols * 2;   // copied per token
-constexpr long long kDrainBudget = 2000000000LL;                     // clock cycles
-static_assert(kRows == 16, "the unpacking below assumes 16 rows per warp");
+constexpr long long kDrainBudget = 2000000000LL;   // clock cycles
+static_assert(kRows == 16, "16 key rows per warp");
 
-__device__ __forceinline__ void unpack8(const uint4& w, float* f) {
-  const uint32_t x[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    f[2 * i] = __uint_as_float(x[i] << 16);
-    f[2 * i + 1] = __uint_as_float(x[i] & 0xffff0000u);
+constexpr uint32_t align128(uint32_t x) { return (x + 127u) / 128u * 128u; }
+
+template <int kCPT>
+struct Cfg {
+  static constexpr int kCols = 32 * kCPT;          // value columns per CTA
+  static constexpr int kSlices = kD / kCols;       // CTAs per (sequence, head)
+  // staged block, two buffers: k, q [16][128] bf16; g [16][128] f32 (exp(g) after
+  // landing, in place); this CTA's v columns [16][kCols] bf16
+  static constexpr uint32_t kOffK = 0;
+  static constexpr uint32_t kOffQ = kOffK + kBlk * kD * 2;
+  static constexpr uint32_t kOffG = kOffQ + kBlk * kD * 2;
+  static constexpr uint32_t kOffV = kOffG + kBlk * kD * 4;
+  static constexpr uint32_t kStage = align128(kOffV + kBlk * kCols * 2);
+  static constexpr uint32_t kTokBytes = kD * 2 * 2 + kD * 4 + kCols * 2;   // copied per token
+  // per block, one buffer: k, q as f32 [16][128], beta [16], k.q [16]
+  static constexpr uint32_t kOffKF = 2 * kStage;
+  static constexpr uint32_t kOffQF = kOffKF + kBlk * kD * 4;
+  static constexpr uint32_t kOffBeta = kOffQF + kBlk * kD * 4;
+  static constexpr uint32_t kOffKQ = kOffBeta + kBlk * 4;
+  // per token, two buffers: per warp and lane the partial sums (S'^T k)[kCPT], (S'^T q)[kCPT]
+  static constexpr uint32_t kOffPart = align128(kOffKQ + kBlk * 4);
+  static constexpr uint32_t kPartBuf = kWarps * 32 * 2 * kCPT * 4;
+  static constexpr uint32_t kSmem = kOffPart + 2 * kPartBuf;
+};
+
+template <int kCPT>
+struct Vec;
+template <>
+struct Vec<1> {
+  __device__ static void load(const float* p, float (&x)[1]) { x[0] = *p; }
+  __device__ static void store(float* p, const float (&x)[1]) { *p = x[0]; }
+};
+template <>
+struct Vec<4> {
+  __device__ static void load(const float* p, float (&x)[4]) {
+    const float4 v = *reinterpret_cast<const float4*>(p);
+    x[0] = v.x;
+    x[1] = v.y;
+    x[2] = v.z;
+    x[3] = v.w;
   }
-}
+  __device__ static void store(float* p, const float (&x)[4]) {
+    *reinterpret_cast<float4*>(p) = make_float4(x[0], x[1], x[2], x[3]);
+  }
+};
 
-__device__ __forceinline__ uint16_t f32_to_bf16_rn(float x) {
-  return static_cast<uint16_t>(pack_bf16(x, 0.f) & 0xffffu);
-}
-
-// write a thread's 16 rows of column `col` into the state at `base` ([128][128] FP32)
-__device__ __forceinline__ void store_slice(float* base, const float (&s)[kRows], int warp,
-                                            int col) {
+// write a thread's rows of its columns into the state at `base` ([128][128] FP32)
+template <int kCPT>
+__device__ __forceinline__ void store_slice(float* base, const float (&s)[kRows][kCPT], int warp,
+                                            int col0) {
 #pragma unroll
-  for (int r = 0; r < kRows; ++r) base[static_cast<int64_t>(warp * kRows + r) * kD + col] = s[r];
+  for (int r = 0; r < kRows; ++r)
+    Vec<kCPT>::store(base + static_cast<int64_t>(warp * kRows + r) * kD + col0, s[r]);
 }
 
 __device__ __forceinline__ void record(const TokenParams& p, int32_t code) {
   if (p.status != nullptr) atomicCAS(p.status, 0, code);
 }
 
-extern const uint32_t kSmemAllocBytes = 2 * kBufBytes;
-extern const int kThreadsPerCta = kThreads;
-extern const int kCtasPerUnit = kSlices;
+template <int kCPT>
+__device__ __forceinline__ void store_out(uint16_t* dst, const float (&o)[kCPT]) {
+  if constexpr (kCPT == 1) {
+    *dst = static_cast<uint16_t>(pack_bf16(o[0], 0.f) & 0xffffu);
+  } else {
+    *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16(o[0], o[1]), pack_bf16(o[2], o[3]));
+  }
+}
 
-}  // namespace tok
+template <int kCPT>
+__device__ __forceinline__ void zero_out(uint16_t* dst) {
+  if constexpr (kCPT == 1) {
+    *dst = 0;
+  } else {
+    *reinterpret_cast<uint2*>(dst) = make_uint2(0u, 0u);
+  }
+}
 
-__global__ void __launch_bounds__(tok::kThreads, 3) kda_token_kernel(const TokenParams p) {
-  using namespace tok;
-  extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ float2 part[2][kWarps][32];   // per warp: (S'^T k, S'^T q) partial column sums
-  __shared__ float kqp[2][kWarps];         // per warp: partial k . q
+__device__ __forceinline__ float4 bf16x4_to_f32(const uint2 w) {
+  return make_float4(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xffff0000u),
+                     __uint_as_float(w.y << 16), __uint_as_float(w.y & 0xffff0000u));
+}
+
+template <int kCPT>
+__device__ __forceinline__ void token_body(const TokenParams& p, uint8_t* smem) {
+  using C = Cfg<kCPT>;
   __shared__ __align__(8) uint64_t full[2];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int slice = static_cast<int>(blockIdx.x % kSlices);
-  const int64_t unit = blockIdx.x / kSlices;
+  const int slice = static_cast<int>(blockIdx.x % C::kSlices);
+  const int64_t unit = blockIdx.x / C::kSlices;
   const int32_t n = static_cast<int32_t>(unit / p.H);
   const int32_t h = static_cast<int32_t>(unit - static_cast<int64_t>(n) * p.H);
   if ((p.flags & kFlagValidate) && p.ws != nullptr &&
@@ -105,7 +151,7 @@ __global__ void __launch_bounds__(tok::kThreads, 3) kda_token_kernel(const Token
   }
   const int32_t ck = p.ckpt_offsets ? min(max(p.ckpt_offsets[n], 0), len) : -1;
   const int64_t tok_stride = static_cast<int64_t>(p.H) * kD;   // elements between token rows
-  const int col = slice * kCols + lane;
+  const int col0 = slice * C::kCols + lane * kCPT;              // this thread's first column
   int64_t sidx = n;
   if (p.slot != nullptr) {
     const int32_t si = p.slot[n];
@@ -113,7 +159,7 @@ __global__ void __launch_bounds__(tok::kThreads, 3) kda_token_kernel(const Token
       // padding entry (negative) or out-of-range slot: no state access, zero output
       if (si >= p.pool && tid == 0 && slice == 0 && h == 0) record(p, kStatusBadStateIndex);
       for (int t = warp; t < len; t += kWarps)
-        p.out[(start + t) * tok_stride + h * kD + col] = 0;
+        zero_out<kCPT>(p.out + (start + t) * tok_stride + h * kD + col0);
       return;
     }
     sidx = si;
@@ -132,17 +178,17 @@ __global__ void __launch_bounds__(tok::kThreads, 3) kda_token_kernel(const Token
   // block issue: warp 0 lanes copy one token row each; warp 1 lanes fetch beta into
   // a register that is parked in shared memory once the block has landed
   auto issue = [&](int b) {
-    uint8_t* buf = smem + (b & 1) * kBufBytes;
+    uint8_t* buf = smem + (b & 1) * C::kStage;
     const int t0 = b * kBlk, nt = min(kBlk, len - t0);
     if (warp == 0) {
-      if (lane == 0) mbar_arrive_expect_tx(&full[b & 1], static_cast<uint32_t>(nt) * kTokBytes);
+      if (lane == 0) mbar_arrive_expect_tx(&full[b & 1], static_cast<uint32_t>(nt) * C::kTokBytes);
       if (lane < nt) {
         const int64_t row = static_cast<int64_t>(start + t0 + lane) * tok_stride + h * kD;
-        bulk_load(buf + kOffK + lane * kD * 2, p.k + row, kD * 2, &full[b & 1]);
-        bulk_load(buf + kOffQ + lane * kD * 2, p.q + row, kD * 2, &full[b & 1]);
-        bulk_load(buf + kOffE + lane * kD * 4, p.g + row, kD * 4, &full[b & 1]);
-        bulk_load(buf + kOffV + lane * kCols * 2, p.v + row + slice * kCols, kCols * 2,
-                  &full[b & 1]);
+        bulk_load(buf + C::kOffK + lane * kD * 2, p.k + row, kD * 2, &full[b & 1]);
+        bulk_load(buf + C::kOffQ + lane * kD * 2, p.q + row, kD * 2, &full[b & 1]);
+        bulk_load(buf + C::kOffG + lane * kD * 4, p.g + row, kD * 4, &full[b & 1]);
+        bulk_load(buf + C::kOffV + lane * C::kCols * 2, p.v + row + slice * C::kCols,
+                  C::kCols * 2, &full[b & 1]);
       }
     }
   };
@@ -158,20 +204,26 @@ __global__ void __launch_bounds__(tok::kThreads, 3) kda_token_kernel(const Token
   }
 
   // ---- the state slice (loads overlap the first block's copies)
-  float s[kRows];
+  float s[kRows][kCPT];
   if (p.src != nullptr) {
 #pragma unroll
     for (int r = 0; r < kRows; ++r)
-      s[r] = p.src[soff + static_cast<int64_t>(warp * kRows + r) * kD + col];
+      Vec<kCPT>::load(p.src + soff + static_cast<int64_t>(warp * kRows + r) * kD + col0, s[r]);
   } else {
 #pragma unroll
-    for (int r = 0; r < kRows; ++r) s[r] = 0.f;
+    for (int r = 0; r < kRows; ++r)
+#pragma unroll
+      for (int c = 0; c < kCPT; ++c) s[r][c] = 0.f;
   }
-  if (ck == 0) store_slice(p.ckpt + ck_off, s, warp, col);
+  if (ck == 0) store_slice<kCPT>(p.ckpt + ck_off, s, warp, col0);
 
+  float* kf = reinterpret_cast<float*>(smem + C::kOffKF);
+  float* qf = reinterpret_cast<float*>(smem + C::kOffQF);
+  float* betas = reinterpret_cast<float*>(smem + C::kOffBeta);
+  float* kqs = reinterpret_cast<float*>(smem + C::kOffKQ);
   bool ok = true;
   for (int b = 0; b < nblk && ok; ++b) {
-    uint8_t* buf = smem + (b & 1) * kBufBytes;
+    uint8_t* buf = smem + (b & 1) * C::kStage;
     const int t0 = b * kBlk, nt = min(kBlk, len - t0);
     ok = mbar_wait(&full[b & 1], static_cast<uint32_t>((b >> 1) & 1), p.wait_budget);
     if (__syncthreads_or(!ok)) {
@@ -184,66 +236,144 @@ __global__ void __launch_bounds__(tok::kThreads, 3) kda_token_kernel(const Token
       ok = false;
       break;
     }
-    // g -> exp(g) in place, beta parked
-    float* e = reinterpret_cast<float*>(buf + kOffE);
-    for (int i = tid; i < nt * kD; i += kThreads) e[i] = ex2(e[i] * kLog2e);
-    if (warp == 1 && lane < nt) reinterpret_cast<float*>(buf + kOffB)[lane] = beta_next;
-    fence_proxy_async_smem();   // generic writes ordered before the next bulk copies
+    // ---- per block: exp(g) in place, k and q to f32, k.q per token, beta parked.
+    // Quad i4 covers channels 4 (i4 % 32) .. +3 of token i4 / 32, so the 32 lanes of a
+    // warp together hold one token row and reduce its k.q with shuffles.
+    float* e = reinterpret_cast<float*>(buf + C::kOffG);
+    const uint2* kb = reinterpret_cast<const uint2*>(buf + C::kOffK);
+    const uint2* qb = reinterpret_cast<const uint2*>(buf + C::kOffQ);
+#pragma unroll
+    for (int j = 0; j < kBlk * kD / 4 / kThreads; ++j) {
+      const int i4 = tid + j * kThreads;
+      const int tk = i4 >> 5;   // warp-uniform
+      if (tk < nt) {
+        const float4 gv = reinterpret_cast<const float4*>(e)[i4];
+        reinterpret_cast<float4*>(e)[i4] = make_float4(ex2(gv.x * kLog2e), ex2(gv.y * kLog2e),
+                                                       ex2(gv.z * kLog2e), ex2(gv.w * kLog2e));
+        const float4 kv = bf16x4_to_f32(kb[i4]), qv = bf16x4_to_f32(qb[i4]);
+        reinterpret_cast<float4*>(kf)[i4] = kv;
+        reinterpret_cast<float4*>(qf)[i4] = qv;
+        float dot = fmaf(kv.x, qv.x, fmaf(kv.y, qv.y, fmaf(kv.z, qv.z, kv.w * qv.w)));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+        if (lane == 0) kqs[tk] = dot;
+      }
+    }
+    if (warp == 1 && lane < nt) betas[lane] = beta_next;
+    fence_proxy_async_smem();   // generic writes to the stage ordered before its next bulk copies
     __syncthreads();
     if (b + 1 < nblk) {
       issue(b + 1);
       fetch_beta(b + 1);
     }
-    const float* eb = e;
     for (int i = 0; i < nt; ++i) {
       const int t = t0 + i;
-      const uint4* kp = reinterpret_cast<const uint4*>(buf + kOffK + i * kD * 2 + warp * kRows * 2);
-      const uint4* qp = reinterpret_cast<const uint4*>(buf + kOffQ + i * kD * 2 + warp * kRows * 2);
-      const float4* ep = reinterpret_cast<const float4*>(eb + i * kD + warp * kRows);
-      float kf[kRows], qf[kRows];
-      unpack8(kp[0], kf);
-      unpack8(kp[1], kf + 8);
-      unpack8(qp[0], qf);
-      unpack8(qp[1], qf + 8);
-      float a = 0.f, bq = 0.f, kq = 0.f;
+      const float4* kp = reinterpret_cast<const float4*>(kf + i * kD + warp * kRows);
+      const float4* qp = reinterpret_cast<const float4*>(qf + i * kD + warp * kRows);
+      const float4* ep = reinterpret_cast<const float4*>(e + i * kD + warp * kRows);
+      // two accumulators per sum shorten the FMA chains of the one-column shape; with
+      // four columns the chains are independent already
+      constexpr int kAcc = kCPT == 1 ? 2 : 1;
+      float a[kCPT][kAcc], bq[kCPT][kAcc];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const float4 ev = ep[c];
-        const float ef[4] = {ev.x, ev.y, ev.z, ev.w};
+      for (int c = 0; c < kCPT; ++c)
+#pragma unroll
+        for (int x = 0; x < kAcc; ++x) a[c][x] = bq[c][x] = 0.f;
+#pragma unroll
+      for (int r4 = 0; r4 < 4; ++r4) {
+        const float4 kv = kp[r4], qv = qp[r4], ev = ep[r4];
+        const float kr[4] = {kv.x, kv.y, kv.z, kv.w};
+        const float qr[4] = {qv.x, qv.y, qv.z, qv.w};
+        const float er[4] = {ev.x, ev.y, ev.z, ev.w};
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const int r = 4 * c + j;
-          s[r] *= ef[j];
-          a = fmaf(s[r], kf[r], a);
-          bq = fmaf(s[r], qf[r], bq);
-          kq = fmaf(kf[r], qf[r], kq);
+          const int r = 4 * r4 + j;
+#pragma unroll
+          for (int c = 0; c < kCPT; ++c) {
+            s[r][c] *= er[j];
+            a[c][j % kAcc] = fmaf(s[r][c], kr[j], a[c][j % kAcc]);
+            bq[c][j % kAcc] = fmaf(s[r][c], qr[j], bq[c][j % kAcc]);
+          }
         }
       }
-      part[t & 1][warp][lane] = make_float2(a, bq);
-      if (lane == 0) kqp[t & 1][warp] = kq;
+      float* part = reinterpret_cast<float*>(smem + C::kOffPart + (t & 1) * C::kPartBuf);
+      {
+        float pa[kCPT], pb[kCPT];
+#pragma unroll
+        for (int c = 0; c < kCPT; ++c) {
+          pa[c] = a[c][0];
+          pb[c] = bq[c][0];
+#pragma unroll
+          for (int x = 1; x < kAcc; ++x) {
+            pa[c] += a[c][x];
+            pb[c] += bq[c][x];
+          }
+        }
+        Vec<kCPT>::store(part + (warp * 32 + lane) * 2 * kCPT, pa);
+        Vec<kCPT>::store(part + (warp * 32 + lane) * 2 * kCPT + kCPT, pb);
+      }
       __syncthreads();
-      float A = 0.f, B = 0.f, KQ = 0.f;
+      float A[kCPT], B[kCPT];
+#pragma unroll
+      for (int c = 0; c < kCPT; ++c) A[c] = B[c] = 0.f;
 #pragma unroll
       for (int w = 0; w < kWarps; ++w) {
-        const float2 pw = part[t & 1][w][lane];
-        A += pw.x;
-        B += pw.y;
-        KQ += kqp[t & 1][w];
-      }
-      const float vv = bf16_to_f32(reinterpret_cast<const uint16_t*>(buf + kOffV + i * kCols * 2)[lane]);
-      const float bt = reinterpret_cast<const float*>(buf + kOffB)[i];
-      const float u = bt * (vv - A);
-      if (warp == (t & (kWarps - 1)))
-        p.out[(start + t) * tok_stride + h * kD + col] = f32_to_bf16_rn(p.scale * fmaf(u, KQ, B));
+        float pa[kCPT], pb[kCPT];
+        Vec<kCPT>::load(part + (w * 32 + lane) * 2 * kCPT, pa);
+        Vec<kCPT>::load(part + (w * 32 + lane) * 2 * kCPT + kCPT, pb);
 #pragma unroll
-      for (int r = 0; r < kRows; ++r) s[r] = fmaf(kf[r], u, s[r]);
-      if (t + 1 == ck) store_slice(p.ckpt + ck_off, s, warp, col);
+        for (int c = 0; c < kCPT; ++c) {
+          A[c] += pa[c];
+          B[c] += pb[c];
+        }
+      }
+      const float kq = kqs[i], bt = betas[i];
+      const uint16_t* vrow = reinterpret_cast<const uint16_t*>(buf + C::kOffV + i * C::kCols * 2);
+      float u[kCPT], o[kCPT];
+#pragma unroll
+      for (int c = 0; c < kCPT; ++c) {
+        u[c] = bt * (bf16_to_f32(vrow[lane * kCPT + c]) - A[c]);
+        o[c] = p.scale * fmaf(u[c], kq, B[c]);
+      }
+      if (warp == (t & (kWarps - 1)))
+        store_out<kCPT>(p.out + (start + t) * tok_stride + h * kD + col0, o);
+#pragma unroll
+      for (int r4 = 0; r4 < 4; ++r4) {
+        const float4 kv = kp[r4];
+        const float kr[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+          for (int c = 0; c < kCPT; ++c) s[4 * r4 + j][c] = fmaf(kr[j], u[c], s[4 * r4 + j][c]);
+      }
+      if (t + 1 == ck) store_slice<kCPT>(p.ckpt + ck_off, s, warp, col0);
       if (p.steps != nullptr)
-        store_slice(p.steps + ((static_cast<int64_t>(n) * p.fixed_len + t) * p.H + h) * kD * kD,
-                    s, warp, col);
+        store_slice<kCPT>(
+            p.steps + ((static_cast<int64_t>(n) * p.fixed_len + t) * p.H + h) * kD * kD, s, warp,
+            col0);
     }
+    // (the next block's conversion writes kf, qf, k.q and beta only after the barrier
+    // that follows its landing, which every thread reaches after this token loop)
   }
-  if (ok && p.dst != nullptr) store_slice(p.dst + soff, s, warp, col);
+  if (ok && p.dst != nullptr) store_slice<kCPT>(p.dst + soff, s, warp, col0);
 }
+
+}  // namespace tok
+
+__global__ void __launch_bounds__(tok::kThreads, 3) kda_token_narrow_kernel(const TokenParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  tok::token_body<1>(p, smem);
+}
+
+__global__ void __launch_bounds__(tok::kThreads, 2) kda_token_wide_kernel(const TokenParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  tok::token_body<4>(p, smem);
+}
+
+namespace tok {
+extern const uint32_t kSmemNarrow = Cfg<1>::kSmem;
+extern const uint32_t kSmemWide = Cfg<4>::kSmem;
+extern const int kThreadsPerCta = kThreads;
+}  // namespace tok
 
 }  // namespace kda

@@ -55,6 +55,8 @@ def test_decode_aliasing_rejected():
 
 def test_decode_unknown_flag_rejected():
     assert dcall(dargs(flags=1 << 5)) == capi.KDA_ERR_BAD_OPTION
+    both = capi.KDA_DECODE_NARROW | capi.KDA_DECODE_WIDE
+    assert dcall(dargs(flags=both)) == capi.KDA_ERR_BAD_OPTION
 
 
 def test_decode_valid_arguments_reach_the_device_check_without_gpu():
@@ -68,11 +70,19 @@ def test_decode_valid_arguments_reach_the_device_check_without_gpu():
 
 
 def test_token_variant_describe_and_workspace():
-    shp = capi.make_shape(32, 32 * 48, 12, 48)
+    shp = capi.make_shape(32, 32 * 16, 12, 16)
     d = capi.kda_prefill_describe(shp, False, {"variant": capi.KDA_VARIANT_TOKEN})
-    assert "variant=token" in d and "grid=1536x256" in d, d
+    assert "variant=token" in d and "grid=384x256 (wide" in d, d     # 384 units: one CTA each
+    few = capi.kda_prefill_describe(capi.make_shape(2, 2 * 48, 12, 48), False,
+                                    {"variant": capi.KDA_VARIANT_TOKEN})
+    assert "grid=96x256 (narrow" in few, few                         # 24 units: four CTAs each
+    # the table: up to 16 tokens always, up to 32 for at most 16 units
     auto = capi.kda_prefill_describe(shp, False)
     assert "variant=token" in auto, auto
+    one = capi.kda_prefill_describe(capi.make_shape(1, 32, 12, 32), False)
+    assert "variant=token" in one, one
+    mid = capi.kda_prefill_describe(capi.make_shape(8, 8 * 32, 12, 32), False)
+    assert "variant=split" in mid, mid
     longer = capi.kda_prefill_describe(capi.make_shape(32, 32 * 2048, 12, 2048), False)
     assert "variant=token" not in longer, longer
     # the token variant keeps no chunk records: its workspace is far smaller

@@ -83,14 +83,14 @@ def test_token_forced_timeout_reports_status_and_context_survives():
 
 def test_token_matches_chunked_within_tolerance_and_auto_picks_it():
     import kda_chunked_recurrent_b200 as K
-    inp = make_inputs([64] * 6, 4, seed=515, with_h0=True, fixed_layout=True)
+    inp = make_inputs([16] * 6, 4, seed=515, with_h0=True, fixed_layout=True)
     a = run_gpu(inp, variant=TOKEN)
     b = run_gpu(inp, variant=SPLIT)
     assert float((a["o"] - b["o"]).abs().max()) <= O_TOL
     assert float(rel_fro(a["ht"].numpy(), b["ht"].numpy()).max()) <= S_TOL
     auto = run_gpu(inp)   # every sequence within the table's token bound
     assert torch.equal(auto["o"], a["o"]) and torch.equal(auto["ht"], a["ht"])
-    d = K.capi.kda_prefill_describe(K.capi.make_shape(6, 384, 4, 64), False)
+    d = K.capi.kda_prefill_describe(K.capi.make_shape(6, 96, 4, 16), False)
     assert "variant=token" in d, d
 
 
@@ -140,6 +140,26 @@ def test_decode_single_token(N, H, P):
     d = make_decode_inputs(N, 1, H, P, seed=520 + N, indices=(P > N))
     out, pool, _ = _decode(K, d)
     _check_decode(d, out, pool)
+
+
+@pytest.mark.parametrize("shape_flag", [2, 4])   # KDA_DECODE_NARROW, KDA_DECODE_WIDE
+@pytest.mark.parametrize("N,T,H,P", [(5, 1, 3, 11), (3, 5, 2, 3), (40, 2, 4, 64)])
+def test_decode_both_kernel_shapes(shape_flag, N, T, H, P):
+    import kda_chunked_recurrent_b200 as K
+    d = make_decode_inputs(N, T, H, P, seed=600 + N + T + shape_flag, pad_every=4)
+    out, pool, steps = _decode(K, d, return_step_states=True, flags=shape_flag)
+    _check_decode(d, out, pool, steps=steps)
+
+
+def test_decode_shapes_agree_closely():
+    # both shapes run the same FP32 recurrence; only the order of the row sums
+    # differs (the narrow shape splits them over two accumulators)
+    import kda_chunked_recurrent_b200 as K
+    d = make_decode_inputs(9, 3, 4, 9, seed=610)
+    a = _decode(K, d, flags=K.KDA_DECODE_NARROW)
+    b = _decode(K, d, flags=K.KDA_DECODE_WIDE)
+    assert float((a[0] - b[0]).abs().max()) <= 2e-3          # a BF16 rounding step at most
+    assert float(rel_fro(a[1].numpy(), b[1].numpy()).max()) <= 1e-5
 
 
 def test_decode_padding_rows_and_permuted_slots():
