@@ -272,6 +272,9 @@ kda_status_t kda_prefill_noalloc(const void* q, const void* k, const void* v, co
  *   device_status  INT32 device word, 4-byte aligned, or NULL: the first device
  *             error is stored there with atomicCAS from KDA_OK (the caller clears
  *             it); without it device errors are not reported.
+ *   frontend  NULL, or the input front end (kda_frontend_t above): q, k, g and beta
+ *             then hold raw projections that the kernel turns into the recurrence
+ *             inputs.
  *   flags     KDA_DECODE_KEEP_STATE: the pool is read only.  KDA_DECODE_NARROW /
  *             KDA_DECODE_WIDE force the kernel shape (timing aid; the default
  *             picks by the number of (sequence, head) units).
@@ -281,6 +284,37 @@ kda_status_t kda_prefill_noalloc(const void* q, const void* k, const void* v, co
  * or each other (KDA_ERR_OUT_ALIAS).  Returns KDA_OK when the launch was
  * enqueued.  No workspace and no allocation; CUDA-graph capturable.
  */
+/*
+ * Optional input front end of kda_decode: the kernel forms the recurrence inputs
+ * from raw projections, in FP32, so that no rounded intermediate reaches the
+ * state.  The parameter set (A_log per head, dt_bias per head and key channel, a
+ * finite negative lower bound, q/k L2 normalisation, beta given as a logit) is
+ * FlashInfer PR #4262's "Dispatch contract"; the pages print no formula, and the
+ * one below is this library's reading (it puts every log-decay in
+ * (lower_bound, 0)):
+ *   KDA_FE_QK_L2NORM   q, k <- x / sqrt(sum_c x_c^2 + l2_eps) per (token, head)
+ *   KDA_FE_GATE        `g` holds the raw gate a as BF16 [N, T, H, 128] (16-byte
+ *                      aligned); g_c = lower_bound * sigmoid(exp(A_log[h]) *
+ *                      (a_c + dt_bias[h][c])), sigmoid(x) = 1 / (1 + exp(-x))
+ *   KDA_FE_BETA_LOGIT  `beta` holds logits; beta <- sigmoid(beta)
+ * A_log [H] FP32 (4-byte aligned) and dt_bias [H, 128] FP32 (16-byte aligned) are
+ * device arrays, read only with KDA_FE_GATE.  lower_bound must lie in [-5, 0)
+ * (the gate bound of lmdeploy PR #5050 "Motivation"), l2_eps in [0, 1]; otherwise
+ * KDA_ERR_BAD_OPTION.
+ */
+enum {
+  KDA_FE_QK_L2NORM = 1u << 0,
+  KDA_FE_GATE = 1u << 1,
+  KDA_FE_BETA_LOGIT = 1u << 2
+};
+typedef struct {
+  uint32_t flags;        /* KDA_FE_*                                            */
+  float lower_bound;     /* KDA_FE_GATE                                         */
+  float l2_eps;          /* KDA_FE_QK_L2NORM                                    */
+  const float* A_log;    /* KDA_FE_GATE: [H]                                    */
+  const float* dt_bias;  /* KDA_FE_GATE: [H, 128]                               */
+} kda_frontend_t;
+
 typedef struct {
   int32_t num_seqs;       /* N >= 1                                               */
   int32_t tokens_per_seq; /* T >= 1 new tokens of every sequence                  */
@@ -300,7 +334,7 @@ kda_status_t kda_decode(const void* q, const void* k, const void* v, const float
                         const void* beta, float scale, float* state,
                         const int32_t* state_indices, const kda_decode_shape_t* shape,
                         void* out, float* step_states, int32_t* device_status, uint32_t flags,
-                        void* stream);
+                        const kda_frontend_t* frontend, void* stream);
 
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
 int kda_version(void);

@@ -21,6 +21,7 @@ KDA_OK = 0
 KDA_VARIANT_AUTO, KDA_VARIANT_SPLIT, KDA_VARIANT_FUSED = 0, 1, 2
 KDA_VARIANT_HYBRID, KDA_VARIANT_TOKEN = 3, 4
 KDA_DECODE_KEEP_STATE, KDA_DECODE_NARROW, KDA_DECODE_WIDE = 1, 2, 4
+KDA_FE_QK_L2NORM, KDA_FE_GATE, KDA_FE_BETA_LOGIT = 1, 2, 4
 KDA_FLAG_VALIDATE, KDA_FLAG_TEST_FORCE_TIMEOUT, KDA_FLAG_CU_SEQLENS_I64 = 1, 2, 4
 
 
@@ -117,13 +118,15 @@ def prefill(q, k, v, g, beta, scale: float, *, h0=None, cu_seqlens=None, num_seq
 
 def decode(q, k, v, g, beta, scale: float, state, *, state_indices=None, out=None,
            step_states=None, return_step_states: bool = False, keep_state: bool = False,
-           device_status=None, flags: int = 0, stream=None):
+           device_status=None, flags: int = 0, frontend: Optional[dict] = None, stream=None):
     """Decode / draft verification over a state pool (kda_decode).
 
     q, k, v: [N, T, H, 128] bf16; g: [N, T, H, 128] fp32; beta: [N, T, H] bf16;
     state: [P, H, 128, 128] fp32 pool, updated in place unless ``keep_state``;
     state_indices: [N] int32 slots (negative = padding row) or None (slot n).
     ``flags`` may add KDA_DECODE_NARROW / KDA_DECODE_WIDE (kernel shape).
+    ``frontend``: dict(flags=KDA_FE_*, lower_bound=..., l2_eps=..., A_log=[H] fp32,
+    dt_bias=[H, 128] fp32); with KDA_FE_GATE, ``g`` is the raw gate in bf16.
     Returns (out, step_states); step_states [N, T, H, 128, 128] when requested.
     """
     import torch
@@ -137,11 +140,16 @@ def decode(q, k, v, g, beta, scale: float, state, *, state_indices=None, out=Non
         step_states = torch.empty(N, T, H, 128, 128, dtype=torch.float32, device=dev)
     shape = capi.make_decode_shape(N, T, H, P)
     s = stream if stream is not None else torch.cuda.current_stream(dev)
+    fe = None
+    if frontend is not None:
+        fe = capi.make_frontend(frontend.get("flags", 0), frontend.get("lower_bound", 0.0),
+                                frontend.get("l2_eps", 0.0), _ptr(frontend.get("A_log")),
+                                _ptr(frontend.get("dt_bias")))
     rc = capi.kda_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale),
                          _ptr(state), _ptr(state_indices), shape, _ptr(out), _ptr(step_states),
                          _ptr(device_status),
                          int(flags) | (KDA_DECODE_KEEP_STATE if keep_state else 0),
-                         s.cuda_stream)
+                         s.cuda_stream, fe)
     if rc != KDA_OK:
         raise KDAError(rc, "kda_decode")
     return out, step_states

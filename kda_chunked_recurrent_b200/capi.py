@@ -35,6 +35,9 @@ KDA_VARIANT_FUSED = 2
 KDA_VARIANT_HYBRID = 3
 KDA_VARIANT_TOKEN = 4
 KDA_DECODE_KEEP_STATE = 1
+KDA_FE_QK_L2NORM = 1
+KDA_FE_GATE = 2
+KDA_FE_BETA_LOGIT = 4
 KDA_DECODE_NARROW = 2
 KDA_DECODE_WIDE = 4
 KDA_FLAG_VALIDATE = 1
@@ -50,6 +53,12 @@ class kda_shape_t(ctypes.Structure):
 class kda_decode_shape_t(ctypes.Structure):
     _fields_ = [("num_seqs", ctypes.c_int32), ("tokens_per_seq", ctypes.c_int32),
                 ("num_heads", ctypes.c_int32), ("pool_size", ctypes.c_int32)]
+
+
+class kda_frontend_t(ctypes.Structure):
+    _fields_ = [("flags", ctypes.c_uint32), ("lower_bound", ctypes.c_float),
+                ("l2_eps", ctypes.c_float), ("A_log", ctypes.c_void_p),
+                ("dt_bias", ctypes.c_void_p)]
 
 
 class kda_options_t(ctypes.Structure):
@@ -83,7 +92,8 @@ def _load():
                                          ctypes.c_size_t]
     lib.kda_decode.restype = ctypes.c_int
     lib.kda_decode.argtypes = [P, P, P, P, P, ctypes.c_float, P, P,
-                               ctypes.POINTER(kda_decode_shape_t), P, P, P, ctypes.c_uint32, P]
+                               ctypes.POINTER(kda_decode_shape_t), P, P, P, ctypes.c_uint32,
+                               ctypes.POINTER(kda_frontend_t), P]
     return lib
 
 
@@ -148,9 +158,16 @@ def make_decode_shape(num_seqs, tokens_per_seq, num_heads, pool_size) -> kda_dec
     return kda_decode_shape_t(int(num_seqs), int(tokens_per_seq), int(num_heads), int(pool_size))
 
 
+def make_frontend(flags, lower_bound=0.0, l2_eps=0.0, A_log=None, dt_bias=None) -> kda_frontend_t:
+    """A_log / dt_bias are device addresses (integers) or None."""
+    return kda_frontend_t(int(flags), float(lower_bound), float(l2_eps), A_log, dt_bias)
+
+
 def kda_decode(q, k, v, g, beta, scale, state, state_indices, shape, out, step_states,
-               device_status, flags, stream) -> int:
-    """All pointer arguments are integers (device addresses) or None."""
+               device_status, flags, stream, frontend=None) -> int:
+    """All pointer arguments are integers (device addresses) or None; frontend is a
+    kda_frontend_t or None."""
+    fe = None if frontend is None else ctypes.byref(frontend)
     return int(lib.kda_decode(q, k, v, g, beta, ctypes.c_float(scale), state, state_indices,
                               ctypes.byref(shape), out, step_states, device_status,
-                              int(flags), stream))
+                              int(flags), fe, stream))

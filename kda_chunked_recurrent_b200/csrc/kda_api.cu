@@ -31,6 +31,8 @@ namespace rec { extern const uint32_t kSmemAllocBytes; extern const int kThreads
 namespace fused { extern const uint32_t kSmemAllocBytes; extern const int kThreadsPerCta; }
 __global__ void kda_token_narrow_kernel(const TokenParams p);
 __global__ void kda_token_wide_kernel(const TokenParams p);
+__global__ void kda_token_narrow_fe_kernel(const TokenParams p);
+__global__ void kda_token_wide_fe_kernel(const TokenParams p);
 namespace tok {
 extern const uint32_t kSmemNarrow;
 extern const uint32_t kSmemWide;
@@ -123,25 +125,32 @@ bool token_wide(int64_t units, uint32_t force) {
 }
 
 // Launch the per-token kernel for `units` (sequence, head) pairs.
+// (The kernels with the input front end compiled in are used only when tp.fe_flags
+// asks for it, so the plain path keeps its register budget.)
 kda_status_t launch_token(const TokenParams& tp, int64_t units, bool wide, cudaStream_t s) {
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    cudaError_t e1 = cudaFuncSetAttribute(kda_token_narrow_kernel,
-                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          tok::kSmemNarrow);
-    cudaError_t e2 = cudaFuncSetAttribute(kda_token_wide_kernel,
-                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          tok::kSmemWide);
-    attr_err = e1 != cudaSuccess ? e1 : e2;
+    const void* narrow[] = {reinterpret_cast<const void*>(kda_token_narrow_kernel),
+                            reinterpret_cast<const void*>(kda_token_narrow_fe_kernel)};
+    const void* wide_k[] = {reinterpret_cast<const void*>(kda_token_wide_kernel),
+                            reinterpret_cast<const void*>(kda_token_wide_fe_kernel)};
+    for (int i = 0; i < 2; ++i) {
+      cudaError_t e1 = cudaFuncSetAttribute(narrow[i], cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            tok::kSmemNarrow);
+      cudaError_t e2 = cudaFuncSetAttribute(wide_k[i], cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            tok::kSmemWide);
+      if (attr_err == cudaSuccess) attr_err = e1 != cudaSuccess ? e1 : e2;
+    }
   });
   if (attr_err != cudaSuccess) return KDA_ERR_LAUNCH_FAILED;
-  if (wide)
-    kda_token_wide_kernel<<<static_cast<unsigned>(units), tok::kThreadsPerCta, tok::kSmemWide,
-                            s>>>(tp);
-  else
-    kda_token_narrow_kernel<<<static_cast<unsigned>(units * 4), tok::kThreadsPerCta,
-                              tok::kSmemNarrow, s>>>(tp);
+  const bool fe = tp.fe_flags != 0;
+  const unsigned grid = static_cast<unsigned>(wide ? units : units * 4);
+  const uint32_t smem = wide ? tok::kSmemWide : tok::kSmemNarrow;
+  if (wide && fe) kda_token_wide_fe_kernel<<<grid, tok::kThreadsPerCta, smem, s>>>(tp);
+  else if (wide) kda_token_wide_kernel<<<grid, tok::kThreadsPerCta, smem, s>>>(tp);
+  else if (fe) kda_token_narrow_fe_kernel<<<grid, tok::kThreadsPerCta, smem, s>>>(tp);
+  else kda_token_narrow_kernel<<<grid, tok::kThreadsPerCta, smem, s>>>(tp);
   return KDA_OK;
 }
 constexpr int kFusedOneGroupMaxChains = 16;
@@ -594,8 +603,19 @@ kda_status_t kda_decode(const void* q, const void* k, const void* v, const float
                         const void* beta, float scale, float* state,
                         const int32_t* state_indices, const kda_decode_shape_t* shape,
                         void* out, float* step_states, int32_t* device_status, uint32_t flags,
-                        void* stream) {
+                        const kda_frontend_t* frontend, void* stream) {
   if (!shape) return KDA_ERR_NULL_ARG;
+  const uint32_t fe = frontend ? frontend->flags : 0u;
+  if (fe & ~static_cast<uint32_t>(KDA_FE_QK_L2NORM | KDA_FE_GATE | KDA_FE_BETA_LOGIT))
+    return KDA_ERR_BAD_OPTION;
+  if (fe & KDA_FE_GATE) {
+    if (!frontend->A_log || !frontend->dt_bias) return KDA_ERR_NULL_ARG;
+    const float lb = frontend->lower_bound;
+    if (!(lb >= -5.0f && lb < 0.0f)) return KDA_ERR_BAD_OPTION;   // also rejects NaN
+  }
+  if ((fe & KDA_FE_QK_L2NORM) &&
+      !(frontend->l2_eps >= 0.0f && frontend->l2_eps <= 1.0f))   // finite, non-negative
+    return KDA_ERR_BAD_OPTION;
   if (flags & ~static_cast<uint32_t>(KDA_DECODE_KEEP_STATE | KDA_DECODE_NARROW |
                                      KDA_DECODE_WIDE))
     return KDA_ERR_BAD_OPTION;
@@ -612,15 +632,21 @@ kda_status_t kda_decode(const void* q, const void* k, const void* v, const float
       !aligned(out, 16) || !aligned(beta, 2) || !aligned(state, 16) ||
       !aligned(step_states, 16) || !aligned(state_indices, 4) || !aligned(device_status, 4))
     return KDA_ERR_MISALIGNED;
+  if ((fe & KDA_FE_GATE) && (!aligned(frontend->A_log, 4) || !aligned(frontend->dt_bias, 16)))
+    return KDA_ERR_MISALIGNED;
   const size_t tok16 = static_cast<size_t>(N * T * H * 128 * 2);
+  const size_t g_bytes = (fe & KDA_FE_GATE) ? tok16 : tok16 * 2;   // raw BF16 gate or FP32 g
   const size_t st1 = static_cast<size_t>(H * 128 * 128 * 4);   // one slot, all heads
   const Range rq = rng(q, tok16), rk = rng(k, tok16), rv = rng(v, tok16),
-              rg = rng(g, tok16 * 2), rb = rng(beta, static_cast<size_t>(N * T * H * 2)),
+              rg = rng(g, g_bytes), rb = rng(beta, static_cast<size_t>(N * T * H * 2)),
               ri = rng(state_indices, static_cast<size_t>(N * 4)),
               rs = rng(state, st1 * static_cast<size_t>(P)), ro = rng(out, tok16),
               rst = rng(step_states, st1 * static_cast<size_t>(N * T)),
               rds = rng(device_status, 4);
-  const Range inputs[] = {rq, rk, rv, rg, rb, ri};
+  const bool gate = (fe & KDA_FE_GATE) != 0;
+  const Range ra = rng(gate ? frontend->A_log : nullptr, static_cast<size_t>(H * 4)),
+              rdt = rng(gate ? frontend->dt_bias : nullptr, static_cast<size_t>(H * 128 * 4));
+  const Range inputs[] = {rq, rk, rv, rg, rb, ri, ra, rdt};
   const Range outputs[] = {rs, ro, rst, rds};
   for (const Range& o : outputs)
     for (const Range& in : inputs)
@@ -652,6 +678,14 @@ kda_status_t kda_decode(const void* q, const void* k, const void* v, const float
   tp.status = device_status;
   tp.flags = 0;
   tp.wait_budget = kDefaultWaitBudget;
+  tp.fe_flags = (fe & KDA_FE_QK_L2NORM ? kFeQkL2Norm : 0u) | (fe & KDA_FE_GATE ? kFeGate : 0u) |
+                (fe & KDA_FE_BETA_LOGIT ? kFeBetaLogit : 0u);
+  if (gate) {
+    tp.A_log = frontend->A_log;
+    tp.dt_bias = frontend->dt_bias;
+    tp.lower_bound = frontend->lower_bound;
+  }
+  if (fe & KDA_FE_QK_L2NORM) tp.l2_eps = frontend->l2_eps;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   (void)cudaGetLastError();
   st = launch_token(tp, N * H, token_wide(N * H, flags), s);

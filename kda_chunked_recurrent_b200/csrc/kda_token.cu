@@ -26,6 +26,17 @@
 // Decode over a slot-indexed state pool and per-token state export follow the
 // FlashInfer KDA decode entry (SGLang kda_flashinfer.py "FlashInferKDAKernel":
 // decode and target-verify over the same per-(sequence, head) state).
+//
+// Optional input front end (kda_decode), formed in FP32 in the per-block step so
+// that no rounded intermediate reaches the recurrence (a BF16 copy of the
+// normalised k or of beta moves the final state by about 2e-3 relative):
+//   k, q <- x / sqrt(sum x^2 + eps)                        (kFeQkL2Norm)
+//   g    <- lower_bound * sigmoid(exp(A_log) (a + dt_bias)) from the raw BF16 gate a
+//                                                          (kFeGate)
+//   beta <- sigmoid(beta)                                  (kFeBetaLogit)
+// The parameter set is FlashInfer PR #4262's "Dispatch contract" (A_log per head,
+// dt_bias per head and key channel, a negative lower bound, the three switches);
+// the formula is this library's reading of it.
 #include <cstdint>
 
 #include "kda_common.cuh"
@@ -49,13 +60,14 @@ struct Cfg {
   static constexpr int kCols = 32 * kCPT;          // value columns per CTA
   static constexpr int kSlices = kD / kCols;       // CTAs per (sequence, head)
   // staged block, two buffers: k, q [16][128] bf16; g [16][128] f32 (exp(g) after
-  // landing, in place); this CTA's v columns [16][kCols] bf16
+  // landing, in place); this CTA's v columns [16][kCols] bf16; the raw gate
+  // [16][128] bf16 when the front end forms g
   static constexpr uint32_t kOffK = 0;
   static constexpr uint32_t kOffQ = kOffK + kBlk * kD * 2;
   static constexpr uint32_t kOffG = kOffQ + kBlk * kD * 2;
   static constexpr uint32_t kOffV = kOffG + kBlk * kD * 4;
-  static constexpr uint32_t kStage = align128(kOffV + kBlk * kCols * 2);
-  static constexpr uint32_t kTokBytes = kD * 2 * 2 + kD * 4 + kCols * 2;   // copied per token
+  static constexpr uint32_t kOffA = align128(kOffV + kBlk * kCols * 2);
+  static constexpr uint32_t kStage = kOffA + kBlk * kD * 2;
   // per block, one buffer: k, q as f32 [16][128], beta [16], k.q [16]
   static constexpr uint32_t kOffKF = 2 * kStage;
   static constexpr uint32_t kOffQF = kOffKF + kBlk * kD * 4;
@@ -119,12 +131,16 @@ __device__ __forceinline__ void zero_out(uint16_t* dst) {
   }
 }
 
+__device__ __forceinline__ float sigmoid_f32(float x) { return 1.f / (1.f + ex2(-x * kLog2e)); }
+
 __device__ __forceinline__ float4 bf16x4_to_f32(const uint2 w) {
   return make_float4(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xffff0000u),
                      __uint_as_float(w.y << 16), __uint_as_float(w.y & 0xffff0000u));
 }
 
-template <int kCPT>
+// kFE: the input front end is compiled in (its switches are read from p.fe_flags);
+// without it the plain path carries none of its registers
+template <int kCPT, bool kFE>
 __device__ __forceinline__ void token_body(const TokenParams& p, uint8_t* smem) {
   using C = Cfg<kCPT>;
   __shared__ __align__(8) uint64_t full[2];
@@ -174,6 +190,10 @@ __device__ __forceinline__ void token_body(const TokenParams& p, uint8_t* smem) 
   }
   __syncthreads();
 
+  const bool fe_gate = kFE && (p.fe_flags & kFeGate) != 0;
+  const bool fe_norm = kFE && (p.fe_flags & kFeQkL2Norm) != 0;
+  const bool fe_beta = kFE && (p.fe_flags & kFeBetaLogit) != 0;
+  const uint32_t tok_bytes = kD * 2 * 2 + (fe_gate ? kD * 2 : kD * 4) + C::kCols * 2;
   const int nblk = (len + kBlk - 1) / kBlk;
   // block issue: warp 0 lanes copy one token row each; warp 1 lanes fetch beta into
   // a register that is parked in shared memory once the block has landed
@@ -181,12 +201,16 @@ __device__ __forceinline__ void token_body(const TokenParams& p, uint8_t* smem) 
     uint8_t* buf = smem + (b & 1) * C::kStage;
     const int t0 = b * kBlk, nt = min(kBlk, len - t0);
     if (warp == 0) {
-      if (lane == 0) mbar_arrive_expect_tx(&full[b & 1], static_cast<uint32_t>(nt) * C::kTokBytes);
+      if (lane == 0) mbar_arrive_expect_tx(&full[b & 1], static_cast<uint32_t>(nt) * tok_bytes);
       if (lane < nt) {
         const int64_t row = static_cast<int64_t>(start + t0 + lane) * tok_stride + h * kD;
         bulk_load(buf + C::kOffK + lane * kD * 2, p.k + row, kD * 2, &full[b & 1]);
         bulk_load(buf + C::kOffQ + lane * kD * 2, p.q + row, kD * 2, &full[b & 1]);
-        bulk_load(buf + C::kOffG + lane * kD * 4, p.g + row, kD * 4, &full[b & 1]);
+        if (fe_gate)
+          bulk_load(buf + C::kOffA + lane * kD * 2, reinterpret_cast<const uint16_t*>(p.g) + row,
+                    kD * 2, &full[b & 1]);
+        else
+          bulk_load(buf + C::kOffG + lane * kD * 4, p.g + row, kD * 4, &full[b & 1]);
         bulk_load(buf + C::kOffV + lane * C::kCols * 2, p.v + row + slice * C::kCols,
                   C::kCols * 2, &full[b & 1]);
       }
@@ -195,9 +219,12 @@ __device__ __forceinline__ void token_body(const TokenParams& p, uint8_t* smem) 
   float beta_next = 0.f;
   auto fetch_beta = [&](int b) {
     const int t0 = b * kBlk;
-    if (warp == 1 && lane < min(kBlk, len - t0))
+    if (warp == 1 && lane < min(kBlk, len - t0)) {
       beta_next = bf16_to_f32(p.beta[static_cast<int64_t>(start + t0 + lane) * p.H + h]);
+      if (fe_beta) beta_next = sigmoid_f32(beta_next);
+    }
   };
+
   if (nblk > 0) {
     issue(0);
     fetch_beta(0);
@@ -242,21 +269,74 @@ __device__ __forceinline__ void token_body(const TokenParams& p, uint8_t* smem) 
     float* e = reinterpret_cast<float*>(buf + C::kOffG);
     const uint2* kb = reinterpret_cast<const uint2*>(buf + C::kOffK);
     const uint2* qb = reinterpret_cast<const uint2*>(buf + C::kOffQ);
+    if constexpr (!kFE) {
 #pragma unroll
-    for (int j = 0; j < kBlk * kD / 4 / kThreads; ++j) {
-      const int i4 = tid + j * kThreads;
-      const int tk = i4 >> 5;   // warp-uniform
-      if (tk < nt) {
-        const float4 gv = reinterpret_cast<const float4*>(e)[i4];
-        reinterpret_cast<float4*>(e)[i4] = make_float4(ex2(gv.x * kLog2e), ex2(gv.y * kLog2e),
-                                                       ex2(gv.z * kLog2e), ex2(gv.w * kLog2e));
-        const float4 kv = bf16x4_to_f32(kb[i4]), qv = bf16x4_to_f32(qb[i4]);
-        reinterpret_cast<float4*>(kf)[i4] = kv;
-        reinterpret_cast<float4*>(qf)[i4] = qv;
-        float dot = fmaf(kv.x, qv.x, fmaf(kv.y, qv.y, fmaf(kv.z, qv.z, kv.w * qv.w)));
+      for (int j = 0; j < kBlk * kD / 4 / kThreads; ++j) {
+        const int i4 = tid + j * kThreads;
+        const int tk = i4 >> 5;   // warp-uniform
+        if (tk < nt) {
+          const float4 gv = reinterpret_cast<const float4*>(e)[i4];
+          reinterpret_cast<float4*>(e)[i4] = make_float4(ex2(gv.x * kLog2e), ex2(gv.y * kLog2e),
+                                                         ex2(gv.z * kLog2e), ex2(gv.w * kLog2e));
+          const float4 kv = bf16x4_to_f32(kb[i4]), qv = bf16x4_to_f32(qb[i4]);
+          reinterpret_cast<float4*>(kf)[i4] = kv;
+          reinterpret_cast<float4*>(qf)[i4] = qv;
+          float dot = fmaf(kv.x, qv.x, fmaf(kv.y, qv.y, fmaf(kv.z, qv.z, kv.w * qv.w)));
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-        if (lane == 0) kqs[tk] = dot;
+          for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+          if (lane == 0) kqs[tk] = dot;
+        }
+      }
+    } else {
+      const uint2* ab = reinterpret_cast<const uint2*>(buf + C::kOffA);
+      // gate parameters of this head for the lane's four key channels (the loop below
+      // gives lane l channels 4 l .. 4 l + 3 of every row); read per block from L1 so
+      // that they hold no registers across the token loop
+      float rate = 0.f;
+      float4 dtb = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (fe_gate) {
+        rate = expf(__ldg(p.A_log + h));
+        dtb = __ldg(reinterpret_cast<const float4*>(p.dt_bias + static_cast<int64_t>(h) * kD) +
+                    lane);
+      }
+#pragma unroll
+      for (int j = 0; j < kBlk * kD / 4 / kThreads; ++j) {
+        const int i4 = tid + j * kThreads;
+        const int tk = i4 >> 5;   // warp-uniform
+        if (tk < nt) {
+          float4 gv;
+          if (fe_gate) {
+            const float4 av = bf16x4_to_f32(ab[i4]);
+            gv = make_float4(p.lower_bound * sigmoid_f32(rate * (av.x + dtb.x)),
+                             p.lower_bound * sigmoid_f32(rate * (av.y + dtb.y)),
+                             p.lower_bound * sigmoid_f32(rate * (av.z + dtb.z)),
+                             p.lower_bound * sigmoid_f32(rate * (av.w + dtb.w)));
+          } else {
+            gv = reinterpret_cast<const float4*>(e)[i4];
+          }
+          reinterpret_cast<float4*>(e)[i4] = make_float4(ex2(gv.x * kLog2e), ex2(gv.y * kLog2e),
+                                                         ex2(gv.z * kLog2e), ex2(gv.w * kLog2e));
+          float4 kv = bf16x4_to_f32(kb[i4]), qv = bf16x4_to_f32(qb[i4]);
+          float dot = fmaf(kv.x, qv.x, fmaf(kv.y, qv.y, fmaf(kv.z, qv.z, kv.w * qv.w)));
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+          if (fe_norm) {
+            float kk = fmaf(kv.x, kv.x, fmaf(kv.y, kv.y, fmaf(kv.z, kv.z, kv.w * kv.w)));
+            float qq = fmaf(qv.x, qv.x, fmaf(qv.y, qv.y, fmaf(qv.z, qv.z, qv.w * qv.w)));
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+              kk += __shfl_xor_sync(0xffffffffu, kk, o);
+              qq += __shfl_xor_sync(0xffffffffu, qq, o);
+            }
+            const float rk = rsqrtf(kk + p.l2_eps), rq = rsqrtf(qq + p.l2_eps);
+            kv = make_float4(kv.x * rk, kv.y * rk, kv.z * rk, kv.w * rk);
+            qv = make_float4(qv.x * rq, qv.y * rq, qv.z * rq, qv.w * rq);
+            dot *= rk * rq;
+          }
+          reinterpret_cast<float4*>(kf)[i4] = kv;
+          reinterpret_cast<float4*>(qf)[i4] = qv;
+          if (lane == 0) kqs[tk] = dot;
+        }
       }
     }
     if (warp == 1 && lane < nt) betas[lane] = beta_next;
@@ -362,12 +442,23 @@ __device__ __forceinline__ void token_body(const TokenParams& p, uint8_t* smem) 
 
 __global__ void __launch_bounds__(tok::kThreads, 3) kda_token_narrow_kernel(const TokenParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
-  tok::token_body<1>(p, smem);
+  tok::token_body<1, false>(p, smem);
 }
 
 __global__ void __launch_bounds__(tok::kThreads, 2) kda_token_wide_kernel(const TokenParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
-  tok::token_body<4>(p, smem);
+  tok::token_body<4, false>(p, smem);
+}
+
+__global__ void __launch_bounds__(tok::kThreads, 3)
+kda_token_narrow_fe_kernel(const TokenParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  tok::token_body<1, true>(p, smem);
+}
+
+__global__ void __launch_bounds__(tok::kThreads, 2) kda_token_wide_fe_kernel(const TokenParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  tok::token_body<4, true>(p, smem);
 }
 
 namespace tok {

@@ -155,3 +155,21 @@ def make_decode_inputs(num_seqs: int, tokens: int, num_heads: int, pool_size: in
     return DecodeInputs(q=base.q.view(*shp, DK), k=base.k.view(*shp, DK), v=base.v.view(*shp, DV),
                         g=base.g.view(*shp, DK), beta=base.beta.view(*shp), scale=base.scale,
                         pool=pool, state_indices=idx)
+
+
+def make_decode_frontend_inputs(num_seqs: int, tokens: int, num_heads: int, pool_size: int,
+                                seed: int, *, pad_every: int = 0):
+    """Raw projections for the decode front end: q, k ~ N(0, 1) BF16 (not normalised),
+    the raw gate a ~ N(0, 1) BF16 in the ``g`` field, beta logits ~ N(0, 1) BF16 in the
+    ``beta`` field, A_log ~ N(0, 0.5) FP32 [H], dt_bias ~ N(0, 0.5) FP32 [H, 128].
+    Returns (DecodeInputs, A_log, dt_bias)."""
+    d = make_decode_inputs(num_seqs, tokens, num_heads, pool_size, seed, pad_every=pad_every)
+    gen = torch.Generator().manual_seed(int(seed) + 11)
+    shp = tuple(d.q.shape)
+    d.q = torch.randn(*shp, generator=gen).to(torch.bfloat16)
+    d.k = torch.randn(*shp, generator=gen).to(torch.bfloat16)
+    d.g = torch.randn(*shp, generator=gen).to(torch.bfloat16)
+    d.beta = torch.randn(*shp[:3], generator=gen).to(torch.bfloat16)
+    A_log = 0.5 * torch.randn(num_heads, generator=gen)
+    dt_bias = 0.5 * torch.randn(num_heads, DK, generator=gen)
+    return d, A_log, dt_bias

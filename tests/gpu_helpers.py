@@ -84,7 +84,7 @@ def assert_parity(m):
         assert m["ckpt_rel"] <= S_TOL, m
 
 
-def decode_oracle(dinp, steps: bool = False):
+def decode_oracle(dinp, steps: bool = False, frontend=None):
     """FP64 oracle for kda_decode: every live sequence (slot in [0, P)) is a prefill
     of T tokens from its pool slot.  Returns dict with "live" (sequence indices),
     "o" [L, T, H, V], "ht" [L, H, K, V] and, with ``steps``, "steps" [L, T, H, K, V]
@@ -100,6 +100,13 @@ def decode_oracle(dinp, steps: bool = False):
     sel = lambda x: np.ascontiguousarray(x.double().numpy()[live].reshape(L * T, H, -1))
     q, k, v, g = sel(dinp.q), sel(dinp.k), sel(dinp.v), sel(dinp.g)
     beta = np.ascontiguousarray(dinp.beta.double().numpy()[live].reshape(L * T, H))
+    if frontend is not None:
+        # frontend: dict(flags, lower_bound, l2_eps, A_log, dt_bias) with oracle switch values
+        q, k, g, beta = oracle.frontend_f64(q, k, g, beta, frontend["A_log"].double().numpy(),
+                                            frontend["dt_bias"].double().numpy(),
+                                            frontend["lower_bound"], frontend["l2_eps"],
+                                            frontend["flags"])
+        q, k, g, beta = (np.ascontiguousarray(x) for x in (q, k, g, beta))
     h0 = np.ascontiguousarray(dinp.pool.double().numpy()[[idx[n] for n in live]])
     cu = np.arange(L + 1, dtype=np.int64) * T
     o, ht, _ = oracle.prefill_f64(q, k, v, g, beta, dinp.scale, cu, h0)

@@ -12,7 +12,7 @@ def dargs(N=4, T=1, H=2, P=8, **over):
     a = dict(q=BASE, k=BASE + 1 * MB, v=BASE + 2 * MB, g=BASE + 3 * MB, beta=BASE + 5 * MB,
              scale=0.088, state=BASE + 16 * MB, idx=BASE + 6 * MB,
              shape=capi.make_decode_shape(N, T, H, P), out=BASE + 8 * MB, steps=None,
-             status=None, flags=0)
+             status=None, flags=0, fe=None)
     a.update(over)
     return a
 
@@ -20,7 +20,7 @@ def dargs(N=4, T=1, H=2, P=8, **over):
 def dcall(a):
     return capi.kda_decode(a["q"], a["k"], a["v"], a["g"], a["beta"], a["scale"], a["state"],
                            a["idx"], a["shape"], a["out"], a["steps"], a["status"], a["flags"],
-                           None)
+                           None, a["fe"])
 
 
 @pytest.mark.parametrize("field", ["q", "k", "v", "g", "beta", "state", "out"])
@@ -89,3 +89,24 @@ def test_token_variant_describe_and_workspace():
     w_tok = capi.kda_prefill_workspace_size(shp, False, {"variant": capi.KDA_VARIANT_TOKEN})
     w_auto = capi.kda_prefill_workspace_size(shp, False)
     assert 0 < w_tok < w_auto // 10
+
+
+def test_decode_frontend_validation():
+    fe = lambda flags, lb=-5.0, eps=1e-6, A=BASE + 30 * MB, dt=BASE + 31 * MB: \
+        capi.make_frontend(flags, lb, eps, A, dt)
+    G, N2, B = capi.KDA_FE_GATE, capi.KDA_FE_QK_L2NORM, capi.KDA_FE_BETA_LOGIT
+    assert dcall(dargs(fe=fe(1 << 4))) == capi.KDA_ERR_BAD_OPTION           # unknown switch
+    for lb in (0.0, -5.5, 1.0, float("nan"), float("-inf")):                # bound in [-5, 0)
+        assert dcall(dargs(fe=fe(G, lb=lb))) == capi.KDA_ERR_BAD_OPTION
+    assert dcall(dargs(fe=fe(N2, eps=-1.0))) == capi.KDA_ERR_BAD_OPTION
+    assert dcall(dargs(fe=fe(N2, eps=float("nan")))) == capi.KDA_ERR_BAD_OPTION
+    assert dcall(dargs(fe=fe(G, A=None))) == capi.KDA_ERR_NULL_ARG
+    assert dcall(dargs(fe=fe(G, dt=None))) == capi.KDA_ERR_NULL_ARG
+    assert dcall(dargs(fe=fe(G, dt=BASE + 31 * MB + 4))) == capi.KDA_ERR_MISALIGNED
+    # dt_bias must not overlap an output
+    assert dcall(dargs(fe=fe(G, dt=BASE + 16 * MB))) == capi.KDA_ERR_OUT_ALIAS
+    torch = pytest.importorskip("torch")
+    if not torch.cuda.is_available():
+        # switches that need no parameters, and the full set, reach the device check
+        assert dcall(dargs(fe=fe(B | N2, A=None, dt=None))) == capi.KDA_ERR_UNSUPPORTED_DEVICE
+        assert dcall(dargs(fe=fe(G | N2 | B, lb=-5.0))) == capi.KDA_ERR_UNSUPPORTED_DEVICE

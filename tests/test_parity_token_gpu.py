@@ -6,7 +6,8 @@ import numpy as np
 import pytest
 import torch
 
-from kda_chunked_recurrent_b200.inputs import make_decode_inputs, make_inputs, workload
+from kda_chunked_recurrent_b200.inputs import (make_decode_frontend_inputs, make_decode_inputs,
+                                               make_inputs, workload)
 from tests.gpu_helpers import (O_TOL, S_TOL, assert_parity, compare, decode_oracle, rel_fro,
                                run_gpu, to_dev)
 
@@ -111,8 +112,8 @@ def _decode(K, d, **kw):
     return out.float().cpu(), pool.cpu(), None if steps is None else steps.cpu()
 
 
-def _check_decode(d, out, pool, steps=None, keep=False):
-    ref = decode_oracle(d, steps=steps is not None)
+def _check_decode(d, out, pool, steps=None, keep=False, frontend=None):
+    ref = decode_oracle(d, steps=steps is not None, frontend=frontend)
     N = d.q.shape[0]
     idx = list(range(N)) if d.state_indices is None else d.state_indices.tolist()
     live = ref["live"]
@@ -236,3 +237,39 @@ def test_decode_cuda_graph_replays():
     g.replay()
     torch.cuda.synchronize()
     _check_decode(b, out.float().cpu(), pool.cpu())
+
+
+# ------------------------------------------------------ kda_decode input front end
+# The oracle's switch values equal the library's KDA_FE_* values (1, 2, 4).
+
+@pytest.mark.parametrize("shape_flag", [2, 4])   # KDA_DECODE_NARROW, KDA_DECODE_WIDE
+@pytest.mark.parametrize("fe_flags", [7, 1, 2, 4])
+def test_decode_frontend_matches_oracle(shape_flag, fe_flags):
+    import kda_chunked_recurrent_b200 as K
+    d, A_log, dt_bias = make_decode_frontend_inputs(6, 3, 3, 9, seed=700 + fe_flags, pad_every=5)
+    if not fe_flags & 2:
+        # without the gate switch g is an FP32 log-decay in [-5, 0]
+        d.g = -5.0 * torch.sigmoid(d.g.float())
+    if not fe_flags & 4:
+        d.beta = torch.sigmoid(d.beta.float()).to(torch.bfloat16)
+    if not fe_flags & 1:
+        # without the norm switch q and k are given unit rows (the delta rule needs them)
+        unit = lambda x: (x.float() / x.float().norm(dim=-1, keepdim=True)).to(torch.bfloat16)
+        d.q, d.k = unit(d.q), unit(d.k)
+    fe = {"flags": fe_flags, "lower_bound": -4.0, "l2_eps": 1e-6, "A_log": A_log,
+          "dt_bias": dt_bias}
+    dev_fe = dict(fe, A_log=A_log.cuda(), dt_bias=dt_bias.cuda())
+    out, pool, steps = _decode(K, d, return_step_states=True, flags=shape_flag, frontend=dev_fe)
+    _check_decode(d, out, pool, steps=steps, frontend=fe)
+
+
+def test_decode_frontend_zero_rows_and_bounds():
+    # a zero q row stays finite (eps), lower_bound -5 and a steep gate rate
+    import kda_chunked_recurrent_b200 as K
+    d, A_log, dt_bias = make_decode_frontend_inputs(4, 2, 2, 4, seed=720)
+    d.q[1, 0, 1] = 0
+    A_log[0] = 3.0
+    fe = {"flags": 7, "lower_bound": -5.0, "l2_eps": 1e-6, "A_log": A_log, "dt_bias": dt_bias}
+    out, pool, _ = _decode(K, d, frontend=dict(fe, A_log=A_log.cuda(), dt_bias=dt_bias.cuda()))
+    assert torch.isfinite(out).all() and torch.isfinite(pool).all()
+    _check_decode(d, out, pool, frontend=fe)
