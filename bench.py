@@ -287,10 +287,18 @@ def run_decode(args):
     torch.cuda.set_device(local)
     import kda_chunked_recurrent_b200 as K
     from kda_chunked_recurrent_b200 import capi
-    from kda_chunked_recurrent_b200.inputs import make_decode_inputs
+    from kda_chunked_recurrent_b200.inputs import make_decode_frontend_inputs, make_decode_inputs
     N, T, H = (int(x) for x in args.decode.split(","))
-    dinp = make_decode_inputs(N, T, H, N, rank_seed(1010, rank), indices=True)
+    fe_on = args.decode_frontend
+    if fe_on:
+        dinp, A_log, dt_bias = make_decode_frontend_inputs(N, T, H, N, rank_seed(1010, rank))
+    else:
+        dinp = make_decode_inputs(N, T, H, N, rank_seed(1010, rank), indices=True)
     dev = torch.device("cuda", local)
+    fe = None
+    if fe_on:
+        A_log, dt_bias = A_log.to(dev), dt_bias.to(dev)
+        fe = capi.make_frontend(7, -5.0, 1e-6, A_log.data_ptr(), dt_bias.data_ptr())
     q, k, v, g, beta, idx = (x.to(dev) for x in (dinp.q, dinp.k, dinp.v, dinp.g, dinp.beta,
                                                   dinp.state_indices))
     pool = dinp.pool.to(dev)
@@ -302,13 +310,15 @@ def run_decode(args):
 
     def step():
         rc = capi.kda_decode(Pt(q), Pt(k), Pt(v), Pt(g), Pt(beta), dinp.scale, Pt(pool), Pt(idx),
-                             shape, Pt(out), None, Pt(status), 0, stream.cuda_stream)
+                             shape, Pt(out), None, Pt(status), 0, stream.cuda_stream, fe)
         if rc != 0:
             raise K.KDAError(rc, "kda_decode")
 
     units = N * T * H
     # bytes a decode step must move: the state slice read and written once, the token rows
-    algo_bytes = N * H * 2 * STATE_BYTES + units * PATH_BYTES_PER_TOKHEAD
+    # (with the front end the raw gate is BF16: 256 B instead of the 512 B FP32 g)
+    row_bytes = PATH_BYTES_PER_TOKHEAD - (256 if fe_on else 0)
+    algo_bytes = N * H * 2 * STATE_BYTES + units * row_bytes
     flush = None
     if algo_bytes < 2 * L2_BYTES:
         flush = torch.empty(256 * 2**20, dtype=torch.uint8, device=dev)
@@ -345,7 +355,7 @@ def run_decode(args):
     value = units * world / (ms / 1e3) / 1e6
     peaks, peak_src = load_peaks()
     achieved = algo_bytes / (kern_ms / 1e3) / 1e9
-    kname = token_kernel_name(capi, N, H)
+    kname = token_kernel_name(capi, N, H).replace("_kernel", "_fe_kernel" if fe_on else "_kernel")
     roof = {"kernel": kname, "bound": "hbm", "achieved": round(achieved, 1),
             "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
             "traffic": ncu_traffic(kname, f"decode_N{N}_T{T}_H{H}", units),
@@ -397,20 +407,27 @@ def run_decode(args):
         reps, dt = 0, 0.0
         while reps == 0 or (dt < 2.0 and reps < 200):
             t = time.perf_counter()
-            oracle.prefill_f64(qs, ks, vs, gs, bs, dinp.scale, cu, h0, threads=cores)
+            if fe_on:
+                fq, fk, fg, fb = oracle.frontend_f64(qs, ks, gs, bs, A_log.cpu().double().numpy(),
+                                                     dt_bias.cpu().double().numpy(), -5.0, 1e-6, 7)
+                oracle.prefill_f64(fq, fk, vs, fg, fb, dinp.scale, cu, h0, threads=cores)
+            else:
+                oracle.prefill_f64(qs, ks, vs, gs, bs, dinp.scale, cu, h0, threads=cores)
             dt += time.perf_counter() - t
             reps += 1
         cpu = {"value": ns * T * H * reps / dt / 1e6, "unit": UNIT, "cores": cores,
                "kind": "oracle",
                "sample": f"first {ns} of {N} sequences x {T} token(s) x {H} heads from their pool "
-                         f"slots, x {reps} run(s), FP64 per-token recurrence"}
+                         f"slots, x {reps} run(s), FP64 " + ("front end and " if fe_on else "") +
+                         "per-token recurrence"}
 
     if rank == 0:
         line = {"metric": DECODE_METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
                 "data": "synthetic",
-                "config": {"workload": f"decode_N{N}_T{T}_H{H}", "num_seqs": N, "tokens_per_seq": T,
+                "config": {"workload": f"decode_N{N}_T{T}_H{H}" + ("_frontend" if fe_on else ""),
+                           "num_seqs": N, "tokens_per_seq": T, "frontend": fe_on,
                            "heads": H, "pool_slots": N, "head_dim": 128,
                            "parallelism": f"dp{world}" if world > 1 else "single",
                            "l2": "state and rows (%.3f GB) larger than 2x L2, no flush" %
@@ -439,6 +456,8 @@ def main():
     ap.add_argument("--op", default="prefill", choices=["prefill", "decode"])
     ap.add_argument("--decode", default="256,1,12",
                     help="N,T,H of the decode workload: N sequences of T new tokens, H heads")
+    ap.add_argument("--decode-frontend", action="store_true",
+                    help="decode from raw projections through the input front end")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.op == "decode":

@@ -74,7 +74,10 @@ struct Cfg {
   static constexpr uint32_t kOffBeta = kOffQF + kBlk * kD * 4;
   static constexpr uint32_t kOffKQ = kOffBeta + kBlk * 4;
   // per token, two buffers: per warp and lane the partial sums (S'^T k)[kCPT], (S'^T q)[kCPT]
-  static constexpr uint32_t kOffPart = align128(kOffKQ + kBlk * 4);
+  // front end: dt_bias of the head [128] f32 (copied with block 0) and exp(A_log)
+  static constexpr uint32_t kOffDt = kOffKQ + kBlk * 4;
+  static constexpr uint32_t kOffRate = kOffDt + kD * 4;
+  static constexpr uint32_t kOffPart = align128(kOffRate + 16);
   static constexpr uint32_t kPartBuf = kWarps * 32 * 2 * kCPT * 4;
   static constexpr uint32_t kSmem = kOffPart + 2 * kPartBuf;
 };
@@ -201,7 +204,15 @@ __device__ __forceinline__ void token_body(const TokenParams& p, uint8_t* smem) 
     uint8_t* buf = smem + (b & 1) * C::kStage;
     const int t0 = b * kBlk, nt = min(kBlk, len - t0);
     if (warp == 0) {
-      if (lane == 0) mbar_arrive_expect_tx(&full[b & 1], static_cast<uint32_t>(nt) * tok_bytes);
+      if (lane == 0) {
+        // block 0 also brings the head's dt_bias row for the gate
+        const bool dt = fe_gate && b == 0;
+        mbar_arrive_expect_tx(&full[b & 1],
+                              static_cast<uint32_t>(nt) * tok_bytes + (dt ? kD * 4 : 0));
+        if (dt)
+          bulk_load(smem + C::kOffDt, p.dt_bias + static_cast<int64_t>(h) * kD, kD * 4,
+                    &full[0]);
+      }
       if (lane < nt) {
         const int64_t row = static_cast<int64_t>(start + t0 + lane) * tok_stride + h * kD;
         bulk_load(buf + C::kOffK + lane * kD * 2, p.k + row, kD * 2, &full[b & 1]);
@@ -243,6 +254,10 @@ __device__ __forceinline__ void token_body(const TokenParams& p, uint8_t* smem) 
       for (int c = 0; c < kCPT; ++c) s[r][c] = 0.f;
   }
   if (ck == 0) store_slice<kCPT>(p.ckpt + ck_off, s, warp, col0);
+  // exp(A_log) of the head, parked before the first block's barrier (its load overlaps
+  // the state loads and the block's copies)
+  if (fe_gate && warp == 1 && lane == 31 && nblk > 0)
+    *reinterpret_cast<float*>(smem + C::kOffRate) = expf(p.A_log[h]);
 
   float* kf = reinterpret_cast<float*>(smem + C::kOffKF);
   float* qf = reinterpret_cast<float*>(smem + C::kOffQF);
@@ -290,14 +305,13 @@ __device__ __forceinline__ void token_body(const TokenParams& p, uint8_t* smem) 
     } else {
       const uint2* ab = reinterpret_cast<const uint2*>(buf + C::kOffA);
       // gate parameters of this head for the lane's four key channels (the loop below
-      // gives lane l channels 4 l .. 4 l + 3 of every row); read per block from L1 so
+      // gives lane l channels 4 l .. 4 l + 3 of every row), from shared memory so
       // that they hold no registers across the token loop
       float rate = 0.f;
       float4 dtb = make_float4(0.f, 0.f, 0.f, 0.f);
       if (fe_gate) {
-        rate = expf(__ldg(p.A_log + h));
-        dtb = __ldg(reinterpret_cast<const float4*>(p.dt_bias + static_cast<int64_t>(h) * kD) +
-                    lane);
+        rate = *reinterpret_cast<const float*>(smem + C::kOffRate);
+        dtb = reinterpret_cast<const float4*>(smem + C::kOffDt)[lane];
       }
 #pragma unroll
       for (int j = 0; j < kBlk * kD / 4 / kThreads; ++j) {
