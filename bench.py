@@ -619,6 +619,18 @@ def main():
     path_bytes = PATH_BYTES_PER_TOKHEAD * units + state_io
     flops = FLOPS_PER_TOKHEAD_C64 * units
     s = ms / 1e3
+    # the serial part: time of the launch that runs the recurrence chains per step of
+    # the longest chain (a 64-token chunk, or a token for the token variant)
+    max_len = max(lens) if lens else 0
+    if variant == "token":
+        chain_steps, chain_ms = max_len, prep_ms + rec_ms
+    else:
+        chain_steps = (max_len + 63) // 64 + (1 if ck is not None else 0)
+        chain_ms = rec_ms if variant in ("split", "hybrid") else prep_ms + rec_ms
+    chain = {"steps_per_chain": int(chain_steps),
+             "step": "token" if variant == "token" else "chunk of 64 tokens",
+             "us_per_step": round(1e3 * chain_ms / chain_steps, 3) if chain_steps else None,
+             "launch_ms": round(chain_ms, 4)}
     path = {"bytes": int(path_bytes), "hbm_frac": round(path_bytes / s / 1e9 / peaks["hbm_gbs"], 4),
             "tc_frac_c64_burst": round(flops / s / 1e12 / peaks["bf16_tflops"], 4),
             "tc_frac_c64_sustained": round(flops / s / 1e12 / peaks["bf16_tflops_sustained"], 4),
@@ -680,7 +692,7 @@ def main():
                     if flush is None else
                     ("inputs (%.3f GB) smaller than 2x L2: 256 MB written before every step, "
                      "each step timed from its first to its last kernel" % (in_bytes / 1e9))},
-                "roofline": roof, "path_roofline": path,
+                "roofline": roof, "path_roofline": path, "chain": chain,
                 "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
                 "clocks": clk.summary()}
         print(json.dumps(line), flush=True)
