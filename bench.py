@@ -454,6 +454,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--op", default="prefill", choices=["prefill", "decode"])
+    ap.add_argument("--frontend", action="store_true",
+                    help="prefill from raw projections through the input front end")
     ap.add_argument("--decode", default="256,1,12",
                     help="N,T,H of the decode workload: N sequences of T new tokens, H heads")
     ap.add_argument("--decode-frontend", action="store_true",
@@ -473,12 +475,18 @@ def main():
     torch.cuda.set_device(local)
     import kda_chunked_recurrent_b200 as K
     from kda_chunked_recurrent_b200 import capi
-    from kda_chunked_recurrent_b200.inputs import WORKLOADS, make_inputs, ragged_lengths
+    from kda_chunked_recurrent_b200.inputs import (WORKLOADS, make_frontend_inputs, make_inputs,
+                                                   ragged_lengths)
 
     w = WORKLOADS[args.workload]
     lens = w["seqlens"] if w.get("seqlens") is not None else ragged_lengths(w["ragged"])
-    inp = make_inputs(lens, w["H"], rank_seed(w["seed"], rank), with_h0=w.get("h0", False),
-                      with_ckpt=w.get("ckpt", False), fixed_layout=w.get("fixed", False))
+    kw = dict(with_h0=w.get("h0", False), with_ckpt=w.get("ckpt", False),
+              fixed_layout=w.get("fixed", False))
+    fe_opt = None
+    if args.frontend:
+        inp, A_log, dt_bias = make_frontend_inputs(lens, w["H"], rank_seed(w["seed"], rank), **kw)
+    else:
+        inp = make_inputs(lens, w["H"], rank_seed(w["seed"], rank), **kw)
     N, T, H = inp.num_seqs, inp.total_tokens, inp.num_heads
     fixed = inp.fixed_layout
     dev = torch.device("cuda", local)
@@ -491,6 +499,9 @@ def main():
     ck = None if cko is None else torch.empty(N, H, 128, 128, dtype=torch.float32, device=dev)
     shape = capi.make_shape(N, T, H, max(lens))
     opts = {"variant": args.variant}
+    if args.frontend:
+        A_log, dt_bias = A_log.to(dev), dt_bias.to(dev)
+        opts["frontend"] = capi.make_frontend(7, -5.0, 1e-6, A_log.data_ptr(), dt_bias.data_ptr())
     ws = K.Workspace(capi.kda_prefill_workspace_size(shape, cko is not None, opts), dev)
     desc = capi.kda_prefill_describe(shape, cko is not None, opts)
     variant = desc.split()[0].split("=")[1] if desc.startswith("variant=") else "split"
@@ -571,14 +582,17 @@ def main():
 
     # ---- roofline of the dominant kernel
     peaks, peak_src = load_peaks()
+    # from raw projections the gate is read as BF16: 256 B less per token and head
+    gate_saving = 256 if args.frontend else 0
+    prep_b, path_b = PREP_BYTES_PER_TOKHEAD - gate_saving, PATH_BYTES_PER_TOKHEAD - gate_saving
     state_io = N * H * STATE_BYTES * ((1 if h0 is not None else 0) + 1 + (1 if ck is not None else 0))
     if variant == "hybrid":
         kernels = {
-            "kda_prepare_kernel": (prep_ms, hybrid_frac * PREP_BYTES_PER_TOKHEAD * units,
+            "kda_prepare_kernel": (prep_ms, hybrid_frac * prep_b * units,
                                    ["kda_prepare.cu", "kda_prepare.cuh", "kda_common.cuh",
                                     "sm100_primitives.cuh"]),
             "kda_fused_kernel": (rec_ms,
-                                 ((1 - hybrid_frac) * PREP_BYTES_PER_TOKHEAD + REC_BYTES_PER_TOKHEAD)
+                                 ((1 - hybrid_frac) * prep_b + REC_BYTES_PER_TOKHEAD)
                                  * units + state_io,
                                  ["kda_fused.cu", "kda_prepare.cuh", "kda_recurrence.cuh",
                                   "kda_common.cuh", "sm100_primitives.cuh"]),
@@ -586,26 +600,29 @@ def main():
     elif variant == "token":
         kernels = {
             token_kernel_name(capi, N, H): (prep_ms + rec_ms,
-                                            PATH_BYTES_PER_TOKHEAD * units + state_io,
+                                            path_b * units + state_io,
                                             TOKEN_SOURCES),
         }
     elif variant == "fused":
         # one launch moves both halves' bytes (the records still go through HBM/L2)
         kernels = {
             "kda_fused_kernel": (prep_ms + rec_ms,
-                                 (PREP_BYTES_PER_TOKHEAD + REC_BYTES_PER_TOKHEAD) * units + state_io,
+                                 (prep_b + REC_BYTES_PER_TOKHEAD) * units + state_io,
                                  ["kda_fused.cu", "kda_prepare.cuh", "kda_recurrence.cuh",
                                   "kda_common.cuh", "sm100_primitives.cuh"]),
         }
     else:
         kernels = {
-            "kda_prepare_kernel": (prep_ms, PREP_BYTES_PER_TOKHEAD * units,
+            "kda_prepare_kernel": (prep_ms, prep_b * units,
                                    ["kda_prepare.cu", "kda_prepare.cuh", "kda_common.cuh",
                                     "sm100_primitives.cuh"]),
             "kda_recurrence_kernel": (rec_ms, REC_BYTES_PER_TOKHEAD * units + state_io,
                                       ["kda_recurrence.cu", "kda_recurrence.cuh", "kda_common.cuh",
                                        "sm100_primitives.cuh"]),
         }
+    if args.frontend:   # the front-end instances of the prepare-side kernels
+        kernels = {(n if n == "kda_recurrence_kernel" else n.replace("_kernel", "_fe_kernel")): v
+                   for n, v in kernels.items()}
     dom = max(kernels, key=lambda n: kernels[n][0])
     dms, dbytes, _ = kernels[dom]
     achieved = dbytes / (dms / 1e3) / 1e9
@@ -616,7 +633,7 @@ def main():
             "kernel_ms": round(dms, 4),
             "algorithmic_bytes": int(dbytes),
             "per_kernel_ms": {n: round(kernels[n][0], 4) for n in kernels}}
-    path_bytes = PATH_BYTES_PER_TOKHEAD * units + state_io
+    path_bytes = path_b * units + state_io
     flops = FLOPS_PER_TOKHEAD_C64 * units
     s = ms / 1e3
     # the serial part: time of the launch that runs the recurrence chains per step of
@@ -672,8 +689,8 @@ def main():
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": round(e_ms, 3)}
 
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    cpu = None   # (the oracle baseline is timed on the plain inputs only)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.frontend:
         cpu = cpu_baseline(args.workload, max_tokens=65536, min_seconds=10.0, one_thread=True)
         cpu.pop("seconds", None)
 
@@ -686,6 +703,7 @@ def main():
                     map(str, sorted(set(lens)))) if len(set(lens)) < 4 else "ragged",
                     "total_tokens": T, "heads": H, "head_dim": 128, "h0": h0 is not None,
                     "checkpoint": ck is not None, "variant": variant,
+                    "frontend": bool(args.frontend),
                     "chunk": None if variant == "token" else 64,
                     "parallelism": f"dp{world}" if world > 1 else "single",
                     "l2": ("inputs (%.2f GB) larger than L2, no flush" % (in_bytes / 1e9))

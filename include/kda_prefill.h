@@ -113,6 +113,38 @@ enum {
                                           exercises the error path, never for production */
 };
 
+/*
+ * Optional input front end (kda_options_t.frontend for kda_prefill, the
+ * `frontend` argument of kda_decode): the kernels form the recurrence inputs from
+ * raw projections, in FP32, so that no rounded intermediate reaches the state
+ * (a BF16 copy of the normalised k or of beta would move it by about 2e-3).  The parameter set (A_log per head, dt_bias per head and key channel, a
+ * finite negative lower bound, q/k L2 normalisation, beta given as a logit) is
+ * FlashInfer PR #4262's "Dispatch contract"; the pages print no formula, and the
+ * one below is this library's reading (it puts every log-decay in
+ * (lower_bound, 0)):
+ *   KDA_FE_QK_L2NORM   q, k <- x / sqrt(sum_c x_c^2 + l2_eps) per (token, head)
+ *   KDA_FE_GATE        `g` holds the raw gate a as BF16, same layout as q (16-byte
+ *                      aligned); g_c = lower_bound * sigmoid(exp(A_log[h]) *
+ *                      (a_c + dt_bias[h][c])), sigmoid(x) = 1 / (1 + exp(-x))
+ *   KDA_FE_BETA_LOGIT  `beta` holds logits; beta <- sigmoid(beta)
+ * A_log [H] FP32 (4-byte aligned) and dt_bias [H, 128] FP32 (16-byte aligned) are
+ * device arrays, read only with KDA_FE_GATE.  lower_bound must lie in [-5, 0)
+ * (the gate bound of lmdeploy PR #5050 "Motivation"), l2_eps in [0, 1]; otherwise
+ * KDA_ERR_BAD_OPTION.
+ */
+enum {
+  KDA_FE_QK_L2NORM = 1u << 0,
+  KDA_FE_GATE = 1u << 1,
+  KDA_FE_BETA_LOGIT = 1u << 2
+};
+typedef struct {
+  uint32_t flags;        /* KDA_FE_*                                            */
+  float lower_bound;     /* KDA_FE_GATE                                         */
+  float l2_eps;          /* KDA_FE_QK_L2NORM                                    */
+  const float* A_log;    /* KDA_FE_GATE: [H]                                    */
+  const float* dt_bias;  /* KDA_FE_GATE: [H, 128]                               */
+} kda_frontend_t;
+
 typedef struct {
   int32_t variant;  /* kda_variant_t                                               */
   uint32_t flags;   /* KDA_FLAG_*                                                   */
@@ -122,7 +154,10 @@ typedef struct {
      after the last kernel of the call.  NULL entries are skipped.  The events
      let a caller time each kernel on the launching stream. */
   void* events[3];
-  int32_t reserved[4];
+  /* NULL, or the input front end (kda_frontend_t above): q, k, g and beta then hold
+     raw projections.  All variants support it. */
+  const kda_frontend_t* frontend;
+  int32_t reserved[2];
 } kda_options_t;
 
 /*
@@ -284,36 +319,6 @@ kda_status_t kda_prefill_noalloc(const void* q, const void* k, const void* v, co
  * or each other (KDA_ERR_OUT_ALIAS).  Returns KDA_OK when the launch was
  * enqueued.  No workspace and no allocation; CUDA-graph capturable.
  */
-/*
- * Optional input front end of kda_decode: the kernel forms the recurrence inputs
- * from raw projections, in FP32, so that no rounded intermediate reaches the
- * state.  The parameter set (A_log per head, dt_bias per head and key channel, a
- * finite negative lower bound, q/k L2 normalisation, beta given as a logit) is
- * FlashInfer PR #4262's "Dispatch contract"; the pages print no formula, and the
- * one below is this library's reading (it puts every log-decay in
- * (lower_bound, 0)):
- *   KDA_FE_QK_L2NORM   q, k <- x / sqrt(sum_c x_c^2 + l2_eps) per (token, head)
- *   KDA_FE_GATE        `g` holds the raw gate a as BF16 [N, T, H, 128] (16-byte
- *                      aligned); g_c = lower_bound * sigmoid(exp(A_log[h]) *
- *                      (a_c + dt_bias[h][c])), sigmoid(x) = 1 / (1 + exp(-x))
- *   KDA_FE_BETA_LOGIT  `beta` holds logits; beta <- sigmoid(beta)
- * A_log [H] FP32 (4-byte aligned) and dt_bias [H, 128] FP32 (16-byte aligned) are
- * device arrays, read only with KDA_FE_GATE.  lower_bound must lie in [-5, 0)
- * (the gate bound of lmdeploy PR #5050 "Motivation"), l2_eps in [0, 1]; otherwise
- * KDA_ERR_BAD_OPTION.
- */
-enum {
-  KDA_FE_QK_L2NORM = 1u << 0,
-  KDA_FE_GATE = 1u << 1,
-  KDA_FE_BETA_LOGIT = 1u << 2
-};
-typedef struct {
-  uint32_t flags;        /* KDA_FE_*                                            */
-  float lower_bound;     /* KDA_FE_GATE                                         */
-  float l2_eps;          /* KDA_FE_QK_L2NORM                                    */
-  const float* A_log;    /* KDA_FE_GATE: [H]                                    */
-  const float* dt_bias;  /* KDA_FE_GATE: [H, 128]                               */
-} kda_frontend_t;
 
 typedef struct {
   int32_t num_seqs;       /* N >= 1                                               */

@@ -77,13 +77,17 @@ class Workspace:
 def prefill(q, k, v, g, beta, scale: float, *, h0=None, cu_seqlens=None, num_seqs=None,
             max_seqlen: int = 0, ckpt_offsets=None, out=None, ht=None, ckpt_state=None,
             output_final_state: bool = True, workspace: Optional[Workspace] = None,
-            variant: int = KDA_VARIANT_AUTO, flags: int = 0, stream=None):
+            variant: int = KDA_VARIANT_AUTO, flags: int = 0, frontend: Optional[dict] = None,
+            stream=None):
     """Launch KDA prefill on device tensors.
 
     q, k, v: [T, H, 128] bf16; g: [T, H, 128] fp32; beta: [T, H] bf16;
     h0/ht/ckpt_state: [N, H, 128, 128] fp32; cu_seqlens: int32 or int64;
     ckpt_offsets: int32.
     Without cu_seqlens, ``num_seqs`` (default 1) equal-length sequences are assumed.
+    ``frontend``: dict(flags=KDA_FE_*, lower_bound=..., l2_eps=..., A_log=[H] fp32,
+    dt_bias=[H, 128] fp32) to start from raw projections (with KDA_FE_GATE, ``g`` is the
+    raw gate in bf16).
     Returns (out, ht, ckpt_state).
     """
     import torch
@@ -101,6 +105,11 @@ def prefill(q, k, v, g, beta, scale: float, *, h0=None, cu_seqlens=None, num_seq
     if cu_seqlens is not None and cu_seqlens.dtype == torch.int64:
         flags |= KDA_FLAG_CU_SEQLENS_I64   # INT64 offsets, narrowed on the device
     opts = {"variant": variant, "flags": flags}
+    if frontend is not None:
+        opts["frontend"] = capi.make_frontend(
+            frontend.get("flags", 0), frontend.get("lower_bound", 0.0),
+            frontend.get("l2_eps", 0.0), _ptr(frontend.get("A_log")),
+            _ptr(frontend.get("dt_bias")))
     s = stream if stream is not None else torch.cuda.current_stream(dev)
     need = capi.kda_prefill_workspace_size(shape, ckpt_offsets is not None, opts)
     if need == 0:

@@ -63,7 +63,8 @@ class kda_frontend_t(ctypes.Structure):
 
 class kda_options_t(ctypes.Structure):
     _fields_ = [("variant", ctypes.c_int32), ("flags", ctypes.c_uint32),
-                ("events", ctypes.c_void_p * 3), ("reserved", ctypes.c_int32 * 4)]
+                ("events", ctypes.c_void_p * 3), ("frontend", ctypes.POINTER(kda_frontend_t)),
+                ("reserved", ctypes.c_int32 * 2)]
 
 
 def _load():
@@ -110,6 +111,10 @@ def _opt(options):
     o.flags = int(options.get("flags", 0))
     for i, ev in enumerate(options.get("events") or ()):
         o.events[i] = ev
+    fe = options.get("frontend")
+    if fe is not None:
+        o._fe = fe if isinstance(fe, kda_frontend_t) else make_frontend(**fe)
+        o.frontend = ctypes.pointer(o._fe)
     return ctypes.byref(o)
 
 

@@ -23,6 +23,9 @@
 namespace kda {
 __global__ void kda_schedule_kernel(const KdaParams p);
 __global__ void kda_prepare_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps);
+__global__ void kda_prepare_fe_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps);
+__global__ void kda_fused_fe_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps,
+                                    int32_t rec_ctas, int64_t prep_items, int32_t prep_groups);
 __global__ void kda_recurrence_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps);
 __global__ void kda_fused_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps,
                                  int32_t rec_ctas, int64_t prep_items, int32_t prep_groups);
@@ -91,6 +94,30 @@ kda_status_t check_options(const kda_options_t* o) {
                                          KDA_FLAG_CU_SEQLENS_I64)))
     return KDA_ERR_BAD_OPTION;
   return KDA_OK;
+}
+
+// The input front end's switches and parameters (pointers only; values of the
+// device arrays are never read on the host).
+kda_status_t check_frontend(const kda_frontend_t* fe) {
+  if (!fe) return KDA_OK;
+  if (fe->flags & ~static_cast<uint32_t>(KDA_FE_QK_L2NORM | KDA_FE_GATE | KDA_FE_BETA_LOGIT))
+    return KDA_ERR_BAD_OPTION;
+  if (fe->flags & KDA_FE_GATE) {
+    if (!fe->A_log || !fe->dt_bias) return KDA_ERR_NULL_ARG;
+    const float lb = fe->lower_bound;
+    if (!(lb >= -5.0f && lb < 0.0f)) return KDA_ERR_BAD_OPTION;   // also rejects NaN
+    if ((reinterpret_cast<uintptr_t>(fe->A_log) % 4) || (reinterpret_cast<uintptr_t>(fe->dt_bias) % 16))
+      return KDA_ERR_MISALIGNED;
+  }
+  if ((fe->flags & KDA_FE_QK_L2NORM) && !(fe->l2_eps >= 0.0f && fe->l2_eps <= 1.0f))
+    return KDA_ERR_BAD_OPTION;
+  return KDA_OK;
+}
+
+uint32_t fe_bits(const kda_frontend_t* fe) {
+  const uint32_t f = fe ? fe->flags : 0u;
+  return (f & KDA_FE_QK_L2NORM ? 1u : 0u) | (f & KDA_FE_GATE ? 2u : 0u) |
+         (f & KDA_FE_BETA_LOGIT ? 4u : 0u);
 }
 
 kda_status_t check_shape(const kda_shape_t* s, bool fixed, bool ckpt) {
@@ -402,6 +429,10 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
   if (T > 0 && (!q || !k || !v || !g || !beta || !out)) return KDA_ERR_NULL_ARG;
   if (!workspace) return KDA_ERR_NULL_ARG;
   if ((ckpt_state == nullptr) != (ckpt_offsets == nullptr)) return KDA_ERR_UNPAIRED_CKPT;
+  const kda_frontend_t* fe = options ? options->frontend : nullptr;
+  st = check_frontend(fe);
+  if (st != KDA_OK) return st;
+  const bool fe_gate = fe && (fe->flags & KDA_FE_GATE);
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(g, 16) ||
       !aligned(out, 16) || !aligned(beta, 2) || !aligned(h0, 16) || !aligned(ht, 16) ||
       !aligned(ckpt_state, 16) || !aligned(cu_seqlens, cu_elem) || !aligned(ckpt_offsets, 4) ||
@@ -410,14 +441,16 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
   const size_t tok16 = static_cast<size_t>(T * H * 128 * 2);
   const size_t state = static_cast<size_t>(N * H * 128 * 128 * 4);
   const Range rq = rng(q, tok16), rk = rng(k, tok16), rv = rng(v, tok16),
-              rg = rng(g, tok16 * 2), rb = rng(beta, static_cast<size_t>(T * H * 2)),
+              rg = rng(g, fe_gate ? tok16 : tok16 * 2), rb = rng(beta, static_cast<size_t>(T * H * 2)),
               rh0 = rng(h0, state), rht = rng(ht, state), rck = rng(ckpt_state, state),
               rcu = rng(cu_seqlens, static_cast<size_t>(N + 1) * cu_elem),
               rco = rng(ckpt_offsets, static_cast<size_t>(N * 4)),
-              rws = rng(workspace, workspace_bytes), ro = rng(out, tok16);
+              rws = rng(workspace, workspace_bytes), ro = rng(out, tok16),
+              ra = rng(fe_gate ? fe->A_log : nullptr, static_cast<size_t>(H * 4)),
+              rdt = rng(fe_gate ? fe->dt_bias : nullptr, static_cast<size_t>(H * 128 * 4));
   if (overlap(rh0, rht) && h0 != ht) return KDA_ERR_PARTIAL_ALIAS;
   if (overlap(rck, rh0) || overlap(rck, rht)) return KDA_ERR_PARTIAL_ALIAS;
-  const Range inputs[] = {rq, rk, rv, rg, rb, rcu, rco};
+  const Range inputs[] = {rq, rk, rv, rg, rb, rcu, rco, ra, rdt};
   for (const Range& in : inputs) {
     if (overlap(ro, in) || overlap(rht, in) || overlap(rck, in) || overlap(rws, in))
       return KDA_ERR_OUT_ALIAS;
@@ -470,6 +503,13 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
   p.slots = r.lay.slots;
   p.flags = flags;
   p.wait_budget = (flags & KDA_FLAG_TEST_FORCE_TIMEOUT) ? -1 : kDefaultWaitBudget;
+  p.fe_flags = fe_bits(fe);
+  if (fe_gate) {
+    p.A_log = fe->A_log;
+    p.dt_bias = fe->dt_bias;
+    p.lower_bound = fe->lower_bound;
+  }
+  if (fe && (fe->flags & KDA_FE_QK_L2NORM)) p.l2_eps = fe->l2_eps;
 
   // ---------------- tensor maps (encoded per call; passed by value)
   SplitMaps maps;
@@ -481,7 +521,10 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
     mok &= make_map_tokens(&maps.v_in, v, T, H);
     mok &= make_map_rows(&maps.q_in, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, T, H, 2);
     mok &= make_map_rows(&maps.k_in, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, k, T, H, 2);
-    mok &= make_map_rows(&maps.g_in, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, g, T, H, 4);
+    if (fe_gate)   // the raw gate, BF16
+      mok &= make_map_rows(&maps.g_in, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g, T, H, 2);
+    else
+      mok &= make_map_rows(&maps.g_in, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, g, T, H, 4);
     mok &= make_map_rows(&maps.o_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, out, T, H, 2);
     mok &= make_map_2d(&maps.wt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ws + r.lay.wt, 64, recs * 128, 64, 128, 2);
     mok &= make_map_2d(&maps.qg, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ws + r.lay.qg, 128, recs * 64, 64, 64, 2);
@@ -505,7 +548,15 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
     cudaError_t e3 = cudaFuncSetAttribute(kda_fused_kernel,
                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           fused::kSmemAllocBytes);
-    attr_err = (e1 != cudaSuccess) ? e1 : (e2 != cudaSuccess ? e2 : e3);
+    cudaError_t e4 = cudaFuncSetAttribute(kda_prepare_fe_kernel,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          prep::kSmemAllocBytes);
+    cudaError_t e5 = cudaFuncSetAttribute(kda_fused_fe_kernel,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          fused::kSmemAllocBytes);
+    const cudaError_t es[] = {e1, e2, e3, e4, e5};
+    for (cudaError_t e : es)
+      if (attr_err == cudaSuccess) attr_err = e;
   });
   if (attr_err != cudaSuccess) return KDA_ERR_LAUNCH_FAILED;
   (void)cudaGetLastError();
@@ -544,6 +595,11 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
     tp.status = reinterpret_cast<int32_t*>(p.ws);
     tp.flags = flags;
     tp.wait_budget = p.wait_budget;
+    tp.fe_flags = p.fe_flags;
+    tp.A_log = p.A_log;
+    tp.dt_bias = p.dt_bias;
+    tp.lower_bound = p.lower_bound;
+    tp.l2_eps = p.l2_eps;
     st = launch_token(tp, N * H, token_wide(N * H, 0), s);
     if (st != KDA_OK) return st;
     mark(2);
@@ -556,7 +612,10 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
       p.split_jmax = static_cast<int32_t>(j0);
       const int64_t items = r.lay.slots * H;
       const int64_t pgrid = std::min<int64_t>(items, 2 * static_cast<int64_t>(sm_count()));
-      kda_prepare_kernel<<<static_cast<unsigned>(pgrid), 256, prep::kSmemAllocBytes, s>>>(p, maps);
+      if (p.fe_flags)
+        kda_prepare_fe_kernel<<<static_cast<unsigned>(pgrid), 256, prep::kSmemAllocBytes, s>>>(p, maps);
+      else
+        kda_prepare_kernel<<<static_cast<unsigned>(pgrid), 256, prep::kSmemAllocBytes, s>>>(p, maps);
       p.split_jmax = INT32_MAX;
     }
     p.fused_j0 = static_cast<int32_t>(j0);
@@ -564,7 +623,9 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
     // one cooperative launch: CTAs 0 .. N H - 1 run the recurrences, the rest of
     // the SMs (one CTA each) prepare the chunk records in chunk-major order
     int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kda_fused_kernel,
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm,
+                                                      p.fe_flags ? kda_fused_fe_kernel
+                                                                 : kda_fused_kernel,
                                                       fused::kThreadsPerCta,
                                                       fused::kSmemAllocBytes) != cudaSuccess ||
         per_sm < 1)
@@ -578,7 +639,9 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
       return KDA_ERR_LAUNCH_FAILED;
     int32_t prep_groups = rec_ctas <= kFusedOneGroupMaxChains ? 1 : 2;
     void* args[] = {&p, &maps, &rec_ctas, &prep_items, &prep_groups};
-    if (cudaLaunchCooperativeKernel(reinterpret_cast<void*>(kda_fused_kernel), dim3(grid),
+    void* fused_fn = p.fe_flags ? reinterpret_cast<void*>(kda_fused_fe_kernel)
+                                : reinterpret_cast<void*>(kda_fused_kernel);
+    if (cudaLaunchCooperativeKernel(fused_fn, dim3(grid),
                                     dim3(fused::kThreadsPerCta), args, fused::kSmemAllocBytes,
                                     s) != cudaSuccess)
       return KDA_ERR_LAUNCH_FAILED;
@@ -588,7 +651,10 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
       // persistent prepare grid: two CTAs per SM walk the (chunk slot, head) items
       const int64_t items = r.lay.slots * H;
       const int64_t grid = std::min<int64_t>(items, 2 * static_cast<int64_t>(sm_count()));
-      kda_prepare_kernel<<<static_cast<unsigned>(grid), 256, prep::kSmemAllocBytes, s>>>(p, maps);
+      if (p.fe_flags)
+        kda_prepare_fe_kernel<<<static_cast<unsigned>(grid), 256, prep::kSmemAllocBytes, s>>>(p, maps);
+      else
+        kda_prepare_kernel<<<static_cast<unsigned>(grid), 256, prep::kSmemAllocBytes, s>>>(p, maps);
     }
     mark(1);
     kda_recurrence_kernel<<<static_cast<unsigned>(N * H), rec::kThreadsPerCta,
@@ -606,16 +672,10 @@ kda_status_t kda_decode(const void* q, const void* k, const void* v, const float
                         const kda_frontend_t* frontend, void* stream) {
   if (!shape) return KDA_ERR_NULL_ARG;
   const uint32_t fe = frontend ? frontend->flags : 0u;
-  if (fe & ~static_cast<uint32_t>(KDA_FE_QK_L2NORM | KDA_FE_GATE | KDA_FE_BETA_LOGIT))
-    return KDA_ERR_BAD_OPTION;
-  if (fe & KDA_FE_GATE) {
-    if (!frontend->A_log || !frontend->dt_bias) return KDA_ERR_NULL_ARG;
-    const float lb = frontend->lower_bound;
-    if (!(lb >= -5.0f && lb < 0.0f)) return KDA_ERR_BAD_OPTION;   // also rejects NaN
+  {
+    const kda_status_t fst = check_frontend(frontend);
+    if (fst != KDA_OK && fst != KDA_ERR_MISALIGNED) return fst;   // alignment after NULL checks
   }
-  if ((fe & KDA_FE_QK_L2NORM) &&
-      !(frontend->l2_eps >= 0.0f && frontend->l2_eps <= 1.0f))   // finite, non-negative
-    return KDA_ERR_BAD_OPTION;
   if (flags & ~static_cast<uint32_t>(KDA_DECODE_KEEP_STATE | KDA_DECODE_NARROW |
                                      KDA_DECODE_WIDE))
     return KDA_ERR_BAD_OPTION;
@@ -632,8 +692,7 @@ kda_status_t kda_decode(const void* q, const void* k, const void* v, const float
       !aligned(out, 16) || !aligned(beta, 2) || !aligned(state, 16) ||
       !aligned(step_states, 16) || !aligned(state_indices, 4) || !aligned(device_status, 4))
     return KDA_ERR_MISALIGNED;
-  if ((fe & KDA_FE_GATE) && (!aligned(frontend->A_log, 4) || !aligned(frontend->dt_bias, 16)))
-    return KDA_ERR_MISALIGNED;
+  if (check_frontend(frontend) != KDA_OK) return KDA_ERR_MISALIGNED;
   const size_t tok16 = static_cast<size_t>(N * T * H * 128 * 2);
   const size_t g_bytes = (fe & KDA_FE_GATE) ? tok16 : tok16 * 2;   // raw BF16 gate or FP32 g
   const size_t st1 = static_cast<size_t>(H * 128 * 128 * 4);   // one slot, all heads
@@ -678,8 +737,7 @@ kda_status_t kda_decode(const void* q, const void* k, const void* v, const float
   tp.status = device_status;
   tp.flags = 0;
   tp.wait_budget = kDefaultWaitBudget;
-  tp.fe_flags = (fe & KDA_FE_QK_L2NORM ? kFeQkL2Norm : 0u) | (fe & KDA_FE_GATE ? kFeGate : 0u) |
-                (fe & KDA_FE_BETA_LOGIT ? kFeBetaLogit : 0u);
+  tp.fe_flags = fe_bits(frontend);
   if (gate) {
     tp.A_log = frontend->A_log;
     tp.dt_bias = frontend->dt_bias;

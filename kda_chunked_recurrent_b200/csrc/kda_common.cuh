@@ -120,6 +120,13 @@ struct KdaParams {
   WorkspaceLayout lay;
   uint32_t flags;
   long long wait_budget;         // clock cycles per bounded wait; < 0 forces a timeout
+  // input front end (0: inputs used as given; bit 0 q/k L2 norm, bit 1 gate from the
+  // raw BF16 gate in g, bit 2 beta from its logit), formed in FP32 by the prepare kernel
+  uint32_t fe_flags;
+  const float* A_log;            // [H]
+  const float* dt_bias;          // [H][128]
+  float lower_bound;
+  float l2_eps;
 };
 
 // Tensor maps of the split variant (passed by value, __grid_constant__).

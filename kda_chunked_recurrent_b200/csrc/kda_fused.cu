@@ -24,9 +24,10 @@ static_assert(rec::kThreads <= kThreads, "recurrence warps fit the CTA");
 
 // prep_groups: prepare groups per prepare CTA (1 or 2).  Few chains need little
 // prepare throughput, and one group then leaves more memory bandwidth to them.
-__global__ void __launch_bounds__(fused::kThreads, 1)
-kda_fused_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps, int32_t rec_ctas,
-                 int64_t prep_items, int32_t prep_groups) {
+template <bool kFE>
+__device__ __forceinline__ void fused_body(const KdaParams& p, const SplitMaps& maps,
+                                           int32_t rec_ctas, int64_t prep_items,
+                                           int32_t prep_groups) {
   extern __shared__ uint8_t smem_raw[];
   if (static_cast<int32_t>(blockIdx.x) < rec_ctas) {
     recurrence_body<true>(p, maps, smem_raw, blockIdx.x);
@@ -34,10 +35,23 @@ kda_fused_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps, int3
     const int grp = threadIdx.x / prep::kThreads;
     if (grp >= prep_groups) return;
     const int64_t groups = prep_groups * static_cast<int64_t>(gridDim.x - rec_ctas);
-    prepare_body<true>(p, maps, smem_raw, grp,
-                       prep_groups * static_cast<int64_t>(blockIdx.x - rec_ctas) + grp, groups,
-                       prep_items);
+    prepare_body<true, kFE>(p, maps, smem_raw, grp,
+                            prep_groups * static_cast<int64_t>(blockIdx.x - rec_ctas) + grp,
+                            groups, prep_items);
   }
+}
+
+__global__ void __launch_bounds__(fused::kThreads, 1)
+kda_fused_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps, int32_t rec_ctas,
+                 int64_t prep_items, int32_t prep_groups) {
+  fused_body<false>(p, maps, rec_ctas, prep_items, prep_groups);
+}
+
+// the same with the input front end compiled into the prepare side
+__global__ void __launch_bounds__(fused::kThreads, 1)
+kda_fused_fe_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps, int32_t rec_ctas,
+                    int64_t prep_items, int32_t prep_groups) {
+  fused_body<true>(p, maps, rec_ctas, prep_items, prep_groups);
 }
 
 }  // namespace kda

@@ -94,7 +94,8 @@ constexpr uint32_t kAuxTmem = kAux + 32;         // u32 TMEM base
 constexpr uint32_t kAuxBeta = kAux + 64;         // f32 [64]
 constexpr uint32_t kAuxTot = kAuxBeta + 256;     // float2 [4][64]
 constexpr uint32_t kAuxFirst = kAuxTot + 2048;   // float2 [4][64]
-constexpr uint32_t kGroupBytes = (kAuxFirst + 2048 + 1023) / 1024 * 1024;   // one prepare group
+constexpr uint32_t kAuxNorm = kAuxFirst + 2048;  // f32 [2][64] inverse norms of k, q rows (front end)
+constexpr uint32_t kGroupBytes = (kAuxNorm + 512 + 1023) / 1024 * 1024;   // one prepare group
 constexpr uint32_t kSmemAlloc = kGroupBytes + 1024;
 static_assert(kZh + 64 * kLdh * 2 <= kR, "solve scratch overlaps the Aqk staging tile");
 static_assert(kAqs + 8192 <= kTb, "Aqk staging overlaps the Tb tile");
@@ -318,7 +319,11 @@ __device__ __forceinline__ void publish_record(const KdaParams& p, int64_t rec) 
 // memory is the grp-th kGroupBytes slice).  Items first, first + stride, ... <
 // nitems; kFused selects the chunk-major item order, the named barriers and the
 // ready flags.
-template <bool kFused>
+// kFE: the input front end is compiled in (switches in p.fe_flags): the gate is formed
+// from the raw BF16 gate tile in the scan, the inverse L2 norms of the k and q rows are
+// folded into the FP32 factors that already multiply them (so every operand keeps its
+// single rounding), and beta is squashed from its logit when parked.
+template <bool kFused, bool kFE = false>
 __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps& maps,
                                              uint8_t* smem_raw, int grp, int64_t first,
                                              int64_t stride, int64_t nitems) {
@@ -335,6 +340,11 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
   float* s_beta = reinterpret_cast<float*>(sm + kAuxBeta);
   float2 (*s_tot)[64] = reinterpret_cast<float2 (*)[64]>(sm + kAuxTot);     // per sub-block sums of g
   float2 (*s_first)[64] = reinterpret_cast<float2 (*)[64]>(sm + kAuxFirst); // first token's running sum
+  float* s_norm = reinterpret_cast<float*>(sm + kAuxNorm);   // front end: 1/|k_r|, then 1/|q_r|
+  const bool fe_gate = kFE && (p.fe_flags & 2u) != 0;
+  const bool fe_norm = kFE && (p.fe_flags & 1u) != 0;
+  const bool fe_beta = kFE && (p.fe_flags & 4u) != 0;
+  const uint32_t raw_g_tx = fe_gate ? 16384u : kRawGTx;   // raw gate tile is BF16
 
   const int tid = threadIdx.x - grp * kThreads;
   const int warp = tid >> 5, lane = tid & 31;
@@ -380,7 +390,7 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
     tma_load_3d(sm + kKraw, &maps.k_in, &raw_qk_bar, 0, it.h, it.t0);
   };
   auto issue_g = [&](const PrepItem& it) {  // thread kGThread only, its Aqk stores read
-    mbar_arrive_expect_tx(&raw_g_bar, kRawGTx);
+    mbar_arrive_expect_tx(&raw_g_bar, raw_g_tx);
     tma_load_3d(sm + kGraw, &maps.g_in, &raw_g_bar, 0, it.h, it.t0);
   };
 
@@ -415,6 +425,14 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
     qk_for_cur = g_for_cur = false;
     uint16_t beta_raw = 0;   // consumed only after the operand pass, so its latency hides
     if (tid < c) beta_raw = p.beta[static_cast<int64_t>(t0 + tid) * p.H + h];
+    float fe_rate = 0.f;                          // front end: exp(A_log[h]), dt_bias pair
+    float2 fe_dtb = make_float2(0.f, 0.f);
+    if constexpr (kFE) {
+      if (fe_gate) {
+        fe_rate = expf(__ldg(p.A_log + h));
+        fe_dtb = __ldg(reinterpret_cast<const float2*>(p.dt_bias + static_cast<int64_t>(h) * kD) + cp);
+      }
+    }
 
     // ---- L2 prefetch of the next item's tiles (q, k, g, v) and beta rows
     if (nxt_valid) {
@@ -448,9 +466,44 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const bool in = ok && blk * 16 + i < c;   // rows past the chunk read as zero
-        G[i] = in ? gs[i * 64] : make_float2(0.f, 0.f);
+        if (fe_gate) {
+          // g = lower_bound * sigmoid(exp(A_log) (a + dt_bias)) from the raw BF16 gate a
+          const uint32_t a2 = in ? reinterpret_cast<const uint32_t*>(sm + kGraw)[(blk * 16 + i) * 64 + cp] : 0u;
+          const float2 a = bf2_to_f2(a2);
+          const float x0 = fe_rate * (a.x + fe_dtb.x), x1 = fe_rate * (a.y + fe_dtb.y);
+          G[i] = in ? make_float2(p.lower_bound / (1.f + ex2(-x0 * kLog2e)),
+                                  p.lower_bound / (1.f + ex2(-x1 * kLog2e)))
+                    : make_float2(0.f, 0.f);
+        } else {
+          G[i] = in ? gs[i * 64] : make_float2(0.f, 0.f);
+        }
         kw[i] = in ? ks[i * 64] : 0u;
         qw[i] = in ? qs[i * 64] : 0u;
+      }
+    }
+    if constexpr (kFE) {
+      if (fe_norm) {   // (warp-uniform; on a failed wait the values are never used)
+        // inverse L2 norms of the chunk's k and q rows: warp w takes rows 8 w .. 8 w + 7,
+        // lane l channels 4 l .. 4 l + 3 (the raw tiles are intact until the barrier below)
+        const uint2* kr = reinterpret_cast<const uint2*>(sm + kKraw);
+        const uint2* qr = reinterpret_cast<const uint2*>(sm + kQraw);
+#pragma unroll 2
+        for (int rr = 0; rr < 8; ++rr) {
+          const int row = warp * 8 + rr;
+          const float2 k01 = bf2_to_f2(kr[row * 32 + lane].x), k23 = bf2_to_f2(kr[row * 32 + lane].y);
+          const float2 q01 = bf2_to_f2(qr[row * 32 + lane].x), q23 = bf2_to_f2(qr[row * 32 + lane].y);
+          float sk = fmaf(k01.x, k01.x, fmaf(k01.y, k01.y, fmaf(k23.x, k23.x, k23.y * k23.y)));
+          float sq = fmaf(q01.x, q01.x, fmaf(q01.y, q01.y, fmaf(q23.x, q23.x, q23.y * q23.y)));
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) {
+            sk += __shfl_xor_sync(0xffffffffu, sk, o);
+            sq += __shfl_xor_sync(0xffffffffu, sq, o);
+          }
+          if (lane == 0) {
+            s_norm[row] = rsqrtf(sk + p.l2_eps);
+            s_norm[64 + row] = rsqrtf(sq + p.l2_eps);
+          }
+        }
       }
     }
     // ---- gate scan within the sub-block; one exchange gives every sub-block start
@@ -529,20 +582,37 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
       for (int i = 0; i < 16; ++i) {
         const uint32_t xo = ((chunk ^ static_cast<uint32_t>(i & 7)) << 4) + static_cast<uint32_t>(i) * 128u;
         const float2 g2 = G[i];
-        const float e0 = ex2(g2.x - B.x), e1 = ex2(g2.y - B.y);
-        const float i0 = ex2(B.x - g2.x), i1 = ex2(B.y - g2.y);
-        // bf16 operands: factors rounded to bf16, products in packed bf16 math
-        const uint32_t e2 = pack_bf16(e0, e1), inv2 = pack_bf16(i0, i1);
-        sts32(bL + xo, hmul2_bf16(kw[i], e2));
-        sts32(bL + xo + 64u * 128u, hmul2_bf16(qw[i], e2));
-        const uint32_t rd2 = hmul2_bf16(kw[i], inv2);
-        sts32(bRo + xo, rd2);
-        if (blk < 1) sts32(bR + xo + 16u * 128u, hmul2_bf16(rd2, c1b));
-        if (blk < 2) sts32(bR + xo + 48u * 128u, hmul2_bf16(rd2, c2b));
-        if (blk < 3) sts32(bR + xo + 96u * 128u, hmul2_bf16(rd2, c3b));
-        const uint32_t gm2 = hmul2_bf16(e2, cB2);
-        sts32(bKG + xo, hmul2_bf16(kw[i], gm2));
-        qg_out[i * 64] = hmul2_bf16(qw[i], gm2);
+        float e0 = ex2(g2.x - B.x), e1 = ex2(g2.y - B.y);
+        float i0 = ex2(B.x - g2.x), i1 = ex2(B.y - g2.y);
+        if (kFE && fe_norm) {
+          // front end: the row's inverse norms ride on the FP32 factors (one rounding each)
+          const float rk = s_norm[blk * 16 + i], rq = s_norm[64 + blk * 16 + i];
+          const uint32_t e2k = pack_bf16(e0 * rk, e1 * rk), e2q = pack_bf16(e0 * rq, e1 * rq);
+          sts32(bL + xo, hmul2_bf16(kw[i], e2k));
+          sts32(bL + xo + 64u * 128u, hmul2_bf16(qw[i], e2q));
+          const uint32_t rd2 = hmul2_bf16(kw[i], pack_bf16(i0 * rk, i1 * rk));
+          sts32(bRo + xo, rd2);
+          if (blk < 1) sts32(bR + xo + 16u * 128u, hmul2_bf16(rd2, c1b));
+          if (blk < 2) sts32(bR + xo + 48u * 128u, hmul2_bf16(rd2, c2b));
+          if (blk < 3) sts32(bR + xo + 96u * 128u, hmul2_bf16(rd2, c3b));
+          sts32(bKG + xo, hmul2_bf16(kw[i], pack_bf16(e0 * cB.x * rk, e1 * cB.y * rk)));
+          qg_out[i * 64] = hmul2_bf16(qw[i], pack_bf16(e0 * cB.x * rq, e1 * cB.y * rq));
+          i0 *= rk;
+          i1 *= rk;
+        } else {
+          // bf16 operands: factors rounded to bf16, products in packed bf16 math
+          const uint32_t e2 = pack_bf16(e0, e1), inv2 = pack_bf16(i0, i1);
+          sts32(bL + xo, hmul2_bf16(kw[i], e2));
+          sts32(bL + xo + 64u * 128u, hmul2_bf16(qw[i], e2));
+          const uint32_t rd2 = hmul2_bf16(kw[i], inv2);
+          sts32(bRo + xo, rd2);
+          if (blk < 1) sts32(bR + xo + 16u * 128u, hmul2_bf16(rd2, c1b));
+          if (blk < 2) sts32(bR + xo + 48u * 128u, hmul2_bf16(rd2, c2b));
+          if (blk < 3) sts32(bR + xo + 96u * 128u, hmul2_bf16(rd2, c3b));
+          const uint32_t gm2 = hmul2_bf16(e2, cB2);
+          sts32(bKG + xo, hmul2_bf16(kw[i], gm2));
+          qg_out[i * 64] = hmul2_bf16(qw[i], gm2);
+        }
         // Kd feeds the FP16 state update: FP32 products, one rounding
         const float2 kf = bf2_to_f2(kw[i]);
         kd_out[i * 64] = pack_f16(kf.x * i0 * cE.x, kf.y * i1 * cE.y);
@@ -551,7 +621,10 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
         reinterpret_cast<float2*>(p.ws + p.lay.gc + rec * kTileGC)[cp] =
             make_float2(ex2(E.x), ex2(E.y));
     }
-    if (tid < kC) s_beta[tid] = bf16_to_f32(beta_raw);
+    if (tid < kC) {
+      const float b = bf16_to_f32(beta_raw);
+      s_beta[tid] = fe_beta ? 1.f / (1.f + ex2(-b * kLog2e)) : b;
+    }
 
     // ---- UMMA 1: D[0:128, 0:160] = [K+; Q+] . R^T   (bf16 -> f32)
     fence_proxy_async_smem();

@@ -173,3 +173,23 @@ def make_decode_frontend_inputs(num_seqs: int, tokens: int, num_heads: int, pool
     A_log = 0.5 * torch.randn(num_heads, generator=gen)
     dt_bias = 0.5 * torch.randn(num_heads, DK, generator=gen)
     return d, A_log, dt_bias
+
+
+def make_frontend_inputs(seqlens: List[int], num_heads: int, seed: int, *, with_h0: bool = False,
+                         with_ckpt: bool = False, fixed_layout: bool = False):
+    """Raw projections for a prefill through the input front end: the KDAInputs of
+    make_inputs with q, k replaced by N(0, 1) BF16 rows (not normalised), the ``g``
+    field by the raw gate ~ N(0, 1) BF16 and ``beta`` by logits ~ N(0, 1) BF16; plus
+    A_log ~ N(0, 0.5) FP32 [H] and dt_bias ~ N(0, 0.5) FP32 [H, 128].
+    Returns (KDAInputs, A_log, dt_bias)."""
+    inp = make_inputs(seqlens, num_heads, seed, with_h0=with_h0, with_ckpt=with_ckpt,
+                      fixed_layout=fixed_layout)
+    gen = torch.Generator().manual_seed(int(seed) + 13)
+    T, H = inp.total_tokens, inp.num_heads
+    inp.q = torch.randn(T, H, DK, generator=gen).to(torch.bfloat16)
+    inp.k = torch.randn(T, H, DK, generator=gen).to(torch.bfloat16)
+    inp.g = torch.randn(T, H, DK, generator=gen).to(torch.bfloat16)
+    inp.beta = torch.randn(T, H, generator=gen).to(torch.bfloat16)
+    A_log = 0.5 * torch.randn(H, generator=gen)
+    dt_bias = 0.5 * torch.randn(H, DK, generator=gen)
+    return inp, A_log, dt_bias

@@ -25,7 +25,7 @@ def to_dev(inp):
 
 
 def run_gpu(inp, *, inplace=False, flags=0, variant=0, fixed=None, workspace=None,
-            h0_override=None):
+            h0_override=None, frontend=None):
     """Run kda_prefill on inp; returns dict of CPU tensors and the device status word."""
     import kda_chunked_recurrent_b200 as K
     d = to_dev(inp)
@@ -41,7 +41,10 @@ def run_gpu(inp, *, inplace=False, flags=0, variant=0, fixed=None, workspace=Non
                             cu_seqlens=None if fixed else d["cu_seqlens"], num_seqs=N,
                             max_seqlen=max(inp.seqlens) if inp.seqlens else 0,
                             ckpt_offsets=d["ckpt_offsets"], ht=ht, workspace=workspace,
-                            variant=variant, flags=flags)
+                            variant=variant, flags=flags,
+                            frontend=None if frontend is None else dict(
+                                frontend, A_log=frontend["A_log"].cuda(),
+                                dt_bias=frontend["dt_bias"].cuda()))
     torch.cuda.synchronize()
     ws = workspace
     return {"o": out.float().cpu(), "ht": None if ht is None else ht.cpu(),
@@ -56,8 +59,26 @@ def rel_fro(a, b):
     return num / den
 
 
-def compare(inp, res, seqs=None, heads=None, threads=0):
-    """Oracle on the selected (sequence, head) pairs vs the GPU result; returns metrics."""
+def frontend_reference_inputs(inp, fe):
+    """The recurrence inputs the FP64 front-end oracle forms from raw projections
+    (fe: dict(flags, lower_bound, l2_eps, A_log, dt_bias) with CPU tensors), as a
+    KDAInputs of float64 tensors for oracle.prefill."""
+    import copy
+    q, k, g, beta = oracle.frontend_f64(inp.q.double().numpy(), inp.k.double().numpy(),
+                                        inp.g.double().numpy(), inp.beta.double().numpy(),
+                                        fe["A_log"].double().numpy(), fe["dt_bias"].double().numpy(),
+                                        fe["lower_bound"], fe["l2_eps"], fe["flags"])
+    ref = copy.copy(inp)
+    ref.q, ref.k, ref.g, ref.beta = (torch.from_numpy(np.ascontiguousarray(x))
+                                     for x in (q, k, g, beta))
+    return ref
+
+
+def compare(inp, res, seqs=None, heads=None, threads=0, frontend=None):
+    """Oracle on the selected (sequence, head) pairs vs the GPU result; returns metrics.
+    With ``frontend`` the inputs are raw projections and the FP64 front end runs first."""
+    if frontend is not None:
+        inp = frontend_reference_inputs(inp, frontend)
     ref = oracle.prefill(inp, threads=threads, heads=heads, seqs=seqs)
     seqs, heads, rows = ref["seqs"], ref["heads"], ref["rows"]
     m = {}

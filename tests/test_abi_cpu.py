@@ -179,3 +179,29 @@ def test_int64_cu_seqlens_validation():
     assert call(a) == capi.KDA_ERR_MISALIGNED        # INT64 entries need 8-byte alignment
     if not torch.cuda.is_available():
         assert call(dict(a, cu=BASE + 20 * MB)) == capi.KDA_ERR_UNSUPPORTED_DEVICE
+
+
+def test_prefill_frontend_validation():
+    torch = pytest.importorskip("torch")
+    G, N2, B = capi.KDA_FE_GATE, capi.KDA_FE_QK_L2NORM, capi.KDA_FE_BETA_LOGIT
+
+    def opts(flags, lb=-5.0, eps=1e-6, A=BASE + 30 * MB, dt=BASE + 31 * MB):
+        o = capi.kda_options_t()
+        o._fe = capi.make_frontend(flags, lb, eps, A, dt)
+        o.frontend = ctypes.pointer(o._fe)
+        return o
+
+    assert call(fake_args(opts=opts(1 << 6))) == capi.KDA_ERR_BAD_OPTION
+    assert call(fake_args(opts=opts(G, lb=0.0))) == capi.KDA_ERR_BAD_OPTION
+    assert call(fake_args(opts=opts(G, lb=float("nan")))) == capi.KDA_ERR_BAD_OPTION
+    assert call(fake_args(opts=opts(N2, eps=-1.0))) == capi.KDA_ERR_BAD_OPTION
+    assert call(fake_args(opts=opts(G, A=None))) == capi.KDA_ERR_NULL_ARG
+    assert call(fake_args(opts=opts(G, dt=BASE + 31 * MB + 8))) == capi.KDA_ERR_MISALIGNED
+    # the gate parameters are inputs: an output on top of them is refused
+    assert call(fake_args(opts=opts(G, dt=BASE + 8 * MB))) == capi.KDA_ERR_OUT_ALIAS
+    # with the gate switch g is BF16: a buffer right after its half size does not overlap it
+    a = fake_args(opts=opts(G | N2 | B))
+    half_g_end = a["g"] + 128 * 2 * 128 * 2
+    if not torch.cuda.is_available():
+        assert call(dict(a, out=half_g_end)) == capi.KDA_ERR_UNSUPPORTED_DEVICE
+        assert call(a) == capi.KDA_ERR_UNSUPPORTED_DEVICE

@@ -1,0 +1,56 @@
+"""Prefill from raw projections: the input front end (q/k L2 norm, gate from A_log and
+dt_bias under a lower bound, beta from its logit) inside every variant's kernels vs the
+FP64 front-end oracle followed by the FP64 recurrence oracle (needs a B200)."""
+import pytest
+import torch
+
+from kda_chunked_recurrent_b200.inputs import make_frontend_inputs
+from tests.gpu_helpers import assert_parity, compare, run_gpu
+
+pytestmark = pytest.mark.gpu
+
+SPLIT, FUSED, HYBRID, TOKEN = 1, 2, 3, 4
+
+
+def fe_dict(A_log, dt_bias, flags=7, lower_bound=-5.0):
+    return {"flags": flags, "lower_bound": lower_bound, "l2_eps": 1e-6, "A_log": A_log,
+            "dt_bias": dt_bias}
+
+
+@pytest.mark.parametrize("variant", [SPLIT, FUSED, HYBRID, TOKEN])
+def test_frontend_all_switches_every_variant(variant):
+    lens = [300, 0, 129, 64, 1, 77] if variant != TOKEN else [13, 0, 16, 1, 9]
+    inp, A_log, dt = make_frontend_inputs(lens, 3, seed=800 + variant, with_h0=True,
+                                          with_ckpt=True)
+    fe = fe_dict(A_log, dt)
+    assert_parity(compare(inp, run_gpu(inp, variant=variant, frontend=fe), frontend=fe))
+
+
+@pytest.mark.parametrize("flags", [1, 2, 4])
+def test_frontend_single_switches_split(flags):
+    inp, A_log, dt = make_frontend_inputs([200, 70], 2, seed=810 + flags, with_h0=True)
+    if not flags & 2:
+        inp.g = -5.0 * torch.sigmoid(inp.g.float())          # an FP32 log-decay in [-5, 0]
+    if not flags & 4:
+        inp.beta = torch.sigmoid(inp.beta.float()).to(torch.bfloat16)
+    if not flags & 1:
+        unit = lambda x: (x.float() / x.float().norm(dim=-1, keepdim=True)).to(torch.bfloat16)
+        inp.q, inp.k = unit(inp.q), unit(inp.k)
+    fe = fe_dict(A_log, dt, flags=flags, lower_bound=-3.0)
+    assert_parity(compare(inp, run_gpu(inp, variant=SPLIT, frontend=fe), frontend=fe))
+
+
+def test_frontend_hybrid_equals_split_bitwise():
+    inp, A_log, dt = make_frontend_inputs([4100, 64, 2000], 3, seed=820, with_h0=True)
+    fe = fe_dict(A_log, dt)
+    a = run_gpu(inp, variant=HYBRID, frontend=fe)
+    b = run_gpu(inp, variant=SPLIT, frontend=fe)
+    assert torch.equal(a["o"], b["o"]) and torch.equal(a["ht"], b["ht"])
+    assert_parity(compare(inp, a, frontend=fe))
+
+
+def test_frontend_full_length_sampled():
+    inp, A_log, dt = make_frontend_inputs([8192], 12, seed=830, fixed_layout=True)
+    fe = fe_dict(A_log, dt)
+    res = run_gpu(inp, frontend=fe)   # the table's choice (fused for 12 chains)
+    assert_parity(compare(inp, res, seqs=[0], heads=[0, 6, 11], frontend=fe))
