@@ -275,6 +275,11 @@ def token_kernel_name(capi, N, H):
     return "kda_token_wide_kernel" if "(wide" in d else "kda_token_narrow_kernel"
 
 
+def variant_hint_token(capi, shape, variant):
+    """Whether kda_prefill runs the token variant for this shape and variant option."""
+    return capi.kda_prefill_describe(shape, False, {"variant": variant}).startswith("variant=token")
+
+
 DECODE_METRIC = "KDA decode Mtokens·heads/s at 1 B200 (state pool, one launch per step)"
 
 
@@ -501,7 +506,13 @@ def main():
     opts = {"variant": args.variant}
     if args.frontend:
         A_log, dt_bias = A_log.to(dev), dt_bias.to(dev)
-        opts["frontend"] = capi.make_frontend(7, -5.0, 1e-6, A_log.data_ptr(), dt_bias.data_ptr())
+        # beta from logits only in the token variant; the chunked variants take BF16 beta
+        fe_flags = 7 if variant_hint_token(capi, shape, args.variant) else 3
+        if fe_flags == 3:
+            beta = torch.sigmoid(beta.float()).to(torch.bfloat16)
+            inp.beta = beta.cpu()
+        opts["frontend"] = capi.make_frontend(fe_flags, -5.0, 1e-6, A_log.data_ptr(),
+                                              dt_bias.data_ptr())
     ws = K.Workspace(capi.kda_prefill_workspace_size(shape, cko is not None, opts), dev)
     desc = capi.kda_prefill_describe(shape, cko is not None, opts)
     variant = desc.split()[0].split("=")[1] if desc.startswith("variant=") else "split"

@@ -154,8 +154,11 @@ typedef struct {
      after the last kernel of the call.  NULL entries are skipped.  The events
      let a caller time each kernel on the launching stream. */
   void* events[3];
-  /* NULL, or the input front end (kda_frontend_t above): q, k, g and beta then hold
-     raw projections.  All variants support it. */
+  /* NULL, or the input front end (kda_frontend_t above): q, k, g (and beta) then hold
+     raw projections.  Every variant takes KDA_FE_QK_L2NORM and KDA_FE_GATE;
+     KDA_FE_BETA_LOGIT only the token variant (the chunked variants keep
+     T diag(beta) as a BF16 tensor-core operand whose diagonal is beta itself, exact
+     only for a BF16 beta), else KDA_ERR_BAD_OPTION. */
   const kda_frontend_t* frontend;
   int32_t reserved[2];
 } kda_options_t;

@@ -462,6 +462,10 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
   const Resolved r = resolve(shape, fixed, ckpt, options);
   const size_t need = kda_prefill_workspace_size(shape, ckpt ? 1 : 0, options);
   if (workspace_bytes < need || workspace_bytes < r.lay.total) return KDA_ERR_WORKSPACE_TOO_SMALL;
+  // beta from logits only in the token variant: the chunked variants hold T diag(beta)
+  // as a BF16 tensor-core operand whose diagonal is beta itself, exact only for BF16 beta
+  if (fe && (fe->flags & KDA_FE_BETA_LOGIT) && r.variant != KDA_VARIANT_TOKEN)
+    return KDA_ERR_BAD_OPTION;
   // the fused launch needs an SM per chain plus SMs for its prepare CTAs
   if ((r.variant == KDA_VARIANT_FUSED || r.variant == KDA_VARIANT_HYBRID) && !fused_eligible(shape))
     return KDA_ERR_BAD_OPTION;

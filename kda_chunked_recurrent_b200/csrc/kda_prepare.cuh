@@ -320,9 +320,10 @@ __device__ __forceinline__ void publish_record(const KdaParams& p, int64_t rec) 
 // nitems; kFused selects the chunk-major item order, the named barriers and the
 // ready flags.
 // kFE: the input front end is compiled in (switches in p.fe_flags): the gate is formed
-// from the raw BF16 gate tile in the scan, the inverse L2 norms of the k and q rows are
-// folded into the FP32 factors that already multiply them (so every operand keeps its
-// single rounding), and beta is squashed from its logit when parked.
+// from the raw BF16 gate tile in the scan, and the inverse L2 norms of the k and q rows
+// are folded into the FP32 factors that already multiply them (so every operand keeps
+// its single rounding).  Beta from a logit is not offered here: T diag(beta) is a BF16
+// operand whose diagonal is beta itself, exact only for a BF16 beta.
 template <bool kFused, bool kFE = false>
 __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps& maps,
                                              uint8_t* smem_raw, int grp, int64_t first,
@@ -343,7 +344,6 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
   float* s_norm = reinterpret_cast<float*>(sm + kAuxNorm);   // front end: 1/|k_r|, then 1/|q_r|
   const bool fe_gate = kFE && (p.fe_flags & 2u) != 0;
   const bool fe_norm = kFE && (p.fe_flags & 1u) != 0;
-  const bool fe_beta = kFE && (p.fe_flags & 4u) != 0;
   const uint32_t raw_g_tx = fe_gate ? 16384u : kRawGTx;   // raw gate tile is BF16
 
   const int tid = threadIdx.x - grp * kThreads;
@@ -621,10 +621,7 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
         reinterpret_cast<float2*>(p.ws + p.lay.gc + rec * kTileGC)[cp] =
             make_float2(ex2(E.x), ex2(E.y));
     }
-    if (tid < kC) {
-      const float b = bf16_to_f32(beta_raw);
-      s_beta[tid] = fe_beta ? 1.f / (1.f + ex2(-b * kLog2e)) : b;
-    }
+    if (tid < kC) s_beta[tid] = bf16_to_f32(beta_raw);
 
     // ---- UMMA 1: D[0:128, 0:160] = [K+; Q+] . R^T   (bf16 -> f32)
     fence_proxy_async_smem();

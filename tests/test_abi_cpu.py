@@ -199,9 +199,14 @@ def test_prefill_frontend_validation():
     assert call(fake_args(opts=opts(G, dt=BASE + 31 * MB + 8))) == capi.KDA_ERR_MISALIGNED
     # the gate parameters are inputs: an output on top of them is refused
     assert call(fake_args(opts=opts(G, dt=BASE + 8 * MB))) == capi.KDA_ERR_OUT_ALIAS
+    # beta from logits: only the token variant (the chunked ones hold T diag(beta) in BF16)
+    assert call(fake_args(opts=opts(B))) == capi.KDA_ERR_BAD_OPTION       # AUTO -> chunked
+    tok = opts(G | N2 | B)
+    tok.variant = capi.KDA_VARIANT_TOKEN
     # with the gate switch g is BF16: a buffer right after its half size does not overlap it
-    a = fake_args(opts=opts(G | N2 | B))
+    a = fake_args(opts=opts(G | N2))
     half_g_end = a["g"] + 128 * 2 * 128 * 2
     if not torch.cuda.is_available():
         assert call(dict(a, out=half_g_end)) == capi.KDA_ERR_UNSUPPORTED_DEVICE
         assert call(a) == capi.KDA_ERR_UNSUPPORTED_DEVICE
+        assert call(fake_args(opts=tok)) == capi.KDA_ERR_UNSUPPORTED_DEVICE

@@ -1,6 +1,7 @@
 """Prefill from raw projections: the input front end (q/k L2 norm, gate from A_log and
-dt_bias under a lower bound, beta from its logit) inside every variant's kernels vs the
-FP64 front-end oracle followed by the FP64 recurrence oracle (needs a B200)."""
+dt_bias under a lower bound; beta from its logit in the token variant) inside every
+variant's kernels vs the FP64 front-end oracle followed by the FP64 recurrence oracle
+(needs a B200)."""
 import pytest
 import torch
 
@@ -17,16 +18,37 @@ def fe_dict(A_log, dt_bias, flags=7, lower_bound=-5.0):
             "dt_bias": dt_bias}
 
 
-@pytest.mark.parametrize("variant", [SPLIT, FUSED, HYBRID, TOKEN])
-def test_frontend_all_switches_every_variant(variant):
-    lens = [300, 0, 129, 64, 1, 77] if variant != TOKEN else [13, 0, 16, 1, 9]
-    inp, A_log, dt = make_frontend_inputs(lens, 3, seed=800 + variant, with_h0=True,
-                                          with_ckpt=True)
-    fe = fe_dict(A_log, dt)
+def chunked_inputs(lens, H, seed, **kw):
+    """Raw q, k and gate; beta given as a BF16 value (the chunked variants' contract)."""
+    inp, A_log, dt = make_frontend_inputs(lens, H, seed, **kw)
+    inp.beta = torch.sigmoid(inp.beta.float()).to(torch.bfloat16)
+    return inp, A_log, dt
+
+
+@pytest.mark.parametrize("variant", [SPLIT, FUSED, HYBRID])
+def test_frontend_norm_and_gate_chunked_variants(variant):
+    inp, A_log, dt = chunked_inputs([300, 0, 129, 64, 1, 77], 3, seed=800 + variant,
+                                    with_h0=True, with_ckpt=True)
+    fe = fe_dict(A_log, dt, flags=3)
     assert_parity(compare(inp, run_gpu(inp, variant=variant, frontend=fe), frontend=fe))
 
 
-@pytest.mark.parametrize("flags", [1, 2, 4])
+def test_frontend_all_switches_token_variant():
+    inp, A_log, dt = make_frontend_inputs([13, 0, 16, 1, 9], 3, seed=804, with_h0=True,
+                                          with_ckpt=True)
+    fe = fe_dict(A_log, dt)
+    assert_parity(compare(inp, run_gpu(inp, variant=TOKEN, frontend=fe), frontend=fe))
+
+
+def test_frontend_beta_logit_refused_by_chunked_variants():
+    import kda_chunked_recurrent_b200 as K
+    inp, A_log, dt = make_frontend_inputs([100], 2, seed=805, fixed_layout=True)
+    with pytest.raises(K.KDAError) as e:
+        run_gpu(inp, variant=SPLIT, frontend=fe_dict(A_log, dt))
+    assert e.value.code == K.capi.KDA_ERR_BAD_OPTION
+
+
+@pytest.mark.parametrize("flags", [1, 2])
 def test_frontend_single_switches_split(flags):
     inp, A_log, dt = make_frontend_inputs([200, 70], 2, seed=810 + flags, with_h0=True)
     if not flags & 2:
@@ -41,8 +63,8 @@ def test_frontend_single_switches_split(flags):
 
 
 def test_frontend_hybrid_equals_split_bitwise():
-    inp, A_log, dt = make_frontend_inputs([4100, 64, 2000], 3, seed=820, with_h0=True)
-    fe = fe_dict(A_log, dt)
+    inp, A_log, dt = chunked_inputs([4100, 64, 2000], 3, seed=820, with_h0=True)
+    fe = fe_dict(A_log, dt, flags=3)
     a = run_gpu(inp, variant=HYBRID, frontend=fe)
     b = run_gpu(inp, variant=SPLIT, frontend=fe)
     assert torch.equal(a["o"], b["o"]) and torch.equal(a["ht"], b["ht"])
@@ -50,7 +72,7 @@ def test_frontend_hybrid_equals_split_bitwise():
 
 
 def test_frontend_full_length_sampled():
-    inp, A_log, dt = make_frontend_inputs([8192], 12, seed=830, fixed_layout=True)
-    fe = fe_dict(A_log, dt)
+    inp, A_log, dt = chunked_inputs([8192], 12, seed=830, fixed_layout=True)
+    fe = fe_dict(A_log, dt, flags=3)
     res = run_gpu(inp, frontend=fe)   # the table's choice (fused for 12 chains)
     assert_parity(compare(inp, res, seqs=[0], heads=[0, 6, 11], frontend=fe))
