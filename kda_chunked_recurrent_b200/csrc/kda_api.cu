@@ -238,10 +238,13 @@ int choose_variant(const kda_shape_t* s, const kda_options_t* o) {
 // record (measured: B6 T8192 H12 with a 47-chunk tail), so the free SMs (2
 // groups each) keep up with jmax * f * 41 / R rows of R records, f = free SM
 // share; 0.9 of that keeps the producer ahead.
-int64_t hybrid_tail_chunks(int64_t jmax, int64_t chains) {
+// With the input front end the prepare side is slower (measured 0.585 vs 0.369 ms for
+// the prepare launch at B8 T8192 H12), so its tail is shorter by that ratio.
+int64_t hybrid_tail_chunks(int64_t jmax, int64_t chains, bool frontend = false) {
   const double sms = static_cast<double>(sm_count());
   const double f = (sms - static_cast<double>(chains)) / sms;
-  int64_t tail = static_cast<int64_t>(0.9 * static_cast<double>(jmax) * f * 41.0 /
+  const double rate = frontend ? 41.0 * 0.369 / 0.585 : 41.0;
+  int64_t tail = static_cast<int64_t>(0.9 * static_cast<double>(jmax) * f * rate /
                                       static_cast<double>(chains));
   return std::max<int64_t>(1, std::min<int64_t>(tail, jmax - 1));
 }
@@ -385,7 +388,8 @@ kda_status_t kda_prefill_describe(const kda_shape_t* shape, int has_ckpt,
              wide ? 1 : 4, wide ? 128 : 32, r.lay.total);
   } else if (r.variant == KDA_VARIANT_HYBRID) {
     const int64_t jmax = max_chunks_per_seq(shape, false, has_ckpt != 0);
-    const int64_t tail = hybrid_tail_chunks(jmax, chains);
+    const bool fe = options && options->frontend && options->frontend->flags;
+    const int64_t tail = hybrid_tail_chunks(jmax, chains, fe);
     snprintf(buf, n,
              "variant=hybrid chunk=%d prepare_chunks=%lld/%lld (split prepare launch) then "
              "grid=%dx%d (recurrence CTAs %lld, prepare CTAs %lld, cooperative) workspace_bytes=%zu",
@@ -612,7 +616,7 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
     int64_t j0 = 0;
     if (r.variant == KDA_VARIANT_HYBRID && T > 0) {
       // the prepare launch makes chunks [0, j0) of every sequence first
-      j0 = jmax - hybrid_tail_chunks(jmax, N * H);
+      j0 = jmax - hybrid_tail_chunks(jmax, N * H, p.fe_flags != 0);
       p.split_jmax = static_cast<int32_t>(j0);
       const int64_t items = r.lay.slots * H;
       const int64_t pgrid = std::min<int64_t>(items, 2 * static_cast<int64_t>(sm_count()));

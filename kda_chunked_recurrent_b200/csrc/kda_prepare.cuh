@@ -471,8 +471,10 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
           const uint32_t a2 = in ? reinterpret_cast<const uint32_t*>(sm + kGraw)[(blk * 16 + i) * 64 + cp] : 0u;
           const float2 a = bf2_to_f2(a2);
           const float x0 = fe_rate * (a.x + fe_dtb.x), x1 = fe_rate * (a.y + fe_dtb.y);
-          G[i] = in ? make_float2(p.lower_bound / (1.f + ex2(-x0 * kLog2e)),
-                                  p.lower_bound / (1.f + ex2(-x1 * kLog2e)))
+          // (fast reciprocal: 1 + 2^y is at least 1, and a huge denominator gives 0, the
+          // limit of the logistic)
+          G[i] = in ? make_float2(__fdividef(p.lower_bound, 1.f + ex2(-x0 * kLog2e)),
+                                  __fdividef(p.lower_bound, 1.f + ex2(-x1 * kLog2e)))
                     : make_float2(0.f, 0.f);
         } else {
           G[i] = in ? gs[i * 64] : make_float2(0.f, 0.f);
@@ -484,22 +486,29 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
     if constexpr (kFE) {
       if (fe_norm) {   // (warp-uniform; on a failed wait the values are never used)
         // inverse L2 norms of the chunk's k and q rows: warp w takes rows 8 w .. 8 w + 7,
-        // lane l channels 4 l .. 4 l + 3 (the raw tiles are intact until the barrier below)
-        const uint2* kr = reinterpret_cast<const uint2*>(sm + kKraw);
-        const uint2* qr = reinterpret_cast<const uint2*>(sm + kQraw);
-#pragma unroll 2
-        for (int rr = 0; rr < 8; ++rr) {
-          const int row = warp * 8 + rr;
-          const float2 k01 = bf2_to_f2(kr[row * 32 + lane].x), k23 = bf2_to_f2(kr[row * 32 + lane].y);
-          const float2 q01 = bf2_to_f2(qr[row * 32 + lane].x), q23 = bf2_to_f2(qr[row * 32 + lane].y);
-          float sk = fmaf(k01.x, k01.x, fmaf(k01.y, k01.y, fmaf(k23.x, k23.x, k23.y * k23.y)));
-          float sq = fmaf(q01.x, q01.x, fmaf(q01.y, q01.y, fmaf(q23.x, q23.x, q23.y * q23.y)));
+        // two rows at a time, half-warp h = lane / 16 one row, lane channels 8 (lane % 16)
+        // .. + 7 (the raw tiles are intact until the barrier below)
+        const uint4* kr = reinterpret_cast<const uint4*>(sm + kKraw);
+        const uint4* qr = reinterpret_cast<const uint4*>(sm + kQraw);
+        const int hl = lane & 15;
 #pragma unroll
-          for (int o = 16; o > 0; o >>= 1) {
+        for (int rr = 0; rr < 4; ++rr) {
+          const int row = warp * 8 + rr * 2 + (lane >> 4);
+          const uint4 kv = kr[row * 16 + hl], qv = qr[row * 16 + hl];
+          float sk = 0.f, sq = 0.f;
+          const uint32_t kx[4] = {kv.x, kv.y, kv.z, kv.w}, qx[4] = {qv.x, qv.y, qv.z, qv.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float2 a = bf2_to_f2(kx[j]), b = bf2_to_f2(qx[j]);
+            sk = fmaf(a.x, a.x, fmaf(a.y, a.y, sk));
+            sq = fmaf(b.x, b.x, fmaf(b.y, b.y, sq));
+          }
+#pragma unroll
+          for (int o = 8; o > 0; o >>= 1) {
             sk += __shfl_xor_sync(0xffffffffu, sk, o);
             sq += __shfl_xor_sync(0xffffffffu, sq, o);
           }
-          if (lane == 0) {
+          if (hl == 0) {
             s_norm[row] = rsqrtf(sk + p.l2_eps);
             s_norm[64 + row] = rsqrtf(sq + p.l2_eps);
           }
