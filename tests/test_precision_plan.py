@@ -1,0 +1,70 @@
+"""The operand precisions of the chunked path, checked with the rounding model against
+the FP64 oracle (CPU): each kept choice meets the 1e-3 state gate, each rejected one
+misses it, so the reasons the kernels are built this way stay reproducible."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from kda_chunked_recurrent_b200.inputs import make_frontend_inputs, make_inputs
+from tests.rounding_model import final_states
+
+S_TOL = 1e-3
+
+
+def worst_rel(a, b):
+    a = a.reshape(a.shape[0], a.shape[1], -1)
+    b = b.reshape(b.shape[0], b.shape[1], -1)
+    return float((np.linalg.norm(a - b, axis=-1) /
+                  np.maximum(np.linalg.norm(b, axis=-1), 1e-30)).max())
+
+
+@pytest.fixture(scope="module")
+def plain_case():
+    inp = make_inputs([300, 200], 2, seed=1003, with_h0=True)
+    arr = [x.double().numpy() for x in (inp.q, inp.k, inp.v, inp.g, inp.beta)]
+    cu = inp.cu_seqlens.tolist()
+    h0 = inp.h0.double().numpy()
+    _, ht, _ = oracle.prefill_f64(*arr, inp.scale, cu, h0)
+    return arr, inp.scale, cu, h0, ht
+
+
+@pytest.fixture(scope="module")
+def squashed_beta_case():
+    """Unit q/k rows, an FP32 log-decay and beta = sigmoid(logit) kept in FP32, as the
+    input front end forms it."""
+    inp, _, _ = make_frontend_inputs([300, 129, 77], 3, seed=801, with_h0=True)
+    unit = lambda x: (x.float() / x.float().norm(dim=-1, keepdim=True)).to(torch.bfloat16)
+    q, k = unit(inp.q).double().numpy(), unit(inp.k).double().numpy()
+    g = (-5.0 * torch.sigmoid(inp.g.float())).double().numpy()
+    beta = torch.sigmoid(inp.beta.double()).float().double().numpy()
+    v = inp.v.double().numpy()
+    cu = inp.cu_seqlens.tolist()
+    h0 = inp.h0.double().numpy()
+    _, ht, _ = oracle.prefill_f64(q, k, v, g, beta, inp.scale, cu, h0)
+    return (q, k, v, g, beta), inp.scale, cu, h0, ht
+
+
+def test_kernel_plan_meets_the_gate(plain_case):
+    arr, scale, cu, h0, ht = plain_case
+    assert worst_rel(final_states(*arr, scale, cu, h0), ht) < 0.5 * S_TOL
+
+
+@pytest.mark.parametrize("choice", [dict(ud="bf16"), dict(ud="bf16", kd="bf16", aqk="bf16")],
+                         ids=["Ud_bf16", "all_bf16"])
+def test_bf16_state_operands_miss_the_gate(plain_case, choice):
+    arr, scale, cu, h0, ht = plain_case
+    assert worst_rel(final_states(*arr, scale, cu, h0, **choice), ht) > S_TOL
+
+
+def test_fp32_beta_through_a_bf16_tb_misses_the_gate(squashed_beta_case):
+    # why the chunked variants refuse beta from logits: T diag(beta) is a BF16 operand
+    arr, scale, cu, h0, ht = squashed_beta_case
+    assert worst_rel(final_states(*arr, scale, cu, h0, tb="bf16"), ht) > S_TOL
+
+
+@pytest.mark.parametrize("choice", [dict(tb="f16"), dict(tb="bf16", beta_split=True)],
+                         ids=["tb_f16", "split_beta"])
+def test_fixes_for_fp32_beta_meet_the_gate(squashed_beta_case, choice):
+    arr, scale, cu, h0, ht = squashed_beta_case
+    assert worst_rel(final_states(*arr, scale, cu, h0, **choice), ht) < S_TOL
