@@ -68,3 +68,12 @@ def test_fp32_beta_through_a_bf16_tb_misses_the_gate(squashed_beta_case):
 def test_fixes_for_fp32_beta_meet_the_gate(squashed_beta_case, choice):
     arr, scale, cu, h0, ht = squashed_beta_case
     assert worst_rel(final_states(*arr, scale, cu, h0, **choice), ht) < S_TOL
+
+
+def test_a_128_token_chunk_keeps_the_plan_within_the_gate(plain_case, monkeypatch):
+    # the same operand plan over 128-token chunks (the C = 128 row of the variant table
+    # to come): the 16-token sub-block factors stay bounded and the error does not grow
+    import tests.rounding_model as RM
+    arr, scale, cu, h0, ht = plain_case
+    monkeypatch.setattr(RM, "C", 128)
+    assert worst_rel(RM.final_states(*arr, scale, cu, h0), ht) < 0.5 * S_TOL
