@@ -40,6 +40,7 @@ STATE_BYTES = 128 * 128 * 4
 # per-kernel bytes per token and head, as designed (split variant)
 PREP_BYTES_PER_TOKHEAD = 768 + 512 + 2 + 1160     # reads q,k,v,g,beta; writes W,QG,U,Kd,Aqk,Gamma
 REC_BYTES_PER_TOKHEAD = 1160 + 256                 # reads the prepared tiles; writes o
+OUT_BYTES_PER_TOKHEAD = 256                        # the o row every prefill writes
 # tensor-core FLOPs per token and head at a fixed C = 64 count: 6 K V + 10 C d
 FLOPS_PER_TOKHEAD_C64 = 6 * 128 * 128 + 10 * 64 * 128
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -275,11 +276,6 @@ def token_kernel_name(capi, N, H):
     return "kda_token_wide_kernel" if "(wide" in d else "kda_token_narrow_kernel"
 
 
-def variant_hint_token(capi, shape, variant):
-    """Whether kda_prefill runs the token variant for this shape and variant option."""
-    return capi.kda_prefill_describe(shape, False, {"variant": variant}).startswith("variant=token")
-
-
 DECODE_METRIC = "KDA decode Mtokens·heads/s at 1 B200 (state pool, one launch per step)"
 
 
@@ -506,11 +502,8 @@ def main():
     opts = {"variant": args.variant}
     if args.frontend:
         A_log, dt_bias = A_log.to(dev), dt_bias.to(dev)
-        # beta from logits only in the token variant; the chunked variants take BF16 beta
-        fe_flags = 7 if variant_hint_token(capi, shape, args.variant) else 3
-        if fe_flags == 3:
-            beta = torch.sigmoid(beta.float()).to(torch.bfloat16)
-            inp.beta = beta.cpu()
+        # every variant forms q/k norms, the gate and beta from the raw projections
+        fe_flags = 7
         opts["frontend"] = capi.make_frontend(fe_flags, -5.0, 1e-6, A_log.data_ptr(),
                                               dt_bias.data_ptr())
     ws = K.Workspace(capi.kda_prefill_workspace_size(shape, cko is not None, opts), dev)
@@ -596,38 +589,40 @@ def main():
     # from raw projections the gate is read as BF16: 256 B less per token and head
     gate_saving = 256 if args.frontend else 0
     prep_b, path_b = PREP_BYTES_PER_TOKHEAD - gate_saving, PATH_BYTES_PER_TOKHEAD - gate_saving
+    in_b = path_b - OUT_BYTES_PER_TOKHEAD     # the inputs every prefill must read
     state_io = N * H * STATE_BYTES * ((1 if h0 is not None else 0) + 1 + (1 if ck is not None else 0))
+    # Per launch: (ms, algorithmic bytes, designed bytes, sources).  The algorithmic
+    # bytes of a launch are its share of the path's bytes: the inputs of the token-heads
+    # whose chunk records it makes, the o rows it writes and the state I/O it does; over
+    # the launches of one step they add up to path_b per token-head plus the state I/O.
+    # The designed bytes add the chunk records each launch writes or reads.
+    F = hybrid_frac
+    fused_src = ["kda_fused.cu", "kda_prepare.cuh", "kda_recurrence.cuh", "kda_common.cuh",
+                 "sm100_primitives.cuh"]
+    prep_src = ["kda_prepare.cu", "kda_prepare.cuh", "kda_common.cuh", "sm100_primitives.cuh"]
     if variant == "hybrid":
         kernels = {
-            "kda_prepare_kernel": (prep_ms, hybrid_frac * prep_b * units,
-                                   ["kda_prepare.cu", "kda_prepare.cuh", "kda_common.cuh",
-                                    "sm100_primitives.cuh"]),
-            "kda_fused_kernel": (rec_ms,
-                                 ((1 - hybrid_frac) * prep_b + REC_BYTES_PER_TOKHEAD)
-                                 * units + state_io,
-                                 ["kda_fused.cu", "kda_prepare.cuh", "kda_recurrence.cuh",
-                                  "kda_common.cuh", "sm100_primitives.cuh"]),
+            "kda_prepare_kernel": (prep_ms, F * in_b * units, F * prep_b * units, prep_src),
+            "kda_fused_kernel": (rec_ms, ((1 - F) * in_b + OUT_BYTES_PER_TOKHEAD) * units + state_io,
+                                 ((1 - F) * prep_b + REC_BYTES_PER_TOKHEAD) * units + state_io,
+                                 fused_src),
         }
     elif variant == "token":
         kernels = {
-            token_kernel_name(capi, N, H): (prep_ms + rec_ms,
-                                            path_b * units + state_io,
-                                            TOKEN_SOURCES),
+            token_kernel_name(capi, N, H): (prep_ms + rec_ms, path_b * units + state_io,
+                                            path_b * units + state_io, TOKEN_SOURCES),
         }
     elif variant == "fused":
         # one launch moves both halves' bytes (the records still go through HBM/L2)
         kernels = {
-            "kda_fused_kernel": (prep_ms + rec_ms,
-                                 (prep_b + REC_BYTES_PER_TOKHEAD) * units + state_io,
-                                 ["kda_fused.cu", "kda_prepare.cuh", "kda_recurrence.cuh",
-                                  "kda_common.cuh", "sm100_primitives.cuh"]),
+            "kda_fused_kernel": (prep_ms + rec_ms, path_b * units + state_io,
+                                 (prep_b + REC_BYTES_PER_TOKHEAD) * units + state_io, fused_src),
         }
     else:
         kernels = {
-            "kda_prepare_kernel": (prep_ms, prep_b * units,
-                                   ["kda_prepare.cu", "kda_prepare.cuh", "kda_common.cuh",
-                                    "sm100_primitives.cuh"]),
-            "kda_recurrence_kernel": (rec_ms, REC_BYTES_PER_TOKHEAD * units + state_io,
+            "kda_prepare_kernel": (prep_ms, in_b * units, prep_b * units, prep_src),
+            "kda_recurrence_kernel": (rec_ms, OUT_BYTES_PER_TOKHEAD * units + state_io,
+                                      REC_BYTES_PER_TOKHEAD * units + state_io,
                                       ["kda_recurrence.cu", "kda_recurrence.cuh", "kda_common.cuh",
                                        "sm100_primitives.cuh"]),
         }
@@ -635,14 +630,17 @@ def main():
         kernels = {(n if n == "kda_recurrence_kernel" else n.replace("_kernel", "_fe_kernel")): v
                    for n, v in kernels.items()}
     dom = max(kernels, key=lambda n: kernels[n][0])
-    dms, dbytes, _ = kernels[dom]
+    dms, dbytes, dsgn, _ = kernels[dom]
     achieved = dbytes / (dms / 1e3) / 1e9
+    traffic = ncu_traffic(dom, variant, units)
     roof = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1),
             "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-            "traffic": ncu_traffic(dom, variant, units), "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
+            "traffic": traffic, "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
             if peak_src == "measured" else "fallback 6650 GB/s",
             "kernel_ms": round(dms, 4),
             "algorithmic_bytes": int(dbytes),
+            "designed_bytes": int(dsgn),
+            "traffic_ratio": None if traffic is None else round(traffic / dbytes, 3),
             "per_kernel_ms": {n: round(kernels[n][0], 4) for n in kernels}}
     path_bytes = path_b * units + state_io
     flops = FLOPS_PER_TOKHEAD_C64 * units

@@ -68,6 +68,9 @@ typedef enum {
   KDA_ERR_UNSUPPORTED_DEVICE = 8,  /* current device is not compute capability 10.0  */
   KDA_ERR_LAUNCH_FAILED = 9,       /* the CUDA runtime refused a launch              */
   KDA_ERR_BAD_OPTION = 10,         /* unknown variant / chunk / flag value           */
+  KDA_ERR_SCRATCH_UNAVAILABLE = 11,/* kda_prefill_noalloc: the built-in scratch area
+                                      could not be set up on this device (e.g. out of
+                                      memory when the library's device code loads)  */
   /* codes the kernels record in the workspace status word */
   KDA_ERR_BAD_CU_SEQLENS = 16,     /* cu_seqlens[0] != 0, decreasing, or last != T,
                                       or a length above max_seqlen (validate mode)   */
@@ -97,12 +100,18 @@ typedef enum {
                             the fused launch, whose prepare CTAs make the last chunks while
                             its recurrence CTAs already run.  Same SM condition as FUSED;
                             AUTO picks it above 56 chains of at least 64 chunks.          */
-  KDA_VARIANT_TOKEN = 4   /* the recurrence one token at a time with the state in
+  KDA_VARIANT_TOKEN = 4,  /* the recurrence one token at a time with the state in
                             registers: 4 CTAs of 32 value columns per (sequence, head)
                             below 128 units, one CTA of 128 columns per unit from 128 on;
                             no chunk records, workspace = header only.  AUTO picks it when
                             max_seqlen (else T_total) is at most 16, or at most 32 with
                             N*H <= 16.                                                   */
+  KDA_VARIANT_STREAM = 5  /* one cooperative launch of two CTAs per SM: one recurrence CTA
+                            per (sequence, head) (state with the key channel on the tensor-
+                            memory lanes, 256 columns) and prepare CTAs on every other slot,
+                            beside the recurrences on the same SMs; records reach the
+                            recurrence through L2 and are dropped from it once read.  Needs
+                            N*H + 16 <= 2 x SM count, else KDA_ERR_BAD_OPTION.           */
 } kda_variant_t;
 
 enum {
@@ -155,10 +164,9 @@ typedef struct {
      let a caller time each kernel on the launching stream. */
   void* events[3];
   /* NULL, or the input front end (kda_frontend_t above): q, k, g (and beta) then hold
-     raw projections.  Every variant takes KDA_FE_QK_L2NORM and KDA_FE_GATE;
-     KDA_FE_BETA_LOGIT only the token variant (the chunked variants keep
-     T diag(beta) as a BF16 tensor-core operand whose diagonal is beta itself, exact
-     only for a BF16 beta), else KDA_ERR_BAD_OPTION. */
+     raw projections.  Every variant takes all three switches (the chunked variants
+     keep T diag(beta) as an FP16 tensor-core operand, so a beta squashed in FP32
+     keeps 2^-11 relative precision on its diagonal). */
   const kda_frontend_t* frontend;
   int32_t reserved[2];
 } kda_options_t;
@@ -166,8 +174,16 @@ typedef struct {
 /*
  * Bytes of workspace kda_prefill needs for this shape and option set (NULL
  * options = defaults).  `has_ckpt` != 0 when checkpoint export is requested.
- * Returns 0 for an invalid shape.  The workspace must be 256-byte aligned and,
- * before its first use, initialised once with kda_workspace_init.
+ * Returns 0 for an invalid shape or option set.  The workspace must be 256-byte
+ * aligned and, before its first use, initialised once with kda_workspace_init.
+ *
+ * Source: the pages' prefill backends take their scratch from one caller-owned
+ * workspace so that a warmed call allocates nothing and can be captured in a CUDA
+ * graph (FlashInfer PR #4633 "Description": decomp's two launches share one scratch
+ * arena, and graph capture goes through a caller-owned workspace; FlashInfer PR
+ * #4262 "CUDA graph and tensor-map safety").  The size is a pure function of the
+ * host-side shape, so it can be queried before any device work.  The layout in it
+ * (per-chunk records, chunk table, status word) is this library's own.
  */
 size_t kda_prefill_workspace_size(const kda_shape_t* shape, int has_ckpt,
                                   const kda_options_t* options);
@@ -175,6 +191,9 @@ size_t kda_prefill_workspace_size(const kda_shape_t* shape, int has_ckpt,
 /*
  * Initialise a workspace (clears its status word).  Enqueued on `stream`.
  * Needed once per workspace allocation, before the first kda_prefill with it.
+ * Source: this library's design (the status word below); the pages' workspaces
+ * are warmed eagerly before capture (FlashInfer PR #4262 "CUDA graph and
+ * tensor-map safety"), and this is the equivalent one-time step here.
  */
 kda_status_t kda_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
 
@@ -184,7 +203,8 @@ kda_status_t kda_workspace_init(void* workspace, size_t workspace_bytes, void* s
  *   q, k      [T_total, H, 128] BF16, contiguous, 16-byte aligned.  Rows of all
  *             sequences packed back to back (fixed layout [B, T, H, 128] is the
  *             same memory).  k is expected to be L2-normalised per row: the
- *             FP16 tensor-core operands assume |S| and |v| well inside 65504.
+ *             FP16 tensor-core operands (the state read, v, W, U) assume |S| and
+ *             |v| well inside 65504.
  *   v         [T_total, H, 128] BF16, contiguous, 16-byte aligned.
  *   g         [T_total, H, 128] FP32 log-decay per key channel, contiguous,
  *             16-byte aligned; expected in [-5, 0] (outside it the chunked
@@ -224,17 +244,26 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
  * Read (and clear when `clear` != 0) the status word the kernels of earlier
  * kda_prefill calls recorded in `workspace`.  Synchronises `stream`.  The word
  * keeps the first device-side error since the last clear (KDA_OK if none).
+ * Source: this library's design, with no counterpart passage on the pages.  The
+ * pages never read device metadata on the host (lmdeploy PR #5050 "Motivation":
+ * offset values are the caller's responsibility, no device-to-host copy on the hot
+ * path), so errors found on the device (validate mode, a bounded wait that gave
+ * up) are recorded here and read only when the caller asks.
  */
 kda_status_t kda_prefill_status(void* workspace, void* stream, int32_t* device_status,
                                  int clear);
 
-/* Static description of a status code (never NULL). */
+/* Static description of a status code (never NULL).  Source: this library's
+   design (the codes above); no counterpart passage on the pages. */
 const char* kda_status_string(int status);
 
 /*
  * Write a one-line description of what kda_prefill would launch for this
  * shape (variant, chunk size, grids, workspace bytes) into buf (NUL-
  * terminated, truncated to n bytes).  Host only.
+ * Source: FlashInfer PR #4633 "Description" picks decomp or fused per call from a
+ * measured table keyed on the SM count and offers describe_variant_policy to report
+ * the policy a device gets; this call is that report for one shape.
  */
 kda_status_t kda_prefill_describe(const kda_shape_t* shape, int has_ckpt,
                                   const kda_options_t* options, char* buf, size_t n);
@@ -257,16 +286,24 @@ kda_status_t kda_prefill_describe(const kda_shape_t* shape, int has_ckpt,
  *   - Shapes whose kda_prefill_workspace_size exceeds KDA_NOALLOC_SCRATCH_BYTES
  *     are refused with KDA_ERR_WORKSPACE_TOO_SMALL before anything is enqueued
  *     (48 MiB covers, e.g., 12 heads x 2048 tokens, or 8 x 1024 tokens at H = 4).
- *   - The first call on a device looks up the area's device address
- *     (cudaGetSymbolAddress) with that device current; make that first call
+ *   - Every call looks up the area's device address (cudaGetSymbolAddress) with
+ *     the current device.  With lazy module loading (the CUDA default) the first
+ *     call on a device may load the library's device code and create the area
+ *     there; if that fails (out of memory) the call returns
+ *     KDA_ERR_SCRATCH_UNAVAILABLE and enqueues nothing.  Make that first call
  *     outside any stream capture.
  *   - All calls on a device share the one area: calls that may overlap on the
  *     GPU (different streams without ordering between them) race and must not
  *     be issued.  Calls ordered on one stream are fine; nothing in the area has
  *     to be cleared between calls.
  *   - The device status word lives in the built-in area and is not readable
- *     through this entry point; use kda_prefill with your own workspace when
- *     validate mode or status reporting is needed.
+ *     through this entry point, so KDA_FLAG_VALIDATE and
+ *     KDA_FLAG_TEST_FORCE_TIMEOUT are refused (KDA_ERR_BAD_OPTION), and a bounded
+ *     wait that gives up on the device cannot be seen here: use kda_prefill with
+ *     your own workspace when validate mode or status reporting is needed.
+ *   - Checks run in this order: options and shape (their kda_prefill codes), the
+ *     device (KDA_ERR_UNSUPPORTED_DEVICE), the area's size
+ *     (KDA_ERR_WORKSPACE_TOO_SMALL), then kda_prefill's own checks.
  */
 #define KDA_NOALLOC_SCRATCH_BYTES ((size_t)48 << 20)
 kda_status_t kda_prefill_noalloc(const void* q, const void* k, const void* v, const float* g,
@@ -344,7 +381,8 @@ kda_status_t kda_decode(const void* q, const void* k, const void* v, const float
                         void* out, float* step_states, int32_t* device_status, uint32_t flags,
                         const kda_frontend_t* frontend, void* stream);
 
-/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH.  Source: this library's
+   design; no counterpart passage on the pages. */
 int kda_version(void);
 
 #ifdef __cplusplus

@@ -19,7 +19,7 @@ _CAPI_NAMES = {"kda_prefill", "kda_prefill_describe", "kda_prefill_status",
                "kda_workspace_init", "make_shape", "kda_decode", "make_decode_shape"}
 KDA_OK = 0
 KDA_VARIANT_AUTO, KDA_VARIANT_SPLIT, KDA_VARIANT_FUSED = 0, 1, 2
-KDA_VARIANT_HYBRID, KDA_VARIANT_TOKEN = 3, 4
+KDA_VARIANT_HYBRID, KDA_VARIANT_TOKEN, KDA_VARIANT_STREAM = 3, 4, 5
 KDA_DECODE_KEEP_STATE, KDA_DECODE_NARROW, KDA_DECODE_WIDE = 1, 2, 4
 KDA_FE_QK_L2NORM, KDA_FE_GATE, KDA_FE_BETA_LOGIT = 1, 2, 4
 KDA_FLAG_VALIDATE, KDA_FLAG_TEST_FORCE_TIMEOUT, KDA_FLAG_CU_SEQLENS_I64 = 1, 2, 4

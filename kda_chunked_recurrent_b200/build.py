@@ -15,9 +15,9 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libkda_prefill.so")
 SOURCES = ["kda_api.cu", "kda_schedule.cu", "kda_prepare.cu", "kda_recurrence.cu",
-           "kda_fused.cu", "kda_token.cu", "kda_noalloc.cu"]
+           "kda_fused.cu", "kda_stream.cu", "kda_token.cu", "kda_noalloc.cu"]
 HEADERS = ["kda_common.cuh", "sm100_primitives.cuh", "kda_prepare.cuh", "kda_recurrence.cuh",
-           "kda_token.cuh"]
+           "kda_chain.cuh", "kda_token.cuh"]
 
 
 def nvcc_path() -> str:

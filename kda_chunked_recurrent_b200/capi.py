@@ -24,6 +24,7 @@ KDA_ERR_WORKSPACE_TOO_SMALL = 7
 KDA_ERR_UNSUPPORTED_DEVICE = 8
 KDA_ERR_LAUNCH_FAILED = 9
 KDA_ERR_BAD_OPTION = 10
+KDA_ERR_SCRATCH_UNAVAILABLE = 11
 KDA_ERR_BAD_CU_SEQLENS = 16
 KDA_ERR_BAD_CKPT_OFFSET = 17
 KDA_ERR_TIMEOUT = 18
@@ -34,6 +35,7 @@ KDA_VARIANT_SPLIT = 1
 KDA_VARIANT_FUSED = 2
 KDA_VARIANT_HYBRID = 3
 KDA_VARIANT_TOKEN = 4
+KDA_VARIANT_STREAM = 5
 KDA_DECODE_KEEP_STATE = 1
 KDA_FE_QK_L2NORM = 1
 KDA_FE_GATE = 2

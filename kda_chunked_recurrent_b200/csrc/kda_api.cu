@@ -29,7 +29,12 @@ __global__ void kda_fused_fe_kernel(const KdaParams p, const __grid_constant__ S
 __global__ void kda_recurrence_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps);
 __global__ void kda_fused_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps,
                                  int32_t rec_ctas, int64_t prep_items, int32_t prep_groups);
+__global__ void kda_stream_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps,
+                                  int32_t rec_ctas, int64_t prep_items);
+__global__ void kda_stream_fe_kernel(const KdaParams p, const __grid_constant__ SplitMaps maps,
+                                     int32_t rec_ctas, int64_t prep_items);
 namespace prep { extern const uint32_t kSmemAllocBytes; }
+namespace stream { extern const uint32_t kSmemAllocBytes; extern const int kThreadsPerCta; }
 namespace rec { extern const uint32_t kSmemAllocBytes; extern const int kThreadsPerCta; }
 namespace fused { extern const uint32_t kSmemAllocBytes; extern const int kThreadsPerCta; }
 __global__ void kda_token_narrow_kernel(const TokenParams p);
@@ -89,7 +94,7 @@ struct Resolved {
 
 kda_status_t check_options(const kda_options_t* o) {
   if (!o) return KDA_OK;
-  if (o->variant < KDA_VARIANT_AUTO || o->variant > KDA_VARIANT_TOKEN) return KDA_ERR_BAD_OPTION;
+  if (o->variant < KDA_VARIANT_AUTO || o->variant > KDA_VARIANT_STREAM) return KDA_ERR_BAD_OPTION;
   if (o->flags & ~(static_cast<uint32_t>(KDA_FLAG_VALIDATE | KDA_FLAG_TEST_FORCE_TIMEOUT |
                                          KDA_FLAG_CU_SEQLENS_I64)))
     return KDA_ERR_BAD_OPTION;
@@ -215,6 +220,14 @@ bool fused_eligible(const kda_shape_t* s) {
   return chains + kFusedMinPrepCtas <= sm_count();
 }
 
+// The stream launch holds two CTAs per SM: one recurrence CTA per chain and prepare
+// CTAs on every other slot, at least kFusedMinPrepCtas of them.
+constexpr int kStreamCtasPerSm = 2;
+bool stream_eligible(const kda_shape_t* s) {
+  const int64_t chains = static_cast<int64_t>(s->num_seqs) * s->num_heads;
+  return chains + kFusedMinPrepCtas <= kStreamCtasPerSm * static_cast<int64_t>(sm_count());
+}
+
 int64_t max_chunks_per_seq(const kda_shape_t* s, bool fixed, bool ckpt);
 
 int choose_variant(const kda_shape_t* s, const kda_options_t* o) {
@@ -227,6 +240,7 @@ int choose_variant(const kda_shape_t* s, const kda_options_t* o) {
       if ((rule.variant == KDA_VARIANT_FUSED || rule.variant == KDA_VARIANT_HYBRID) &&
           !fused_eligible(s))
         continue;
+      if (rule.variant == KDA_VARIANT_STREAM && !stream_eligible(s)) continue;
       return rule.variant;
     }
   return KDA_VARIANT_SPLIT;
@@ -263,7 +277,8 @@ Resolved resolve(const kda_shape_t* s, bool fixed, bool ckpt, const kda_options_
   // the token variant needs no per-record tiles; AUTO sizes for the largest variant
   // so that one workspace serves whatever the table picks
   const bool tiles = !(o && o->variant == KDA_VARIANT_TOKEN);
-  r.lay = make_layout(s->num_seqs, s->total_tokens, s->num_heads, fixed, tiles, ckpt);
+  r.lay = make_layout(s->num_seqs, s->total_tokens, s->num_heads, fixed, tiles, ckpt,
+                      r.variant == KDA_VARIANT_STREAM);
   return r;
 }
 
@@ -340,6 +355,7 @@ const char* kda_status_string(int s) {
     case KDA_ERR_UNSUPPORTED_DEVICE: return "current device is not compute capability 10.0";
     case KDA_ERR_LAUNCH_FAILED: return "kernel launch failed";
     case KDA_ERR_BAD_OPTION: return "unknown or unavailable option";
+    case KDA_ERR_SCRATCH_UNAVAILABLE: return "the built-in scratch area could not be set up";
     case KDA_ERR_BAD_CU_SEQLENS: return "cu_seqlens invalid (validate mode)";
     case KDA_ERR_BAD_CKPT_OFFSET: return "checkpoint offset outside its sequence (validate mode)";
     case KDA_ERR_TIMEOUT: return "a bounded on-device wait timed out";
@@ -395,6 +411,13 @@ kda_status_t kda_prefill_describe(const kda_shape_t* shape, int has_ckpt,
              "grid=%dx%d (recurrence CTAs %lld, prepare CTAs %lld, cooperative) workspace_bytes=%zu",
              kC, static_cast<long long>(jmax - tail), static_cast<long long>(jmax), sm_count(),
              fused::kThreadsPerCta, chains, static_cast<long long>(sm_count()) - chains,
+             r.lay.total);
+  } else if (r.variant == KDA_VARIANT_STREAM) {
+    const long long grid = static_cast<long long>(kStreamCtasPerSm) * sm_count();
+    snprintf(buf, n,
+             "variant=stream chunk=%d grid=%lldx%d (recurrence CTAs %lld, prepare CTAs %lld, "
+             "%d CTAs per SM, cooperative) workspace_bytes=%zu",
+             kC, grid, stream::kThreadsPerCta, chains, grid - chains, kStreamCtasPerSm,
              r.lay.total);
   } else if (r.variant == KDA_VARIANT_FUSED) {
     snprintf(buf, n,
@@ -466,13 +489,10 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
   const Resolved r = resolve(shape, fixed, ckpt, options);
   const size_t need = kda_prefill_workspace_size(shape, ckpt ? 1 : 0, options);
   if (workspace_bytes < need || workspace_bytes < r.lay.total) return KDA_ERR_WORKSPACE_TOO_SMALL;
-  // beta from logits only in the token variant: the chunked variants hold T diag(beta)
-  // as a BF16 tensor-core operand whose diagonal is beta itself, exact only for BF16 beta
-  if (fe && (fe->flags & KDA_FE_BETA_LOGIT) && r.variant != KDA_VARIANT_TOKEN)
-    return KDA_ERR_BAD_OPTION;
   // the fused launch needs an SM per chain plus SMs for its prepare CTAs
   if ((r.variant == KDA_VARIANT_FUSED || r.variant == KDA_VARIANT_HYBRID) && !fused_eligible(shape))
     return KDA_ERR_BAD_OPTION;
+  if (r.variant == KDA_VARIANT_STREAM && !stream_eligible(shape)) return KDA_ERR_BAD_OPTION;
 
   // ---------------- device
   st = device_check();
@@ -534,9 +554,13 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
     else
       mok &= make_map_rows(&maps.g_in, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, g, T, H, 4);
     mok &= make_map_rows(&maps.o_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, out, T, H, 2);
-    mok &= make_map_2d(&maps.wt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ws + r.lay.wt, 64, recs * 128, 64, 128, 2);
-    mok &= make_map_2d(&maps.qg, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ws + r.lay.qg, 128, recs * 64, 64, 64, 2);
-    mok &= make_map_2d(&maps.ut, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws + r.lay.ut, 64, recs * 128, 64, 128, 2);
+    if (r.variant == KDA_VARIANT_STREAM) {
+      mok &= make_map_2d(&maps.qw, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws + r.lay.qw, 128, recs * 128, 64, 128, 2);
+    } else {
+      mok &= make_map_2d(&maps.wt, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws + r.lay.wt, 64, recs * 128, 64, 128, 2);
+      mok &= make_map_2d(&maps.qg, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws + r.lay.qg, 128, recs * 64, 64, 64, 2);
+      mok &= make_map_2d(&maps.ut, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws + r.lay.ut, 64, recs * 128, 64, 128, 2);
+    }
     mok &= make_map_2d(&maps.kd, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws + r.lay.kd, 128, recs * 64, 64, 64, 2);
     mok &= make_map_2d(&maps.aqk, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws + r.lay.aqk, 64, recs * 64, 64, 64, 2);
   }
@@ -562,7 +586,13 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
     cudaError_t e5 = cudaFuncSetAttribute(kda_fused_fe_kernel,
                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           fused::kSmemAllocBytes);
-    const cudaError_t es[] = {e1, e2, e3, e4, e5};
+    cudaError_t e6 = cudaFuncSetAttribute(kda_stream_kernel,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          stream::kSmemAllocBytes);
+    cudaError_t e7 = cudaFuncSetAttribute(kda_stream_fe_kernel,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          stream::kSmemAllocBytes);
+    const cudaError_t es[] = {e1, e2, e3, e4, e5, e6, e7};
     for (cudaError_t e : es)
       if (attr_err == cudaSuccess) attr_err = e;
   });
@@ -610,6 +640,33 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
     tp.l2_eps = p.l2_eps;
     st = launch_token(tp, N * H, token_wide(N * H, 0), s);
     if (st != KDA_OK) return st;
+    mark(2);
+  } else if (r.variant == KDA_VARIANT_STREAM) {
+    mark(1);
+    // one cooperative launch of two CTAs per SM: CTAs 0 .. N H - 1 run the recurrences,
+    // the rest prepare the chunk records in chunk-major order
+    void* fn = p.fe_flags ? reinterpret_cast<void*>(kda_stream_fe_kernel)
+                          : reinterpret_cast<void*>(kda_stream_kernel);
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, stream::kThreadsPerCta,
+                                                      stream::kSmemAllocBytes) != cudaSuccess ||
+        per_sm < 1)
+      return KDA_ERR_LAUNCH_FAILED;
+    per_sm = std::min(per_sm, kStreamCtasPerSm);
+    int32_t rec_ctas = static_cast<int32_t>(N * H);
+    const int64_t grid = static_cast<int64_t>(per_sm) * sm_count();
+    if (rec_ctas + kFusedMinPrepCtas > grid) return KDA_ERR_BAD_OPTION;
+    const int64_t jmax = max_chunks_per_seq(shape, fixed, ckpt);
+    int64_t prep_items = jmax * static_cast<int64_t>(rec_ctas);
+    if (r.lay.slots > 0 &&
+        cudaMemsetAsync(ws + r.lay.ready, 0, static_cast<size_t>(r.lay.slots) * H * sizeof(int32_t),
+                        s) != cudaSuccess)
+      return KDA_ERR_LAUNCH_FAILED;
+    void* args[] = {&p, &maps, &rec_ctas, &prep_items};
+    if (cudaLaunchCooperativeKernel(fn, dim3(static_cast<unsigned>(grid)),
+                                    dim3(stream::kThreadsPerCta), args, stream::kSmemAllocBytes,
+                                    s) != cudaSuccess)
+      return KDA_ERR_LAUNCH_FAILED;
     mark(2);
   } else if (r.variant == KDA_VARIANT_FUSED || r.variant == KDA_VARIANT_HYBRID) {
     const int64_t jmax = max_chunks_per_seq(shape, fixed, ckpt);

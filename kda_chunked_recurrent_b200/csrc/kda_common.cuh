@@ -32,18 +32,22 @@ constexpr float kLog2e = 1.4426950408889634f;
 // header (status word, per-call validity) | chunk table | per-record tiles.
 // A "record" is one (chunk slot, head) pair: rec = slot * H + h.
 constexpr size_t kHeaderBytes = 1024;
-constexpr size_t kTileWT = 128 * 64 * 2;   // W^T   [128 k][64 tok] bf16
-constexpr size_t kTileQG = 64 * 128 * 2;   // Q*Gamma [64 tok][128 k] bf16 (token rows)
+constexpr size_t kTileWT = 128 * 64 * 2;   // W^T   [128 k][64 tok] f16
+constexpr size_t kTileQG = 64 * 128 * 2;   // Q*Gamma [64 tok][128 k] f16 (token rows)
 constexpr size_t kTileUT = 128 * 64 * 2;   // U^T   [128 v][64 tok] f16
 constexpr size_t kTileKd = 64 * 128 * 2;   // Kd    [64 tok][128 k] f16 (token rows)
 constexpr size_t kTileAqk = 64 * 64 * 2;   // Aqk   [64 r][64 s]  f16
 constexpr size_t kTileGC = 128 * 4;        // Gamma at the chunk end, f32 [128]
+// records of the stream variant (same bytes per record, token-row orientation)
+constexpr size_t kTileQW = 128 * 128 * 2;  // [Q*Gamma; W] [128 rows][128 k] f16 (rows 0..63 Q Gamma)
+constexpr size_t kTileU = 64 * 128 * 2;    // U [64 tok][128 v] f16
 
 struct WorkspaceLayout {
   size_t cu32;         // int32 [N+1]   narrowed copy of INT64 cu_seqlens
   size_t chunk_base;   // int32 [N+1]   first slot of each sequence
   size_t seq_order;    // int32 [N]     longest-first order of sequences
   size_t wt, qg, ut, kd, aqk, gc;     // per-record tiles
+  size_t qw, u;                       // per-record tiles of the stream variant
   size_t ready;        // int32 [recs]  per-record ready flags (fused variant)
   size_t total;
   int64_t slots;       // chunk slots (upper bound on the number of chunks)
@@ -61,7 +65,7 @@ __host__ __device__ inline int64_t chunk_slots(int64_t N, int64_t T, bool fixed,
 }
 
 inline WorkspaceLayout make_layout(int64_t N, int64_t T, int64_t H, bool fixed, bool split,
-                                   bool ckpt) {
+                                   bool ckpt, bool stream = false) {
   WorkspaceLayout L{};
   size_t off = kHeaderBytes;
   L.cu32 = off;
@@ -72,9 +76,14 @@ inline WorkspaceLayout make_layout(int64_t N, int64_t T, int64_t H, bool fixed, 
   off = align_up(off + sizeof(int32_t) * N, 1024);
   L.slots = (N > 0 && T > 0) ? chunk_slots(N, T, fixed, ckpt) : 0;
   const size_t recs = split ? static_cast<size_t>(L.slots * H) : 0;
-  L.wt = off;  off = align_up(off + recs * kTileWT, 1024);
-  L.qg = off;  off = align_up(off + recs * kTileQG, 1024);
-  L.ut = off;  off = align_up(off + recs * kTileUT, 1024);
+  if (stream) {   // [Q Gamma; W] and U replace W^T, Q Gamma and U^T (same bytes)
+    L.qw = off;  off = align_up(off + recs * kTileQW, 1024);
+    L.u = off;   off = align_up(off + recs * kTileU, 1024);
+  } else {
+    L.wt = off;  off = align_up(off + recs * kTileWT, 1024);
+    L.qg = off;  off = align_up(off + recs * kTileQG, 1024);
+    L.ut = off;  off = align_up(off + recs * kTileUT, 1024);
+  }
   L.kd = off;  off = align_up(off + recs * kTileKd, 1024);
   L.aqk = off; off = align_up(off + recs * kTileAqk, 1024);
   L.gc = off;  off = align_up(off + recs * kTileGC, 1024);
@@ -136,11 +145,12 @@ struct SplitMaps {
   CUtensorMap k_in;     // k, as q
   CUtensorMap g_in;     // g [T][H][128] f32, box (128 ch, 1 head, 64 tok), no swizzle
   CUtensorMap o_out;    // out [T][H][128] bf16, box (128 ch, 1 head, 64 tok), no swizzle
-  CUtensorMap wt;       // [recs*128][64] bf16, box (64, 128)
-  CUtensorMap qg;       // [recs*64][128] bf16, box (64, 64): one 64-channel panel
+  CUtensorMap wt;       // [recs*128][64] f16, box (64, 128)
+  CUtensorMap qg;       // [recs*64][128] f16, box (64, 64): one 64-channel panel
   CUtensorMap ut;       // [recs*128][64] f16, box (64, 128)
   CUtensorMap kd;       // [recs*64][128] f16, box (64, 64)
   CUtensorMap aqk;      // [recs*64][64] f16, box (64, 64)
+  CUtensorMap qw;       // stream: [recs*128][128] f16, box (64, 128): one 64-channel panel
 };
 
 enum : int32_t {

@@ -12,10 +12,10 @@
 // It runs exactly the same kernels as kda_prefill (it calls kda_prefill with the
 // built-in area as the workspace), so results are identical.  Nothing in the
 // area has to be cleared between calls: every table and tile a call reads is
-// written earlier in the same call (the area starts zeroed at load time).
+// written earlier in the same call (the area starts zeroed at load time).  The
+// status word in the area is never read through this entry point, so the modes
+// that report only through it (validate, the forced-timeout test hook) are refused.
 #include <cuda_runtime.h>
-
-#include <mutex>
 
 #include "../../include/kda_prefill.h"
 
@@ -24,25 +24,27 @@ namespace {
 constexpr size_t kScratchBytes = KDA_NOALLOC_SCRATCH_BYTES;
 static __device__ __align__(256) unsigned char g_kda_noalloc_scratch[kScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void* g_scratch_addr[kMaxDevices] = {};
-
-// Device address of the built-in area on the current device.  The array's name
-// in host code is only a stand-in for the symbol, so the address is looked up
-// once per device (with that device current) and remembered.
-kda_status_t scratch_on_current_device(void** out) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+kda_status_t current_device_supported() {
+  int dev = -1, major = 0, minor = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return KDA_ERR_UNSUPPORTED_DEVICE;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
     return KDA_ERR_UNSUPPORTED_DEVICE;
-  std::lock_guard<std::mutex> lock(g_mu);
-  if (g_scratch_addr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_kda_noalloc_scratch) != cudaSuccess || p == nullptr)
-      return KDA_ERR_LAUNCH_FAILED;
-    g_scratch_addr[dev] = p;
+  return (major == 10 && minor == 0) ? KDA_OK : KDA_ERR_UNSUPPORTED_DEVICE;
+}
+
+// Device address of the built-in area on the current device.  The array's name in
+// host code is only a stand-in for the symbol, so the address is looked up with the
+// device current, on every call: the lookup is cheap, and a cached address would go
+// stale if the context were torn down and the module loaded again elsewhere.
+kda_status_t scratch_on_current_device(void** out) {
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_kda_noalloc_scratch);
+  if (e != cudaSuccess || p == nullptr) {
+    (void)cudaGetLastError();   // a failed lazy load leaves no sticky error behind
+    return KDA_ERR_SCRATCH_UNAVAILABLE;
   }
-  *out = g_scratch_addr[dev];
+  *out = p;
   return KDA_OK;
 }
 
@@ -55,13 +57,22 @@ extern "C" kda_status_t kda_prefill_noalloc(const void* q, const void* k, const 
                                             float* ckpt_state, const int32_t* ckpt_offsets,
                                             const kda_options_t* options, void* stream) {
   if (shape == nullptr) return KDA_ERR_NULL_ARG;
-  const size_t need = kda_prefill_workspace_size(shape, ckpt_state != nullptr, options);
-  if (need == 0)  // invalid shape or options: kda_prefill names the error, launching nothing
-    return kda_prefill(q, k, v, g, beta, scale, h0, cu_seqlens, shape, out, ht, ckpt_state,
-                       ckpt_offsets, nullptr, 0, options, stream);
+  // the status word of the built-in area is not readable here: refuse the modes that
+  // would report only through it (kda_prefill with a workspace of the caller's serves them)
+  if (options && (options->flags & (KDA_FLAG_VALIDATE | KDA_FLAG_TEST_FORCE_TIMEOUT)))
+    return KDA_ERR_BAD_OPTION;
+  const int has_ckpt = ckpt_state != nullptr;
+  // options and shape first, with the codes kda_prefill would give
+  char note[8];
+  kda_status_t st = kda_prefill_describe(shape, has_ckpt, options, note, sizeof(note));
+  if (st != KDA_OK) return st;
+  st = current_device_supported();
+  if (st != KDA_OK) return st;
+  const size_t need = kda_prefill_workspace_size(shape, has_ckpt, options);
+  if (need == 0) return KDA_ERR_BAD_SHAPE;
   if (need > kScratchBytes) return KDA_ERR_WORKSPACE_TOO_SMALL;  // shape too large for the area
   void* scratch = nullptr;
-  const kda_status_t st = scratch_on_current_device(&scratch);
+  st = scratch_on_current_device(&scratch);
   if (st != KDA_OK) return st;
   return kda_prefill(q, k, v, g, beta, scale, h0, cu_seqlens, shape, out, ht, ckpt_state,
                      ckpt_offsets, scratch, kScratchBytes, options, stream);

@@ -5,9 +5,9 @@
 // the records (chunk slot, head).  For each 64-token chunk it forms the decay-weighted
 // intra-chunk products, solves the unit-lower-triangular UT/WY system and
 // writes the per-chunk operands the recurrence kernel consumes:
-//   W^T [128 k][64 tok] bf16, U^T [128 v][64 tok] f16, Aqk [64][64] f16
+//   W^T [128 k][64 tok] f16, U^T [128 v][64 tok] f16, Aqk [64][64] f16
 //   (UMMA results, staged in shared memory and written by TMA tile stores),
-//   Q*Gamma [64 tok][128 k] bf16, Kd [64 tok][128 k] f16 (token rows, written
+//   Q*Gamma [64 tok][128 k] f16, Kd [64 tok][128 k] f16 (token rows, written
 //   straight from the element-wise pass with 128-byte warp stores),
 //   Gamma_end [128] f32.
 // A checkpoint offset p inside a sequence is a chunk boundary of the schedule
@@ -23,7 +23,7 @@
 // as that chunk's first UMMA and its Aqk store are done with R (the start of its
 // solve), q and k once its second UMMA has completed; all of them were
 // prefetched into L2 one chunk earlier.  v follows by TMA straight into its
-// UMMA operand layout.
+// UMMA operand layout and is converted from BF16 to FP16 in place during the solve.
 //
 // Thread mapping for the element-wise part: thread t owns the channel pair
 // (2p, 2p+1), p = t % 64, in sub-block b = t / 64 (tokens 16b .. 16b+15), so a
@@ -61,7 +61,8 @@ namespace kda {
 namespace prep {
 constexpr int kThreads = 256;
 constexpr uint32_t kV = 0;           // 16 KB  v tile, MN-major A of U^T: 2 panels [64 tok][64 v]
-constexpr uint32_t kKG = 16384;      // 16 KB  K*Gamma tile, MN-major A of W^T
+                                     //        (lands as BF16, converted to FP16 in place)
+constexpr uint32_t kKG = 16384;      // 16 KB  K*Gamma tile (f16), MN-major A of W^T
 constexpr uint32_t kL = 32768;       // 32 KB  [K+; Q+], K-major A: 2 panels [128 rows][64 ch]
 constexpr uint32_t kR = 65536;       // 40 KB  R^0..R^3, K-major B: 2 panels [160 rows][64 ch]
 constexpr uint32_t kBytes = 65536 + 40960;
@@ -82,11 +83,11 @@ constexpr uint32_t kMf = kL;                    // f32 [4][16][17] diagonal bloc
 constexpr uint32_t kMh = kMf + 4 * 16 * 17 * 4; // f16 [64][72] off-diagonal blocks of M
 constexpr uint32_t kXh = kMh + 64 * kLdh * 2;   // f16 [64][72] T = (I + M)^-1
 constexpr uint32_t kZh = kXh + 64 * kLdh * 2;   // f16 [64][72] Z_ik = -X_ii M_ik
-constexpr uint32_t kWs = kL;                    // W^T staging [128 k][64 tok] bf16, 128B swizzle
+constexpr uint32_t kWs = kL;                    // W^T staging [128 k][64 tok] f16, 128B swizzle
 constexpr uint32_t kUs = kL + 16384;            // U^T staging [128 v][64 tok] f16, 128B swizzle
 // aliases of R once the first UMMA has completed
 constexpr uint32_t kAqs = kR;                   // Aqk staging [64 r][64 s] f16, 128B swizzle
-constexpr uint32_t kTb = 98304;                 // 8 KB T diag(beta) bf16, K-major [64 r][64 s]
+constexpr uint32_t kTb = 98304;                 // 8 KB T diag(beta) f16, K-major [64 r][64 s]
 // small per-group state after the tiles: mbarriers, TMEM slot, beta, gate sums
 constexpr uint32_t kAux = kBytes;
 constexpr uint32_t kAuxBars = kAux;              // 4 x u64 mbarriers
@@ -162,7 +163,7 @@ __device__ __forceinline__ void store_frag16(__half* base, int ld, const float (
       __floats2half2_rn(s * c1[2], s * c1[3]);
 }
 
-// Store the same 16x16 block of T, scaled by beta of its column, as bf16 into the
+// Store the same 16x16 block of T, scaled by beta of its column, as FP16 into the
 // 128B-swizzled K-major Tb tile (rows r0.., columns c0..).
 __device__ __forceinline__ void store_tb16(uint32_t tb, const float* beta, int r0, int c0,
                                            const float (&x0)[4], const float (&x1)[4], int lane) {
@@ -171,15 +172,15 @@ __device__ __forceinline__ void store_tb16(uint32_t tb, const float* beta, int r
     const int s = c0 + 2 * q;
     const float b0 = beta[s], b1 = beta[s + 1];
     const uint32_t off = static_cast<uint32_t>((s & 7) * 2);
-    sts32(tb + sw128_offset(r0 + g, s >> 3) + off, pack_bf16(x0[0] * b0, x0[1] * b1));
-    sts32(tb + sw128_offset(r0 + g + 8, s >> 3) + off, pack_bf16(x0[2] * b0, x0[3] * b1));
+    sts32(tb + sw128_offset(r0 + g, s >> 3) + off, pack_f16(x0[0] * b0, x0[1] * b1));
+    sts32(tb + sw128_offset(r0 + g + 8, s >> 3) + off, pack_f16(x0[2] * b0, x0[3] * b1));
   }
   {
     const int s = c0 + 8 + 2 * q;
     const float b0 = beta[s], b1 = beta[s + 1];
     const uint32_t off = static_cast<uint32_t>((s & 7) * 2);
-    sts32(tb + sw128_offset(r0 + g, s >> 3) + off, pack_bf16(x1[0] * b0, x1[1] * b1));
-    sts32(tb + sw128_offset(r0 + g + 8, s >> 3) + off, pack_bf16(x1[2] * b0, x1[3] * b1));
+    sts32(tb + sw128_offset(r0 + g, s >> 3) + off, pack_f16(x1[0] * b0, x1[1] * b1));
+    sts32(tb + sw128_offset(r0 + g + 8, s >> 3) + off, pack_f16(x1[2] * b0, x1[3] * b1));
   }
 }
 
@@ -320,11 +321,11 @@ __device__ __forceinline__ void publish_record(const KdaParams& p, int64_t rec) 
 // nitems; kFused selects the chunk-major item order, the named barriers and the
 // ready flags.
 // kFE: the input front end is compiled in (switches in p.fe_flags): the gate is formed
-// from the raw BF16 gate tile in the scan, and the inverse L2 norms of the k and q rows
+// from the raw BF16 gate tile in the scan, the inverse L2 norms of the k and q rows
 // are folded into the FP32 factors that already multiply them (so every operand keeps
-// its single rounding).  Beta from a logit is not offered here: T diag(beta) is a BF16
-// operand whose diagonal is beta itself, exact only for a BF16 beta.
-template <bool kFused, bool kFE = false>
+// its single rounding), and beta is squashed from its logit in FP32.  T diag(beta) is
+// an FP16 operand, so the squashed beta on its diagonal keeps 2^-11 relative precision.
+template <bool kFused, bool kFE = false, bool kStream = false>
 __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps& maps,
                                              uint8_t* smem_raw, int grp, int64_t first,
                                              int64_t stride, int64_t nitems) {
@@ -344,6 +345,7 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
   float* s_norm = reinterpret_cast<float*>(sm + kAuxNorm);   // front end: 1/|k_r|, then 1/|q_r|
   const bool fe_gate = kFE && (p.fe_flags & 2u) != 0;
   const bool fe_norm = kFE && (p.fe_flags & 1u) != 0;
+  const bool fe_beta = kFE && (p.fe_flags & 4u) != 0;
   const uint32_t raw_g_tx = fe_gate ? 16384u : kRawGTx;   // raw gate tile is BF16
 
   const int tid = threadIdx.x - grp * kThreads;
@@ -581,11 +583,13 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
       const uint32_t bR = sbase + kR + panel * 20480u + inner;
       const uint32_t bRo = bR + static_cast<uint32_t>(seg_own) * 128u;
       const uint32_t bKG = sbase + kKG + panel * 8192u + inner;
-      const uint32_t cB2 = pack_bf16(cB.x, cB.y);
       const uint32_t c1b = pack_bf16(c1.x, c1.y), c2b = pack_bf16(c2.x, c2.y),
                      c3b = pack_bf16(c3.x, c3.y);
       // Q Gamma and Kd token rows: this thread's channel pair of rows 16 blk + i
-      uint32_t* qg_out = reinterpret_cast<uint32_t*>(p.ws + p.lay.qg + rec * kTileQG) + blk * 16 * 64 + cp;
+      // (the stream records keep Q Gamma as rows 0..63 of the [Q Gamma; W] tile)
+      uint32_t* qg_out = reinterpret_cast<uint32_t*>(
+                             kStream ? p.ws + p.lay.qw + rec * kTileQW : p.ws + p.lay.qg + rec * kTileQG) +
+                         blk * 16 * 64 + cp;
       uint32_t* kd_out = reinterpret_cast<uint32_t*>(p.ws + p.lay.kd + rec * kTileKd) + blk * 16 * 64 + cp;
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
@@ -604,8 +608,10 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
           if (blk < 1) sts32(bR + xo + 16u * 128u, hmul2_bf16(rd2, c1b));
           if (blk < 2) sts32(bR + xo + 48u * 128u, hmul2_bf16(rd2, c2b));
           if (blk < 3) sts32(bR + xo + 96u * 128u, hmul2_bf16(rd2, c3b));
-          sts32(bKG + xo, hmul2_bf16(kw[i], pack_bf16(e0 * cB.x * rk, e1 * cB.y * rk)));
-          qg_out[i * 64] = hmul2_bf16(qw[i], pack_bf16(e0 * cB.x * rq, e1 * cB.y * rq));
+          const float2 kf = bf2_to_f2(kw[i]), qf = bf2_to_f2(qw[i]);
+          const float gx = e0 * cB.x, gy = e1 * cB.y;   // Gamma_r, FP32
+          sts32(bKG + xo, pack_f16(kf.x * (gx * rk), kf.y * (gy * rk)));
+          qg_out[i * 64] = pack_f16(qf.x * (gx * rq), qf.y * (gy * rq));
           i0 *= rk;
           i1 *= rk;
         } else {
@@ -618,9 +624,12 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
           if (blk < 1) sts32(bR + xo + 16u * 128u, hmul2_bf16(rd2, c1b));
           if (blk < 2) sts32(bR + xo + 48u * 128u, hmul2_bf16(rd2, c2b));
           if (blk < 3) sts32(bR + xo + 96u * 128u, hmul2_bf16(rd2, c3b));
-          const uint32_t gm2 = hmul2_bf16(e2, cB2);
-          sts32(bKG + xo, hmul2_bf16(kw[i], gm2));
-          qg_out[i * 64] = hmul2_bf16(qw[i], gm2);
+          // K Gamma (A of the W UMMA) and Q Gamma (B of the state read): FP16 products of
+          // FP32 factors, one rounding each
+          const float2 kf = bf2_to_f2(kw[i]), qf = bf2_to_f2(qw[i]);
+          const float gx = e0 * cB.x, gy = e1 * cB.y;   // Gamma_r, FP32
+          sts32(bKG + xo, pack_f16(kf.x * gx, kf.y * gy));
+          qg_out[i * 64] = pack_f16(qf.x * gx, qf.y * gy);
         }
         // Kd feeds the FP16 state update: FP32 products, one rounding
         const float2 kf = bf2_to_f2(kw[i]);
@@ -630,7 +639,12 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
         reinterpret_cast<float2*>(p.ws + p.lay.gc + rec * kTileGC)[cp] =
             make_float2(ex2(E.x), ex2(E.y));
     }
-    if (tid < kC) s_beta[tid] = bf16_to_f32(beta_raw);
+    if (tid < kC) {
+      // beta (or, from raw projections, sigmoid of its BF16 logit, in FP32): it scales M
+      // in FP32 and reaches the tensor core only through the FP16 T diag(beta)
+      const float b = bf16_to_f32(beta_raw);
+      s_beta[tid] = fe_beta ? 1.f / (1.f + ex2(-b * kLog2e)) : b;
+    }
 
     // ---- UMMA 1: D[0:128, 0:160] = [K+; Q+] . R^T   (bf16 -> f32)
     fence_proxy_async_smem();
@@ -745,11 +759,11 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
         }
         const int col = bi * 16 + jj;
         const float bcol = s_beta[col];
-        __nv_bfloat16* tbp = reinterpret_cast<__nv_bfloat16*>(sm + kTb + (col & 7) * 2);
+        __half* tbp = reinterpret_cast<__half*>(sm + kTb + (col & 7) * 2);
 #pragma unroll
         for (int rr = 0; rr < 16; ++rr) {
           Xh[(bi * 16 + rr) * kLdh + col] = __float2half_rn(x[rr]);
-          tbp[sw128_offset(bi * 16 + rr, col >> 3) >> 1] = __float2bfloat16_rn(x[rr] * bcol);
+          tbp[sw128_offset(bi * 16 + rr, col >> 3) >> 1] = __float2half_rn(x[rr] * bcol);
         }
       } else {
         // ---- strictly upper blocks of Tb are zero
@@ -757,6 +771,21 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
           const int r = slot >> 3, ch = slot & 7;
           if (ch >= 2 * ((r >> 4) + 1))
             *reinterpret_cast<uint4*>(sm + kTb + sw128_offset(r, ch)) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        // ---- the v tile (BF16, landed by TMA in its operand layout) becomes FP16 in
+        // place: the U UMMA multiplies it by the FP16 T diag(beta), and both operands of
+        // one UMMA share a type.  (BF16 -> FP16 is exact for |v| in the FP16 normal range.)
+        if (mbar_wait(&tma_bar, tma_parity, budget)) {
+          uint4* vt = reinterpret_cast<uint4*>(sm + kV);
+          for (int i = tid - 64; i < 16384 / 16; i += kThreads - 64) {
+            const uint4 x = vt[i];
+            const float2 a = bf2_to_f2(x.x), b = bf2_to_f2(x.y), c2 = bf2_to_f2(x.z),
+                         d = bf2_to_f2(x.w);
+            vt[i] = make_uint4(pack_f16(a.x, a.y), pack_f16(b.x, b.y), pack_f16(c2.x, c2.y),
+                               pack_f16(d.x, d.y));
+          }
+        } else {
+          ok = false;
         }
       }
       prep_sync<kFused>(grp);
@@ -807,13 +836,26 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
       tma_seen = mbar_wait(&tma_bar, tma_parity, budget);
       if (tma_seen) {
         tc_fence_after();
-        const uint32_t idesc = idesc_f16(128, 64, kFmtBF16, kMNMajor, kKMajor);
-        const uint32_t aKG = sbase + kKG, aV = sbase + kV, bT = sbase + kTb;
+        if constexpr (kStream) {
+          // token rows [U | W] = (T diag beta) [V | K Gamma]: A = T diag(beta) as rows
+          // 64..127 of an M = 128 operand (rows 0..63 read the 8 KB below it; their
+          // products land in TMEM lanes 0..63, which no one reads); B = [V | K Gamma],
+          // MN-major, four 64-column panels 8 KB apart (V, then K Gamma); N = 256
+          const uint32_t idesc = idesc_f16(128, 256, kFmtF16, kKMajor, kMNMajor);
+          const uint32_t aT = sbase + kTb - 8192, bVK = sbase + kV;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t bd = sdesc_sw128(bT + kk * 32, 16, 1024);
-          umma_f16(tbase + 0, sdesc_sw128(aKG + kk * 2048, 8192, 1024), bd, idesc, kk > 0);
-          umma_f16(tbase + 64, sdesc_sw128(aV + kk * 2048, 8192, 1024), bd, idesc, kk > 0);
+          for (int kk = 0; kk < 4; ++kk)
+            umma_f16(tbase, sdesc_sw128(aT + kk * 32, 16, 1024), sdesc_sw128(bVK + kk * 2048, 8192, 1024),
+                     idesc, kk > 0);
+        } else {
+          const uint32_t idesc = idesc_f16(128, 64, kFmtF16, kMNMajor, kKMajor);
+          const uint32_t aKG = sbase + kKG, aV = sbase + kV, bT = sbase + kTb;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t bd = sdesc_sw128(bT + kk * 32, 16, 1024);
+            umma_f16(tbase + 0, sdesc_sw128(aKG + kk * 2048, 8192, 1024), bd, idesc, kk > 0);
+            umma_f16(tbase + 64, sdesc_sw128(aV + kk * 2048, 8192, 1024), bd, idesc, kk > 0);
+          }
         }
         umma_commit(&mma_bar);
       }
@@ -832,7 +874,33 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
       ++raw_qk_issued;
       qk_for_cur = true;
     }
-    if (ok) {
+    if (ok && kStream) {
+      tc_fence_after();
+      // TMEM lanes 64..127 hold token row r = lane - 64 of [U | W]: warps 2, 3 write the
+      // U row, warps 6, 7 the W row (into rows 64..127 of the [Q Gamma; W] tile), each
+      // 128 FP16 values = 256 contiguous bytes
+      if ((warp & 3) >= 2) {
+        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32);
+        const int r = ((warp & 3) - 2) * 32 + lane;
+        const bool is_w = warp >= 4;
+        uint4* dst = reinterpret_cast<uint4*>(
+            is_w ? p.ws + p.lay.qw + rec * kTileQW + static_cast<int64_t>(64 + r) * 256
+                 : p.ws + p.lay.u + rec * kTileU + static_cast<int64_t>(r) * 256);
+        const uint32_t col0 = is_w ? 128u : 0u;
+        uint32_t a[32];
+#pragma unroll
+        for (int part = 0; part < 4; ++part) {
+          tmem_ld32(tmem_addr(tbase, lane_base, col0 + part * 32), a);
+          tmem_wait_ld();
+#pragma unroll
+          for (int q8 = 0; q8 < 4; ++q8) {
+            const float* f = reinterpret_cast<const float*>(a) + q8 * 8;
+            dst[part * 4 + q8] = make_uint4(pack_f16(f[0], f[1]), pack_f16(f[2], f[3]),
+                                            pack_f16(f[4], f[5]), pack_f16(f[6], f[7]));
+          }
+        }
+      }
+    } else if (ok) {
       tc_fence_after();
       // warps 0-3: W^T rows (lane = k); warps 4-7: U^T rows (lane = v), into the
       // swizzled staging tiles of the TMA stores
@@ -850,13 +918,8 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
         for (int q8 = 0; q8 < 4; ++q8) {
           uint4 o;
           const float* f = reinterpret_cast<const float*>(a) + q8 * 8;
-          if (is_u) {
-            o = make_uint4(pack_f16(f[0], f[1]), pack_f16(f[2], f[3]), pack_f16(f[4], f[5]),
-                           pack_f16(f[6], f[7]));
-          } else {
-            o = make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
-                           pack_bf16(f[6], f[7]));
-          }
+          o = make_uint4(pack_f16(f[0], f[1]), pack_f16(f[2], f[3]), pack_f16(f[4], f[5]),
+                         pack_f16(f[6], f[7]));
           *reinterpret_cast<uint4*>(dst + sw128_offset(row, part * 4 + q8)) = o;
         }
       }
@@ -874,7 +937,7 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
     fence_proxy_async_smem();
     tc_fence_before();
     ok = !prep_sync_or<kFused>(grp, !ok);
-    if (ok && tid == 0) {
+    if (ok && tid == 0 && !kStream) {
       tma_store_2d(&maps.wt, sm + kWs, 0, static_cast<int32_t>(rec * 128));
       tma_store_2d(&maps.ut, sm + kUs, 0, static_cast<int32_t>(rec * 128));
       bulk_commit();

@@ -6,8 +6,8 @@
 // TMA carry it, and the output (intra-chunk causal term plus the read of S by
 // q) is formed in the same CTA.  The state is
 // kept transposed, S^T[v][k], in TMEM lanes v = 0..127, so every UMMA has M = 128:
-//   P_W^T = S0^T W^T                            (N=64, K=128; bf16; B = W^T, MN-major)
-//   P_Q^T = S0^T (Q Gamma)^T                    (N=64, K=128; bf16; B = Q Gamma rows, K-major)
+//   P_W^T = S0^T W^T                            (N=64, K=128; f16; B = W^T, MN-major)
+//   P_Q^T = S0^T (Q Gamma)^T                    (N=64, K=128; f16; B = Q Gamma rows, K-major)
 //   Ud^T  = U^T - P_W^T                         (threads; f16 operand)
 //   S^T   = S0^T Diag(Gamma_end) + Ud^T Kd      (N=128, K=64; f16; B = Kd rows, MN-major)
 //   O^T   = scale (P_Q^T + Ud^T Aqk^T)          (N=64, K=64; f16)
@@ -15,7 +15,7 @@
 // state is S after the chunk that ends at p (h0 for p = 0, the final state for
 // p = len).
 //
-// Serial chain per chunk: S ready -> (state warps) bf16 S0^T into TMEM -> P_W
+// Serial chain per chunk: S ready -> (state warps) f16 S0^T into TMEM -> P_W
 // -> (state warps) f16 Ud^T into TMEM and the decayed S -> S update.  P_Q is
 // issued right behind P_W and runs while the state warps form Ud.
 // S0^T and Ud^T are the A operands of their UMMAs straight from tensor memory,
@@ -29,7 +29,7 @@
 // Tensor memory (512 columns):
 //   [0, 128)    S^T f32 (lane v, column k)
 //   [128, 384)  two regions: P_W^T (64 columns) then P_Q^T / O^T (64 columns)
-//   [384, 448)  S0^T bf16, two k per column (A operand of P_W and P_Q)
+//   [384, 448)  S0^T f16, two k per column (A operand of P_W and P_Q)
 //   [448, 480)  Ud^T f16, two tokens per column (A operand of the update and O)
 //
 // Warp roles:
@@ -56,8 +56,8 @@
 namespace kda {
 
 namespace rec {
-constexpr uint32_t kWQ = 0;          // 16 KB W^T [128 k][64 tok] bf16, MN-major B;
-                                     // 16 KB Q Gamma [64 tok][128 k] bf16, K-major B, 2 panels
+constexpr uint32_t kWQ = 0;          // 16 KB W^T [128 k][64 tok] f16, MN-major B;
+                                     // 16 KB Q Gamma [64 tok][128 k] f16, K-major B, 2 panels
 constexpr uint32_t kUT = 32768;      // 16 KB U^T  [128 v][64 tok] f16 (128B swizzle)
 constexpr uint32_t kKd = 49152;      // 16 KB Kd [64 tok][128 k] f16, MN-major B, 2 panels
 constexpr uint32_t kAqk = 65536;     //  8 KB Aqk  [64 r][64 s] f16, K-major B
@@ -210,8 +210,8 @@ __device__ __forceinline__ void recurrence_body(const KdaParams& p, const SplitM
   } else if (warp == kMmaWarp) {
     // =========================== UMMA issuer =====================================
     const bool lead = (tid & 31) == 0;
-    const uint32_t id_p = idesc_f16(128, 64, kFmtBF16, kKMajor, kMNMajor);
-    const uint32_t id_q = idesc_f16(128, 64, kFmtBF16, kKMajor, kKMajor);
+    const uint32_t id_p = idesc_f16(128, 64, kFmtF16, kKMajor, kMNMajor);
+    const uint32_t id_q = idesc_f16(128, 64, kFmtF16, kKMajor, kKMajor);
     const uint32_t id_s = idesc_f16(128, 128, kFmtF16, kKMajor, kMNMajor);
     const uint32_t id_o = idesc_f16(128, 64, kFmtF16, kKMajor, kKMajor);
     const uint32_t tS0 = tbase + kColS0, tUd = tbase + kColUd;
@@ -383,16 +383,17 @@ __device__ __forceinline__ void recurrence_body(const KdaParams& p, const SplitM
       if (ok) {
         // checkpoint: the state after the chunk that ends at the offset
         if (ckc && si.nA > 0 && j == si.nA) store_state(ckc);
-        // (b) S0^T half row -> bf16 A operand in TMEM
+        // (b) S0^T half row -> f16 A operand in TMEM (FP16: 2^-11 rounding; the state
+        // stays far inside the FP16 range for the inputs the header admits)
         tmem_ld32(tmem_addr(tbase, lane_base, kColS + hw * 64), a);
         tmem_ld32(tmem_addr(tbase, lane_base, kColS + hw * 64 + 32), b);
         tmem_wait_ld();
         uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(__uint_as_float(a[2 * i]), __uint_as_float(a[2 * i + 1]));
+        for (int i = 0; i < 16; ++i) pk[i] = pack_f16(__uint_as_float(a[2 * i]), __uint_as_float(a[2 * i + 1]));
         tmem_st16(tmem_addr(tbase, lane_base, kColS0 + hw * 32), pk);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(__uint_as_float(b[2 * i]), __uint_as_float(b[2 * i + 1]));
+        for (int i = 0; i < 16; ++i) pk[i] = pack_f16(__uint_as_float(b[2 * i]), __uint_as_float(b[2 * i + 1]));
         tmem_st16(tmem_addr(tbase, lane_base, kColS0 + hw * 32 + 16), pk);
         tmem_wait_st();
       }

@@ -1,8 +1,12 @@
 """ctypes front end of the FP64 per-token oracle (kda_oracle.c).
 
 Test infrastructure only (see the package docstring).  The C source is
-compiled with gcc on first use into ``oracle/_build/``; no flag that changes
-the IEEE semantics (no -ffast-math) is used.
+compiled with gcc on first use into ``oracle/_build/`` with -O3 -march=native.
+No flag that changes the IEEE semantics is used: no -ffast-math, and -std=c99
+keeps floating-point contraction off, so the host's FMA units never fuse a
+product into a sum and the results do not depend on the machine.  The library
+name carries a hash of the host's native target flags, so a build made on one
+machine is never loaded on another CPU.
 """
 from __future__ import annotations
 
@@ -17,34 +21,49 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "kda_oracle.c")
 _BUILD = os.path.join(_HERE, "_build")
-_LIB = os.path.join(_BUILD, "libkda_oracle.so")
 _lock = threading.Lock()
 _lib = None
 
 
+CFLAGS = ["-O3", "-march=native", "-fopenmp", "-fPIC", "-shared", "-std=c99", "-Wall"]
+
+
+def _native_tag() -> str:
+    """Short hash of the target flags gcc picks for -march=native on this host."""
+    import hashlib
+    r = subprocess.run(["gcc", "-march=native", "-Q", "--help=target"], capture_output=True,
+                       text=True, check=True)
+    return hashlib.sha1(r.stdout.encode()).hexdigest()[:10]
+
+
+_TAG = None
+
+
 def oracle_library_path() -> str:
-    return _LIB
+    global _TAG
+    if _TAG is None:
+        _TAG = _native_tag()
+    return os.path.join(_BUILD, f"libkda_oracle_{_TAG}.so")
 
 
 def build_oracle(force: bool = False) -> str:
-    """Compile kda_oracle.c into a shared library (gcc, -O2, OpenMP)."""
+    """Compile kda_oracle.c into a shared library (gcc -O3 -march=native, OpenMP)."""
     os.makedirs(_BUILD, exist_ok=True)
-    stale = (not os.path.exists(_LIB)) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC)
+    lib = oracle_library_path()
+    stale = (not os.path.exists(lib)) or os.path.getmtime(lib) < os.path.getmtime(_SRC)
     if force or stale:
-        tmp = _LIB + f".tmp{os.getpid()}"
-        cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c99", "-Wall", "-o", tmp,
-               _SRC, "-lm"]
+        tmp = lib + f".tmp{os.getpid()}"
+        cmd = ["gcc"] + CFLAGS + ["-o", tmp, _SRC, "-lm"]
         subprocess.run(cmd, check=True)
-        os.replace(tmp, _LIB)
-    return _LIB
+        os.replace(tmp, lib)
+    return lib
 
 
 def _load():
     global _lib
     with _lock:
         if _lib is None:
-            build_oracle()
-            lib = ctypes.CDLL(_LIB)
+            lib = ctypes.CDLL(build_oracle())
             P = ctypes.c_void_p
             I64 = ctypes.c_int64
             lib.kda_oracle_prefill.restype = ctypes.c_int

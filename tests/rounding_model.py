@@ -7,11 +7,18 @@ before (or without) running a kernel.  Nothing here is shared with the CUDA path
 models its choices:
 
   A, Aqk   from [K+; Q+] R^T, operands rounded to BF16 per 16-token sub-block
-  T        (I + diag(beta) A)^-1, then T diag(beta) rounded to `tb` (BF16 or FP16)
-  W, U     T diag(beta) (K Gamma), T diag(beta) V; K Gamma rounded to BF16
+  T        (I + diag(beta) A)^-1, then T diag(beta) rounded to `tb` (FP16 or BF16)
+  W, U     T diag(beta) (K Gamma), T diag(beta) V; K Gamma and v in the type of `tb`
+           (both operands of one tensor-core product share a type)
+  S0       the state read by the tensor core, rounded to `s0` (FP16 or BF16), and
+           with it W and Q Gamma, its partners in the same products
   Ud       U - W S0, rounded to FP16 (the state update operand)
   Kd       K exp(G_end - G), rounded to FP16
   Aqk      rounded to FP16 for the output product
+
+The kernels' plan is the default (tb = s0 = FP16).  tb = s0 = BF16 is the earlier plan,
+which misses the 1e-3 state gate when nothing decays (g = 0): with Gamma = 1 every
+chunk's rounding error stays in the state.
 
 ``beta_split`` applies the split-beta scheme: T diag(bf16(beta)) is the rounded
 operand and diag(beta - bf16(beta)) is added unrounded-enough (a second BF16 tile of a
@@ -43,8 +50,8 @@ def to_f32(x):
 ROUND = {"bf16": to_bf16, "f16": to_f16, "f32": to_f32, "exact": lambda x: x}
 
 
-def chunk_step(q, k, v, g, beta, scale, S0, *, tb="bf16", ud="f16", kd="f16", aqk="f16",
-               beta_split=False):
+def chunk_step(q, k, v, g, beta, scale, S0, *, tb="f16", s0="f16", ud="f16", kd="f16",
+               aqk="f16", beta_split=False):
     """One chunk: returns (O [c, V], S1 [K, V])."""
     c = q.shape[0]
     G = to_f32(np.cumsum(to_f32(g), axis=0))
@@ -64,7 +71,8 @@ def chunk_step(q, k, v, g, beta, scale, S0, *, tb="bf16", ud="f16", kd="f16", aq
     T = solve_triangular(np.eye(c) + beta[:, None] * A, np.eye(c), lower=True,
                          unit_diagonal=True)
     gam = to_f32(np.exp(G))
-    kg = to_bf16(k * gam)
+    kg = ROUND[tb](k * gam)
+    v = ROUND[tb](v)
     if beta_split:
         hi = to_bf16(beta)
         lo = beta - hi
@@ -75,9 +83,9 @@ def chunk_step(q, k, v, g, beta, scale, S0, *, tb="bf16", ud="f16", kd="f16", aq
         tbm = ROUND[tb](to_f32(T * beta[None, :]))
         w = to_f32(tbm @ kg)
         u = to_f32(tbm @ v)
-    s0r = to_bf16(S0)
-    d = ROUND[ud](to_f32(to_f16(u) - to_bf16(w) @ s0r))
-    o = scale * (to_f32(to_bf16(q * gam) @ s0r) + to_f32(ROUND[aqk](Aq) @ d))
+    s0r = ROUND[s0](S0)
+    d = ROUND[ud](to_f32(to_f16(u) - ROUND[s0](w) @ s0r))
+    o = scale * (to_f32(ROUND[s0](q * gam) @ s0r) + to_f32(ROUND[aqk](Aq) @ d))
     kdm = ROUND[kd](k * to_f32(np.exp(G[-1][None, :] - G)))
     s1 = to_f32(to_f32(np.exp(G[-1]))[:, None] * S0) + to_f32(kdm.T @ d)
     return o, s1

@@ -32,7 +32,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_status_strings_cover_all_codes():
-    for code in (0, 1, 2, 3, 4, 5, 6, 7, 8, 9, 10, 16, 17, 18, 19):
+    for code in (0, 1, 2, 3, 4, 5, 6, 7, 8, 9, 10, 11, 16, 17, 18, 19):
         s = capi.kda_status_string(code)
         assert s and s != "unknown status"
     assert capi.kda_status_string(12345) == "unknown status"
@@ -53,6 +53,22 @@ def test_describe_reports_grid_and_variant():
     assert "variant=split" in d and "chunk=64" in d and "recurrence_grid=96x448" in d
     h = capi.kda_prefill_describe(capi.make_shape(8, 65536, 12, 8192), False, {"variant": 3})
     assert "variant=hybrid" in h and "prepare_chunks=" in h and "recurrence CTAs 96" in h
+    st = capi.kda_prefill_describe(capi.make_shape(8, 65536, 12, 8192), False, {"variant": 5})
+    assert "variant=stream" in st and "recurrence CTAs 96" in st and "2 CTAs per SM" in st
+    # stream and split records take the same workspace bytes
+    ws = [capi.kda_prefill_workspace_size(capi.make_shape(8, 65536, 12, 8192), False,
+                                          {"variant": v}) for v in (1, 5)]
+    assert ws[0] == ws[1]
+
+
+def test_stream_variant_needs_free_slots():
+    # two CTAs per SM: N H + 16 must fit twice the SM count (148 without a GPU)
+    big = capi.make_shape(2, 2 * 128, 160, 128)           # 320 chains
+    assert capi.kda_prefill_describe(big, False, {"variant": 5}).startswith("variant=stream")
+    o = capi.kda_options_t()
+    o.variant = 5
+    # 290 chains leave fewer than 16 of the 2 x 148 slots for prepare CTAs
+    assert call(fake_args(T=1, H=290, h0=None, ht=None, opts=o)) == capi.KDA_ERR_BAD_OPTION
 
 
 # --- host-side validation with fake, never-dereferenced device addresses ----------
@@ -199,8 +215,10 @@ def test_prefill_frontend_validation():
     assert call(fake_args(opts=opts(G, dt=BASE + 31 * MB + 8))) == capi.KDA_ERR_MISALIGNED
     # the gate parameters are inputs: an output on top of them is refused
     assert call(fake_args(opts=opts(G, dt=BASE + 8 * MB))) == capi.KDA_ERR_OUT_ALIAS
-    # beta from logits: only the token variant (the chunked ones hold T diag(beta) in BF16)
-    assert call(fake_args(opts=opts(B))) == capi.KDA_ERR_BAD_OPTION       # AUTO -> chunked
+    # beta from logits is accepted by every variant (the chunked ones hold T diag(beta)
+    # in FP16, which keeps a squashed FP32 beta on its diagonal to 2^-11)
+    chunked = opts(G | N2 | B)
+    chunked.variant = capi.KDA_VARIANT_SPLIT
     tok = opts(G | N2 | B)
     tok.variant = capi.KDA_VARIANT_TOKEN
     # with the gate switch g is BF16: a buffer right after its half size does not overlap it
@@ -210,3 +228,30 @@ def test_prefill_frontend_validation():
         assert call(dict(a, out=half_g_end)) == capi.KDA_ERR_UNSUPPORTED_DEVICE
         assert call(a) == capi.KDA_ERR_UNSUPPORTED_DEVICE
         assert call(fake_args(opts=tok)) == capi.KDA_ERR_UNSUPPORTED_DEVICE
+        assert call(fake_args(opts=chunked)) == capi.KDA_ERR_UNSUPPORTED_DEVICE
+        assert call(fake_args(opts=opts(B))) == capi.KDA_ERR_UNSUPPORTED_DEVICE
+
+
+def test_noalloc_host_checks_before_any_device_work():
+    """kda_prefill_noalloc refuses the status-word modes, then bad shapes, then a
+    missing B200, all on the host."""
+    lib = ctypes.CDLL(capi.LIB_PATH)
+    f = lib.kda_prefill_noalloc
+    P = ctypes.c_void_p
+    f.restype = ctypes.c_int
+    f.argtypes = [P, P, P, P, P, ctypes.c_float, P, P, ctypes.POINTER(capi.kda_shape_t),
+                  P, P, P, P, ctypes.POINTER(capi.kda_options_t), P]
+    x = BASE
+    shape = capi.make_shape(1, 64, 1)
+    for flag in (capi.KDA_FLAG_VALIDATE, capi.KDA_FLAG_TEST_FORCE_TIMEOUT):
+        o = capi.kda_options_t()
+        o.flags = flag
+        assert f(x, x, x, x, x, 0.1, None, None, ctypes.byref(shape), x + MB, None, None, None,
+                 ctypes.byref(o), None) == capi.KDA_ERR_BAD_OPTION
+    bad = capi.make_shape(0, 64, 1)
+    assert f(x, x, x, x, x, 0.1, None, None, ctypes.byref(bad), x + MB, None, None, None,
+             None, None) == capi.KDA_ERR_BAD_SHAPE
+    torch = pytest.importorskip("torch")
+    if not torch.cuda.is_available():
+        assert f(x, x, x, x, x, 0.1, None, None, ctypes.byref(shape), x + MB, None, None, None,
+                 None, None) == capi.KDA_ERR_UNSUPPORTED_DEVICE

@@ -1,5 +1,5 @@
 """Prefill from raw projections: the input front end (q/k L2 norm, gate from A_log and
-dt_bias under a lower bound; beta from its logit in the token variant) inside every
+dt_bias under a lower bound, beta from its logit) inside every
 variant's kernels vs the FP64 front-end oracle followed by the FP64 recurrence oracle
 (needs a B200)."""
 import pytest
@@ -40,12 +40,25 @@ def test_frontend_all_switches_token_variant():
     assert_parity(compare(inp, run_gpu(inp, variant=TOKEN, frontend=fe), frontend=fe))
 
 
-def test_frontend_beta_logit_refused_by_chunked_variants():
-    import kda_chunked_recurrent_b200 as K
-    inp, A_log, dt = make_frontend_inputs([100], 2, seed=805, fixed_layout=True)
-    with pytest.raises(K.KDAError) as e:
-        run_gpu(inp, variant=SPLIT, frontend=fe_dict(A_log, dt))
-    assert e.value.code == K.capi.KDA_ERR_BAD_OPTION
+@pytest.mark.parametrize("variant", [SPLIT, FUSED, HYBRID])
+def test_frontend_all_switches_chunked_variants(variant):
+    """All three switches, beta from its logit included (FlashInfer PR #4262 "Dispatch
+    contract" lists beta_is_logit with the norm and gate switches on the fast path)."""
+    inp, A_log, dt = make_frontend_inputs([300, 0, 129, 64, 1, 77], 3, seed=805 + variant,
+                                          with_h0=True, with_ckpt=True)
+    fe = fe_dict(A_log, dt)
+    assert_parity(compare(inp, run_gpu(inp, variant=variant, frontend=fe), frontend=fe))
+
+
+@pytest.mark.parametrize("variant", [SPLIT, HYBRID])
+def test_frontend_beta_logit_only_long(variant):
+    """Beta from logits alone over a multi-chunk sequence, g and q/k as given."""
+    inp, A_log, dt = make_frontend_inputs([1100, 700], 3, seed=809, with_h0=True)
+    inp.g = -5.0 * torch.sigmoid(inp.g.float())
+    unit = lambda x: (x.float() / x.float().norm(dim=-1, keepdim=True)).to(torch.bfloat16)
+    inp.q, inp.k = unit(inp.q), unit(inp.k)
+    fe = fe_dict(A_log, dt, flags=4)
+    assert_parity(compare(inp, run_gpu(inp, variant=variant, frontend=fe), frontend=fe))
 
 
 @pytest.mark.parametrize("flags", [1, 2])

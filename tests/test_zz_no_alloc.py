@@ -76,3 +76,52 @@ def test_noalloc_refuses_shapes_beyond_its_area_without_writing():
     assert rc == capi.KDA_ERR_WORKSPACE_TOO_SMALL
     torch.cuda.synchronize()
     assert torch.all(out == 3.0)
+
+
+@pytest.mark.parametrize("variant", [4, 1, 2, 3])   # token, split, fused, hybrid
+def test_noalloc_each_variant_back_to_back_matches_kda_prefill(variant):
+    """The variants lay the shared area out differently (the fused and hybrid ones
+    rely on ready flags cleared by every call): two calls in a row per variant, each
+    compared with kda_prefill on its own workspace."""
+    import kda_chunked_recurrent_b200 as K
+    from kda_chunked_recurrent_b200 import capi
+    inp = make_inputs([200, 65, 0, 131], 2, seed=40 + variant, with_h0=True, with_ckpt=True)
+    d = to_dev(inp)
+    N, T, H = inp.num_seqs, inp.total_tokens, inp.num_heads
+    ref_o, ref_ht, ref_ck = K.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], inp.scale,
+                                      h0=d["h0"], cu_seqlens=d["cu_seqlens"],
+                                      ckpt_offsets=d["ckpt_offsets"], variant=variant)
+    torch.cuda.synchronize()
+    f = _noalloc_fn()
+    shape = capi.make_shape(N, T, H, max(inp.seqlens))
+    opts = capi.kda_options_t()
+    opts.variant = variant
+    stream = torch.cuda.current_stream().cuda_stream
+    for _ in range(2):
+        out = torch.zeros(T, H, 128, dtype=torch.bfloat16, device="cuda")
+        ht = torch.zeros(N, H, 128, 128, dtype=torch.float32, device="cuda")
+        ck = torch.zeros(N, H, 128, 128, dtype=torch.float32, device="cuda")
+        rc = f(_p(d["q"]), _p(d["k"]), _p(d["v"]), _p(d["g"]), _p(d["beta"]), inp.scale,
+               _p(d["h0"]), _p(d["cu_seqlens"]), ctypes.byref(shape), _p(out), _p(ht), _p(ck),
+               _p(d["ckpt_offsets"]), ctypes.byref(opts), stream)
+        assert rc == 0, capi.kda_status_string(rc)
+        torch.cuda.synchronize()
+        assert (out.float() - ref_o.float()).abs().max().item() <= O_TOL
+        for a, b in ((ht, ref_ht), (ck, ref_ck)):
+            num = (a - b).flatten(2).norm(dim=-1)
+            den = b.flatten(2).norm(dim=-1).clamp_min(1e-30)
+            assert (num / den).max().item() <= S_TOL
+
+
+def test_noalloc_refuses_status_word_modes():
+    from kda_chunked_recurrent_b200 import capi
+    f = _noalloc_fn()
+    shape = capi.make_shape(1, 64, 1)
+    x = torch.zeros(64 * 128 * 2, device="cuda")
+    for flag in (1, 2):   # KDA_FLAG_VALIDATE, KDA_FLAG_TEST_FORCE_TIMEOUT
+        opts = capi.kda_options_t()
+        opts.flags = flag
+        rc = f(x.data_ptr(), x.data_ptr(), x.data_ptr(), x.data_ptr(), x.data_ptr(), 0.1, None,
+               None, ctypes.byref(shape), x.data_ptr(), None, None, None, ctypes.byref(opts),
+               torch.cuda.current_stream().cuda_stream)
+        assert rc == capi.KDA_ERR_BAD_OPTION
