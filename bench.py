@@ -612,6 +612,14 @@ def main():
             token_kernel_name(capi, N, H): (prep_ms + rec_ms, path_b * units + state_io,
                                             path_b * units + state_io, TOKEN_SOURCES),
         }
+    elif variant == "stream":
+        # one launch: prepare CTAs and recurrence CTAs side by side, records through L2
+        kernels = {
+            "kda_stream_kernel": (prep_ms + rec_ms, path_b * units + state_io,
+                                  (prep_b + REC_BYTES_PER_TOKHEAD) * units + state_io,
+                                  ["kda_stream.cu", "kda_chain.cuh", "kda_prepare.cuh",
+                                   "kda_common.cuh", "sm100_primitives.cuh"]),
+        }
     elif variant == "fused":
         # one launch moves both halves' bytes (the records still go through HBM/L2)
         kernels = {

@@ -106,12 +106,14 @@ typedef enum {
                             no chunk records, workspace = header only.  AUTO picks it when
                             max_seqlen (else T_total) is at most 16, or at most 32 with
                             N*H <= 16.                                                   */
-  KDA_VARIANT_STREAM = 5  /* one cooperative launch of two CTAs per SM: one recurrence CTA
-                            per (sequence, head) (state with the key channel on the tensor-
-                            memory lanes, 256 columns) and prepare CTAs on every other slot,
-                            beside the recurrences on the same SMs; records reach the
-                            recurrence through L2 and are dropped from it once read.  Needs
-                            N*H + 16 <= 2 x SM count, else KDA_ERR_BAD_OPTION.           */
+  KDA_VARIANT_STREAM = 5  /* one cooperative launch of one 512-thread CTA per SM: on CTA
+                            b < N*H one half carries the recurrence of (sequence, head) b
+                            (state with the key channel on the tensor-memory lanes) and the
+                            other half a prepare group; the other CTAs run two prepare
+                            groups, so prepare work runs on every SM beside the
+                            recurrences; records reach the recurrence through L2 and are
+                            dropped from it once read.  Needs N*H <= SM count, else
+                            KDA_ERR_BAD_OPTION.                                            */
 } kda_variant_t;
 
 enum {

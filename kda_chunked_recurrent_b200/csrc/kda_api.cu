@@ -220,12 +220,11 @@ bool fused_eligible(const kda_shape_t* s) {
   return chains + kFusedMinPrepCtas <= sm_count();
 }
 
-// The stream launch holds two CTAs per SM: one recurrence CTA per chain and prepare
-// CTAs on every other slot, at least kFusedMinPrepCtas of them.
-constexpr int kStreamCtasPerSm = 2;
+// The stream launch holds one CTA per SM; a chain takes half of one CTA, so at most one
+// chain per SM, and every half without a chain runs a prepare group.
 bool stream_eligible(const kda_shape_t* s) {
   const int64_t chains = static_cast<int64_t>(s->num_seqs) * s->num_heads;
-  return chains + kFusedMinPrepCtas <= kStreamCtasPerSm * static_cast<int64_t>(sm_count());
+  return chains <= static_cast<int64_t>(sm_count());
 }
 
 int64_t max_chunks_per_seq(const kda_shape_t* s, bool fixed, bool ckpt);
@@ -413,12 +412,11 @@ kda_status_t kda_prefill_describe(const kda_shape_t* shape, int has_ckpt,
              fused::kThreadsPerCta, chains, static_cast<long long>(sm_count()) - chains,
              r.lay.total);
   } else if (r.variant == KDA_VARIANT_STREAM) {
-    const long long grid = static_cast<long long>(kStreamCtasPerSm) * sm_count();
+    const long long grid = sm_count();
     snprintf(buf, n,
-             "variant=stream chunk=%d grid=%lldx%d (recurrence CTAs %lld, prepare CTAs %lld, "
-             "%d CTAs per SM, cooperative) workspace_bytes=%zu",
-             kC, grid, stream::kThreadsPerCta, chains, grid - chains, kStreamCtasPerSm,
-             r.lay.total);
+             "variant=stream chunk=%d grid=%lldx%d (recurrences %lld, prepare groups %lld, "
+             "one CTA per SM, cooperative) workspace_bytes=%zu",
+             kC, grid, stream::kThreadsPerCta, chains, 2 * grid - chains, r.lay.total);
   } else if (r.variant == KDA_VARIANT_FUSED) {
     snprintf(buf, n,
              "variant=fused chunk=%d grid=%dx%d (recurrence CTAs %lld, prepare CTAs %lld, "
@@ -556,6 +554,7 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
     mok &= make_map_rows(&maps.o_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, out, T, H, 2);
     if (r.variant == KDA_VARIANT_STREAM) {
       mok &= make_map_2d(&maps.qw, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws + r.lay.qw, 128, recs * 128, 64, 128, 2);
+      mok &= make_map_2d(&maps.u, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws + r.lay.u, 128, recs * 64, 64, 64, 2);
     } else {
       mok &= make_map_2d(&maps.wt, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws + r.lay.wt, 64, recs * 128, 64, 128, 2);
       mok &= make_map_2d(&maps.qg, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws + r.lay.qg, 128, recs * 64, 64, 64, 2);
@@ -592,7 +591,14 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
     cudaError_t e7 = cudaFuncSetAttribute(kda_stream_fe_kernel,
                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           stream::kSmemAllocBytes);
-    const cudaError_t es[] = {e1, e2, e3, e4, e5, e6, e7};
+    // the stream CTA's two halves (about 217 KB) need the largest shared-memory carveout
+    cudaError_t e8 = cudaFuncSetAttribute(kda_stream_kernel,
+                                          cudaFuncAttributePreferredSharedMemoryCarveout,
+                                          cudaSharedmemCarveoutMaxShared);
+    cudaError_t e9 = cudaFuncSetAttribute(kda_stream_fe_kernel,
+                                          cudaFuncAttributePreferredSharedMemoryCarveout,
+                                          cudaSharedmemCarveoutMaxShared);
+    const cudaError_t es[] = {e1, e2, e3, e4, e5, e6, e7, e8, e9};
     for (cudaError_t e : es)
       if (attr_err == cudaSuccess) attr_err = e;
   });
@@ -652,16 +658,16 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
                                                       stream::kSmemAllocBytes) != cudaSuccess ||
         per_sm < 1)
       return KDA_ERR_LAUNCH_FAILED;
-    per_sm = std::min(per_sm, kStreamCtasPerSm);
     int32_t rec_ctas = static_cast<int32_t>(N * H);
-    const int64_t grid = static_cast<int64_t>(per_sm) * sm_count();
-    if (rec_ctas + kFusedMinPrepCtas > grid) return KDA_ERR_BAD_OPTION;
+    const int64_t grid = sm_count();
+    if (rec_ctas > grid) return KDA_ERR_BAD_OPTION;
     const int64_t jmax = max_chunks_per_seq(shape, fixed, ckpt);
     int64_t prep_items = jmax * static_cast<int64_t>(rec_ctas);
+    // ready flags and the item counter the prepare CTAs claim from, cleared every call
     if (r.lay.slots > 0 &&
-        cudaMemsetAsync(ws + r.lay.ready, 0, static_cast<size_t>(r.lay.slots) * H * sizeof(int32_t),
-                        s) != cudaSuccess)
+        cudaMemsetAsync(ws + r.lay.ready, 0, r.lay.claim + 8 - r.lay.ready, s) != cudaSuccess)
       return KDA_ERR_LAUNCH_FAILED;
+    p.claim_items = 1;
     void* args[] = {&p, &maps, &rec_ctas, &prep_items};
     if (cudaLaunchCooperativeKernel(fn, dim3(static_cast<unsigned>(grid)),
                                     dim3(stream::kThreadsPerCta), args, stream::kSmemAllocBytes,

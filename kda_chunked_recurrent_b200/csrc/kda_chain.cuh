@@ -1,6 +1,6 @@
-// kda_chain.cuh — the inter-chunk recurrence of the stream variant (one CTA of 256
-// threads per (sequence, head), sized so that a prepare CTA fits beside it on the
-// same SM: 256 tensor-memory columns and about 104 KB of shared memory).
+// kda_chain.cuh — the inter-chunk recurrence of the stream variant (256 threads per
+// (sequence, head), half of a CTA whose other half runs a prepare group on the same
+// SM: 256 tensor-memory columns and 104 KB of shared memory).
 //
 // The state S [k][v] (key channel k on TMEM lane k, value channel v on column v)
 // stays in tensor memory from chunk to chunk.  Per chunk of c <= 64 tokens, with the
@@ -25,15 +25,18 @@
 // .. + 63, so thread (L = lane, h = w / 4) owns S row L, and PQ row L, on that column
 // half.  Warps 0, 1, 4, 5 (PQ lanes 0..63) drain and store the output; warps 2, 3, 6, 7
 // (PQ lanes 64..127) form Ud.  Thread 64 (warp 2, lane 0) issues every UMMA; thread 32
-// (warp 1, lane 0) acquires each record's ready flag and issues its TMA copies.
+// (warp 1, lane 0) acquires the records' ready flags and issues their TMA copies.
 //
 // Per chunk j: [B] every thread waits for S(j) (the previous update), loads its S row
 // half, writes S0 into shared memory and the Gamma-scaled S back into tensor memory;
-// the output warps also drain O(j - 1).  [C] CTA barrier; the issuer starts P.  [D]
-// the Ud warps wait for P and write Ud; the output warps store O(j - 1).  [E] barrier
-// of the Ud warps; the issuer starts the update and O, with separate commits for S
-// and for O.  Every wait is bounded; a failure is ORed across each barrier's
-// participants (bar.red.or) so that all of them leave together.
+// the output warps also drain and store O(j - 1).  [C] barrier of the 256 threads; the
+// issuer starts P; the Ud warps load their U rows of chunk j.  [D] the Ud warps wait
+// for P and write Ud; the producer brings chunk j + 1's A tile and acquires record
+// j + 2 (two chunks ahead, off the chain).  [E] barrier of the Ud warps; the issuer
+// starts the update and O, with separate commits for S and for O.  No register array
+// lives across a barrier (spilled registers would put L2 round trips on the chain).
+// Every wait is bounded; a failure is ORed across each barrier's participants
+// (bar.red.or) so that all of them leave together.
 //
 // The records are consumed from L2 soon after the prepare CTAs of the same launch made
 // them.  Once a record has been read it is dropped from L2 without a write-back
@@ -55,19 +58,20 @@ namespace kda {
 namespace chain {
 constexpr int kThreads = 256;
 constexpr uint32_t kA = 0;          // 32 KB [Q Gamma; W] f16, K-major A of P: 2 panels [128 rows][64 k]
-constexpr uint32_t kKd = 32768;     // 16 KB Kd [64 r][128 k] f16, MN-major A of the update: 2 panels [64 r][64 k]
-constexpr uint32_t kAqk = 49152;    //  8 KB Aqk [64 r][64 s] f16, K-major A of O (its rows 64..127 read
-                                    //        the next 8 KB, which only feed PQ lanes no one reads)
+constexpr uint32_t kAqk = 32768;    //  8 KB Aqk [64 r][64 s] f16, K-major A of O (its rows 64..127 read
+                                    //        the Kd tile after it, only into PQ lanes no one reads)
+constexpr uint32_t kKd = 40960;     // 16 KB Kd [64 r][128 k] f16, MN-major A of the update: 2 panels [64 r][64 k]
 constexpr uint32_t kS0 = 57344;     // 32 KB S0 [128 k][128 v] f16, MN-major B of P: 2 panels [128 k][64 v]
-constexpr uint32_t kUd = 90112;     // 16 KB Ud [64 r][128 v] f16, MN-major B of the update and O
+constexpr uint32_t kUd = 90112;     // 16 KB U, then Ud = U - P_W in place: [64 r][128 v] f16,
+                                    //        MN-major B of the update and O: 2 panels [64 r][64 v]
 constexpr uint32_t kBytes = 106496;
 constexpr uint32_t kSmemAlloc = kBytes + 1024;
-constexpr uint32_t kTxA = 32768, kTxY = 16384 + 8192;
+constexpr uint32_t kTxA = 32768, kTxY = 16384 + 8192 + 16384;
 constexpr uint32_t kColS = 0, kColPQ = 128;
 constexpr int kIssuer = 64;         // warp 2, lane 0
 constexpr int kProducer = 32;       // warp 1, lane 0
 constexpr uint32_t kBarAll = 1, kBarUd = 2;   // named barriers (ids 1, 2)
-static_assert(kUd + 16384 == kBytes, "layout");
+static_assert(kUd + 16384 == kBytes && kKd + 16384 == kS0, "layout");
 }  // namespace chain
 
 // Drop a consumed record's lines from L2 without writing them back (128-byte lines;
@@ -108,14 +112,14 @@ __device__ __forceinline__ bool acquire_record(const KdaParams& p, int64_t rec, 
   }
 }
 
-// The recurrence of one (sequence, head) unit of the stream variant.
+// The recurrence of one (sequence, head) unit of the stream variant, run by threads
+// 0..255 of the CTA.  tbase: 256 tensor-memory columns of the caller's allocation.
 __device__ __forceinline__ void chain_body(const KdaParams& p, const SplitMaps& maps,
-                                           uint8_t* smem_raw, int unit) {
+                                           uint8_t* smem_raw, int unit, uint32_t tbase) {
   using namespace chain;
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
   __shared__ uint64_t fullA_bar, fullY_bar, p_bar, s_bar, o_bar, drain_bar;
-  __shared__ uint32_t tmem_slot;
   __shared__ int32_t s_abort;
   volatile int32_t* abort_flag = &s_abort;
 
@@ -137,6 +141,7 @@ __device__ __forceinline__ void chain_body(const KdaParams& p, const SplitMaps& 
   const uint32_t lane_base = static_cast<uint32_t>(qtr * 32);
   const bool out_warp = qtr < 2;                       // PQ lanes 0..63: output rows
   const int v0 = half * 64;                            // this thread's value columns
+  const int oi = half * 64 + qtr * 32 + lane;          // index among the 128 output threads
 
   if (tid == 0) {
     mbar_init(&fullA_bar, 1);
@@ -148,13 +153,7 @@ __device__ __forceinline__ void chain_body(const KdaParams& p, const SplitMaps& 
     s_abort = 0;
     fence_mbar_init();
   }
-  if (warp == 0) {
-    tmem_alloc(&tmem_slot, 256);
-    tmem_relinquish();
-  }
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tbase = tmem_slot;
+  named_bar_sync(kBarAll, kThreads);
   const uint32_t sbase = smem_u32(sm);
 
   auto rec_of = [&](int j) -> int64_t {   // record index of chunk j, or -1 if out of range
@@ -162,8 +161,16 @@ __device__ __forceinline__ void chain_body(const KdaParams& p, const SplitMaps& 
     if (slot < 0 || slot >= p.slots) return -1;
     return slot * p.H + hd;
   };
-  // producer: TMA of chunk j's A tile, and of its Kd / Aqk tiles
+  // producer: acquire a record's ready flag; TMA of a chunk's A tile and of its Kd / Aqk
   int issuedA = 0, issuedY = 0;
+  auto acquire = [&](int j) -> bool {
+    if (j >= nch) return true;
+    const int64_t r = rec_of(j);
+    if (r < 0) return true;
+    if (!acquire_record(p, r, budget)) return false;
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    return true;
+  };
   auto load_A = [&](int j) {
     const int64_t r = rec_of(j);
     if (r < 0) return;
@@ -179,20 +186,55 @@ __device__ __forceinline__ void chain_body(const KdaParams& p, const SplitMaps& 
     tma_load_2d(sm + kKd, &maps.kd, &fullY_bar, 0, static_cast<int32_t>(r * 64));
     tma_load_2d(sm + kKd + 8192, &maps.kd, &fullY_bar, 64, static_cast<int32_t>(r * 64));
     tma_load_2d(sm + kAqk, &maps.aqk, &fullY_bar, 0, static_cast<int32_t>(r * 64));
+    tma_load_2d(sm + kUd, &maps.u, &fullY_bar, 0, static_cast<int32_t>(r * 64));
+    tma_load_2d(sm + kUd + 8192, &maps.u, &fullY_bar, 64, static_cast<int32_t>(r * 64));
     ++issuedY;
   };
+  auto load_gamma = [&](int j) -> float {   // Gamma_end[L] of chunk j
+    const int64_t r = rec_of(j);
+    return r < 0 ? 1.f
+                 : ldg_cg_f32(reinterpret_cast<const float*>(p.ws + p.lay.gc + static_cast<size_t>(r) * kTileGC) + L);
+  };
+  auto discard_record = [&](int j) {        // the 128 output threads drop a read record from L2
+    const int64_t rp = rec_of(j);
+    if (rp < 0) return;
+    discard_l2(p.ws + p.lay.qw + static_cast<size_t>(rp) * kTileQW, static_cast<uint32_t>(kTileQW), oi, 128);
+    discard_l2(p.ws + p.lay.u + static_cast<size_t>(rp) * kTileU, static_cast<uint32_t>(kTileU), oi, 128);
+    discard_l2(p.ws + p.lay.kd + static_cast<size_t>(rp) * kTileKd, static_cast<uint32_t>(kTileKd), oi, 128);
+    discard_l2(p.ws + p.lay.aqk + static_cast<size_t>(rp) * kTileAqk, static_cast<uint32_t>(kTileAqk), oi, 128);
+  };
+  // an output thread's O row half: scale, round to BF16, store (rows past the chunk skipped)
+  auto drain_out = [&](int32_t ot0, int32_t oc) {
+#pragma unroll
+    for (int part = 0; part < 2; ++part) {
+      uint32_t a[32];
+      tmem_ld32(tmem_addr(tbase, lane_base, kColPQ + v0 + part * 32), a);
+      tmem_wait_ld();
+      if (L < oc) {
+        uint4* dst = reinterpret_cast<uint4*>(
+            p.out + (static_cast<int64_t>(si.start + ot0 + L) * p.H + hd) * kD + v0 + part * 32);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          dst[i] = make_uint4(pack_bf16(p.scale * __uint_as_float(a[8 * i]), p.scale * __uint_as_float(a[8 * i + 1])),
+                              pack_bf16(p.scale * __uint_as_float(a[8 * i + 2]), p.scale * __uint_as_float(a[8 * i + 3])),
+                              pack_bf16(p.scale * __uint_as_float(a[8 * i + 4]), p.scale * __uint_as_float(a[8 * i + 5])),
+                              pack_bf16(p.scale * __uint_as_float(a[8 * i + 6]), p.scale * __uint_as_float(a[8 * i + 7])));
+      }
+    }
+  };
 
+  // producer: records 0 and 1 ready, chunk 0's tiles on their way
   bool ok = true;
   if (tid == kProducer && nch > 0) {
     prefetch_tmap(&maps.qw);
     prefetch_tmap(&maps.kd);
     prefetch_tmap(&maps.aqk);
-    const int64_t r0 = rec_of(0);
-    ok = r0 >= 0 && acquire_record(p, r0, budget);
+    prefetch_tmap(&maps.u);
+    ok = acquire(0);
     if (ok) {
-      asm volatile("fence.proxy.async.global;" ::: "memory");
       load_A(0);
       load_Y(0);
+      ok = acquire(1);
     }
   }
 
@@ -218,49 +260,11 @@ __device__ __forceinline__ void chain_body(const KdaParams& p, const SplitMaps& 
     tmem_wait_st();
   }
 
-  // ---- per-chunk registers
-  float gam = 1.f, gam_next = 1.f;   // Gamma_end[k = L] of the current and the next chunk
-  // Ud warps: U[r][v0 .. v0 + 63] of the current chunk (f16 pairs); output warps: the
-  // held O(j - 1) row half (scaled bf16 pairs).  The two roles never meet in one thread.
-  uint32_t hold[32];
-  int32_t o_t0 = 0, o_c = 0;   // token span of the chunk whose O is held
-  bool o_pending = false;
-  // index among the 128 output threads (warps 0, 1, 4, 5)
-  const int oi = half * 64 + qtr * 32 + lane;
-
-  // the producer published record 0; everyone can read its U / Gamma rows after this
+  // records 0 and 1 are visible to every thread after this barrier
   ok = !named_bar_or(kBarAll, kThreads, !ok);
-  auto load_gamma = [&](int j) {   // Gamma_end[L] of chunk j
-    const int64_t r = rec_of(j);
-    if (r >= 0) gam_next = ldg_cg_f32(reinterpret_cast<const float*>(p.ws + p.lay.gc + static_cast<size_t>(r) * kTileGC) + L);
-  };
-  auto load_u = [&](int j) {       // a Ud thread's U row half of chunk j
-    const int64_t r = rec_of(j);
-    if (r < 0) return;
-    const uint8_t* u = p.ws + p.lay.u + static_cast<size_t>(r) * kTileU +
-                       static_cast<size_t>(L - 64) * 256 + v0 * 2;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const uint4 x = ldg_cg_v4(u + 16 * i);
-      hold[4 * i + 0] = x.x;
-      hold[4 * i + 1] = x.y;
-      hold[4 * i + 2] = x.z;
-      hold[4 * i + 3] = x.w;
-    }
-  };
-  if (ok && nch > 0) {
-    load_gamma(0);
-    if (!out_warp) load_u(0);
-  }
-  // the 128 output threads drop a fully read record from L2
-  auto discard_record = [&](int j) {
-    const int64_t rp = rec_of(j);
-    if (rp < 0) return;
-    discard_l2(p.ws + p.lay.qw + static_cast<size_t>(rp) * kTileQW, static_cast<uint32_t>(kTileQW), oi, 128);
-    discard_l2(p.ws + p.lay.u + static_cast<size_t>(rp) * kTileU, static_cast<uint32_t>(kTileU), oi, 128);
-    discard_l2(p.ws + p.lay.kd + static_cast<size_t>(rp) * kTileKd, static_cast<uint32_t>(kTileKd), oi, 128);
-    discard_l2(p.ws + p.lay.aqk + static_cast<size_t>(rp) * kTileAqk, static_cast<uint32_t>(kTileAqk), oi, 128);
-  };
+  float gam = 1.f, gam_next = 1.f;   // Gamma_end[k = L] of the current / next chunk
+  if (ok && nch > 0) gam_next = load_gamma(0);
+  int32_t o_t0 = 0, o_c = 0;          // token span of the chunk whose O is in PQ
 
   for (int j = 0; j < nch && ok; ++j) {
     int32_t t0, c;
@@ -271,10 +275,10 @@ __device__ __forceinline__ void chain_body(const KdaParams& p, const SplitMaps& 
     ok = __all_sync(0xffffffffu, ok);   // tcgen05.ld / st below are warp-collective
     tc_fence_after();
     if (ok) {
-      // in two parts of 32 columns (register budget)
       const uint32_t srow = sbase + kS0 + static_cast<uint32_t>(half) * 16384u;
       const bool ck_here = ckr && si.nA > 0 && j == si.nA;
-#pragma unroll
+      // (one part at a time: unrolled, the two parts' 64 live values spill)
+#pragma unroll 1
       for (int part = 0; part < 2; ++part) {
         uint32_t a[32];
         tmem_ld32(tmem_addr(tbase, lane_base, kColS + v0 + part * 32), a);
@@ -304,41 +308,22 @@ __device__ __forceinline__ void chain_body(const KdaParams& p, const SplitMaps& 
         tmem_st32(tmem_addr(tbase, lane_base, kColS + v0 + part * 32), a);
       }
     }
-    // output warps: drain O(j - 1) from PQ lanes 0..63 before P(j) overwrites them;
-    // the producer (one of them) then brings chunk j's Kd / Aqk tiles, whose previous
-    // readers (update and O of chunk j - 1) are complete
+    // output warps: drain and store O(j - 1) (PQ lanes 0..63) before P(j) overwrites it;
+    // the producer then brings chunk j's Kd / Aqk, whose last readers (update and O of
+    // chunk j - 1) are complete
     if (out_warp && j > 0) {
       ok = ok && mbar_wait(&o_bar, static_cast<uint32_t>((j - 1) & 1), budget) && !*abort_flag;
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
       if (ok) {
         if (tid == kProducer) load_Y(j);
-#pragma unroll
-        for (int part = 0; part < 2; ++part) {
-          uint32_t a[32];
-          tmem_ld32(tmem_addr(tbase, lane_base, kColPQ + v0 + part * 32), a);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 16; ++i)
-            hold[part * 16 + i] = pack_bf16(p.scale * __uint_as_float(a[2 * i]),
-                                            p.scale * __uint_as_float(a[2 * i + 1]));
-        }
-        o_pending = true;
-      }
-    }
-    // producer: the next record must be ready before this chunk starts, so that every
-    // thread may read its U / Gamma rows after the barrier below
-    if (tid == kProducer && ok && j + 1 < nch) {
-      const int64_t rn = rec_of(j + 1);
-      if (rn >= 0) {
-        ok = acquire_record(p, rn, budget);
-        if (ok) asm volatile("fence.proxy.async.global;" ::: "memory");
+        drain_out(o_t0, o_c);
       }
     }
     tmem_wait_st();
     fence_proxy_async_smem();
     tc_fence_before();
-    // ===== [C] S0 and the scaled S are in place; record j + 1 is visible
+    // ===== [C] S0 and the scaled S are in place
     ok = !named_bar_or(kBarAll, kThreads, !ok || *abort_flag);
     if (!ok) break;
     if (tid == kIssuer) {
@@ -351,37 +336,35 @@ __device__ __forceinline__ void chain_body(const KdaParams& p, const SplitMaps& 
           umma_f16(tbase + kColPQ, sdesc_sw128(sbase + kA + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
                    sdesc_sw128(sbase + kS0 + kk * 2048, 16384, 1024), idesc, kk > 0);
         umma_commit(&p_bar);
+      } else {
+        *abort_flag = 1;
       }
     }
-    if (j + 1 < nch) load_gamma(j + 1);
+    // the next chunk's Gamma_end (record j + 1 was acquired two chunks ago)
+    if (j + 1 < nch) gam_next = load_gamma(j + 1);
+    o_t0 = t0;
+    o_c = c;
     // ===== [D]
     if (out_warp) {
-      // store O(j - 1): row r = L of that chunk, 64 values = 128 bytes
-      if (o_pending) {
-        if (L < o_c) {
-          uint4* dst = reinterpret_cast<uint4*>(p.out + (static_cast<int64_t>(si.start + o_t0 + L) * p.H + hd) * kD + v0);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) dst[i] = make_uint4(hold[4 * i], hold[4 * i + 1], hold[4 * i + 2], hold[4 * i + 3]);
-        }
-        o_pending = false;
-      }
       if (tid == kProducer && ok) {
-        // the A tile is free once P(j) has completed: bring chunk j + 1's
+        // the A tile is free once P(j) has completed: bring chunk j + 1's; then make sure
+        // record j + 2 is ready, two chunks before it is needed
         if (mbar_wait(&p_bar, static_cast<uint32_t>(j & 1), budget)) {
           if (j + 1 < nch) load_A(j + 1);
+          ok = acquire(j + 2);
         } else {
           ok = false;
         }
+        if (!ok) *abort_flag = 1;
       }
-      // the previous record is fully read: U / Gamma rows (loaded a chunk ago) and its
-      // tiles (whose last readers, update and O of chunk j - 1, completed before the
-      // drain above); drop it from L2
+      // the previous record is fully read (its last readers, update and O of chunk
+      // j - 1, completed before the drain above): drop it from L2
       if (j > 0 && ok) discard_record(j - 1);
-      o_t0 = t0;
-      o_c = c;
     } else {
-      // Ud = U - P_W: row r = L - 64, value columns v0 .. v0 + 63, FP16 into the B tile
+      // Ud = U - P_W in place in the B tile: row r = L - 64, value columns v0 .. v0 + 63
+      // (U arrived with chunk j's Kd / Aqk tiles)
       ok = ok && mbar_wait(&p_bar, static_cast<uint32_t>(j & 1), budget) && !*abort_flag;
+      ok = ok && mbar_wait(&fullY_bar, static_cast<uint32_t>(j & 1), budget) && !*abort_flag;
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
       if (ok) {
@@ -394,16 +377,19 @@ __device__ __forceinline__ void chain_body(const KdaParams& p, const SplitMaps& 
           tmem_wait_ld();
 #pragma unroll
           for (int c4 = 0; c4 < 4; ++c4) {
-            const int ch = part * 4 + c4;
+            const uint32_t addr = urow + sw128_offset(r, static_cast<uint32_t>(part * 4 + c4));
+            uint32_t uw[4];
+            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(uw[0]), "=r"(uw[1]), "=r"(uw[2]), "=r"(uw[3])
+                         : "r"(addr));
             uint32_t w[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const float2 uf = __half22float2(*reinterpret_cast<const __half2*>(&hold[ch * 4 + e]));
+              const float2 uf = __half22float2(*reinterpret_cast<const __half2*>(&uw[e]));
               w[e] = pack_f16(uf.x - __uint_as_float(a[c4 * 8 + 2 * e]),
                               uf.y - __uint_as_float(a[c4 * 8 + 2 * e + 1]));
             }
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
-                             urow + sw128_offset(r, static_cast<uint32_t>(ch))),
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
                          "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
                          : "memory");
           }
@@ -429,11 +415,10 @@ __device__ __forceinline__ void chain_body(const KdaParams& p, const SplitMaps& 
             umma_f16(tbase + kColPQ, sdesc_sw128(sbase + kAqk + kk * 32, 16, 1024),
                      sdesc_sw128(sbase + kUd + kk * 2048, 8192, 1024), id_o, 1);
           umma_commit(&o_bar);
+        } else {
+          *abort_flag = 1;
         }
       }
-      if (tid == kIssuer && !ok) *abort_flag = 1;
-      // the next chunk's U row (record j + 1 was acquired before barrier [C])
-      if (ok && j + 1 < nch) load_u(j + 1);
     }
   }
 
@@ -445,22 +430,7 @@ __device__ __forceinline__ void chain_body(const KdaParams& p, const SplitMaps& 
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
       if (ok) {
-#pragma unroll
-        for (int part = 0; part < 2; ++part) {
-          uint32_t a[32];
-          tmem_ld32(tmem_addr(tbase, lane_base, kColPQ + v0 + part * 32), a);
-          tmem_wait_ld();
-          if (L < o_c) {
-            uint4* dst = reinterpret_cast<uint4*>(
-                p.out + (static_cast<int64_t>(si.start + o_t0 + L) * p.H + hd) * kD + v0 + part * 32);
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-              dst[i] = make_uint4(pack_bf16(p.scale * __uint_as_float(a[8 * i]), p.scale * __uint_as_float(a[8 * i + 1])),
-                                  pack_bf16(p.scale * __uint_as_float(a[8 * i + 2]), p.scale * __uint_as_float(a[8 * i + 3])),
-                                  pack_bf16(p.scale * __uint_as_float(a[8 * i + 4]), p.scale * __uint_as_float(a[8 * i + 5])),
-                                  pack_bf16(p.scale * __uint_as_float(a[8 * i + 6]), p.scale * __uint_as_float(a[8 * i + 7])));
-          }
-        }
+        drain_out(o_t0, o_c);
         discard_record(nch - 1);
       }
     }
@@ -502,7 +472,8 @@ __device__ __forceinline__ void chain_body(const KdaParams& p, const SplitMaps& 
     record_status(p.ws, kStatusTimeout);
   }
 
-  // ---- teardown: every TMA copy and UMMA this CTA issued completes before exit
+  // ---- teardown: every TMA copy and UMMA of this unit completes before the caller frees
+  // tensor memory or the CTA exits
   if (tid == kProducer) {
     if (issuedA > 0) mbar_wait(&fullA_bar, static_cast<uint32_t>((issuedA - 1) & 1), drain_budget);
     if (issuedY > 0) mbar_wait(&fullY_bar, static_cast<uint32_t>((issuedY - 1) & 1), drain_budget);
@@ -512,8 +483,7 @@ __device__ __forceinline__ void chain_body(const KdaParams& p, const SplitMaps& 
     mbar_wait(&drain_bar, 0, drain_budget);
   }
   tc_fence_before();
-  __syncthreads();
-  if (warp == 0) tmem_dealloc(tbase, 256);
+  named_bar_sync(kBarAll, kThreads);
 }
 
 }  // namespace kda

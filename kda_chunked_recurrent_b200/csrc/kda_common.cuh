@@ -49,6 +49,7 @@ struct WorkspaceLayout {
   size_t wt, qg, ut, kd, aqk, gc;     // per-record tiles
   size_t qw, u;                       // per-record tiles of the stream variant
   size_t ready;        // int32 [recs]  per-record ready flags (fused variant)
+  size_t claim;        // u64           next item to claim (stream variant); cleared with the flags
   size_t total;
   int64_t slots;       // chunk slots (upper bound on the number of chunks)
 };
@@ -87,7 +88,8 @@ inline WorkspaceLayout make_layout(int64_t N, int64_t T, int64_t H, bool fixed, 
   L.kd = off;  off = align_up(off + recs * kTileKd, 1024);
   L.aqk = off; off = align_up(off + recs * kTileAqk, 1024);
   L.gc = off;  off = align_up(off + recs * kTileGC, 1024);
-  L.ready = off; off = align_up(off + recs * sizeof(int32_t), 1024);
+  L.ready = off; off += recs * sizeof(int32_t);
+  L.claim = align_up(off, 8); off = align_up(L.claim + 8, 1024);
   L.total = off;
   return L;
 }
@@ -128,6 +130,7 @@ struct KdaParams {
   uint8_t* ws;
   WorkspaceLayout lay;
   uint32_t flags;
+  uint32_t claim_items;          // prepare CTAs claim items from the counter at lay.claim
   long long wait_budget;         // clock cycles per bounded wait; < 0 forces a timeout
   // input front end (0: inputs used as given; bit 0 q/k L2 norm, bit 1 gate from the
   // raw BF16 gate in g, bit 2 beta from its logit), formed in FP32 by the prepare kernel
@@ -151,6 +154,7 @@ struct SplitMaps {
   CUtensorMap kd;       // [recs*64][128] f16, box (64, 64)
   CUtensorMap aqk;      // [recs*64][64] f16, box (64, 64)
   CUtensorMap qw;       // stream: [recs*128][128] f16, box (64, 128): one 64-channel panel
+  CUtensorMap u;        // stream: [recs*64][128] f16, box (64, 64): one 64-channel panel
 };
 
 enum : int32_t {

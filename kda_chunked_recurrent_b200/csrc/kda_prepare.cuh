@@ -44,11 +44,11 @@
 // yields A (strict lower part) and Aqk (lower part with the diagonal).
 //
 // UT solve: T = (I + M)^-1 with M = diag(beta) A_strict, in 16x16 blocks.  The
-// diagonal blocks X_ii are inverted in FP32 by forward substitution; then
-// Z_ik = -X_ii M_ik for all i > k in one step, and the off-diagonal blocks
-// follow level by level, X_ij = sum_{k=j}^{i-1} Z_ik X_kj, as FP16 mma.sync
-// products with FP32 accumulation.  Each block of T diag(beta), the B operand
-// of the W/U UMMA, is written from the accumulator as soon as it is final.
+// diagonal blocks X_ii are inverted in FP32 by right-looking forward substitution;
+// then each of three warps walks one block column down, X_ij = -X_ii (sum_{k=j}^{i-1}
+// M_ik X_kj), as FP16 mma.sync products with FP32 accumulation.  Each block of
+// T diag(beta), the operand of the W/U UMMA, is written from the accumulator as soon
+// as it is final.
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -79,10 +79,11 @@ constexpr int kGThread = 224;
 // aliases of [K+; Q+] once the first UMMA has completed: the solve scratch, and
 // after the solve the staging tiles of the W^T / U^T TMA stores
 constexpr int kLdh = 72;
-constexpr uint32_t kMf = kL;                    // f32 [4][16][17] diagonal blocks of M
-constexpr uint32_t kMh = kMf + 4 * 16 * 17 * 4; // f16 [64][72] off-diagonal blocks of M
+constexpr int kMfBlk = 272;                     // floats per diagonal block of Mf (16 x 16 + 16 pad)
+constexpr uint32_t kMf = kL;                    // f32 [4][16 s][16 r] diagonal blocks of M, column-major
+constexpr uint32_t kMh = kMf + 4 * kMfBlk * 4;  // f16 [64][72] off-diagonal blocks of M
 constexpr uint32_t kXh = kMh + 64 * kLdh * 2;   // f16 [64][72] T = (I + M)^-1
-constexpr uint32_t kZh = kXh + 64 * kLdh * 2;   // f16 [64][72] Z_ik = -X_ii M_ik
+constexpr uint32_t kWk = kXh + 64 * kLdh * 2;   // f16 [3][16][72] one 16x16 scratch block per solve warp
 constexpr uint32_t kWs = kL;                    // W^T staging [128 k][64 tok] f16, 128B swizzle
 constexpr uint32_t kUs = kL + 16384;            // U^T staging [128 v][64 tok] f16, 128B swizzle
 // aliases of R once the first UMMA has completed
@@ -96,9 +97,10 @@ constexpr uint32_t kAuxBeta = kAux + 64;         // f32 [64]
 constexpr uint32_t kAuxTot = kAuxBeta + 256;     // float2 [4][64]
 constexpr uint32_t kAuxFirst = kAuxTot + 2048;   // float2 [4][64]
 constexpr uint32_t kAuxNorm = kAuxFirst + 2048;  // f32 [2][64] inverse norms of k, q rows (front end)
-constexpr uint32_t kGroupBytes = (kAuxNorm + 512 + 1023) / 1024 * 1024;   // one prepare group
+constexpr uint32_t kAuxClaim = kAuxNorm + 512;   // i64 [2] claimed item indices (stream launch)
+constexpr uint32_t kGroupBytes = (kAuxClaim + 16 + 1023) / 1024 * 1024;   // one prepare group
 constexpr uint32_t kSmemAlloc = kGroupBytes + 1024;
-static_assert(kZh + 64 * kLdh * 2 <= kR, "solve scratch overlaps the Aqk staging tile");
+static_assert(kWk + 3 * 16 * kLdh * 2 <= kR, "solve scratch overlaps the Aqk staging tile");
 static_assert(kAqs + 8192 <= kTb, "Aqk staging overlaps the Tb tile");
 static_assert(kUs + 16384 <= kR, "W/U staging overlaps R");
 }  // namespace prep
@@ -195,10 +197,11 @@ __device__ __forceinline__ void emit_rows(const uint32_t* val, bool is_q, int rl
   using namespace prep;
   constexpr int NV = 16 * (BL + 1);
   if (!is_q) {
-    float* Mf = reinterpret_cast<float*>(sm + kMf) + BL * (16 * 17) + (rl & 15) * 17;
+    // diagonal block, column-major (entry (r, s) at s * 16 + r) for the column solve
+    float* Mf = reinterpret_cast<float*>(sm + kMf) + BL * kMfBlk + (rl & 15);
 #pragma unroll
     for (int s = 16 * BL; s < 16 * BL + 16; ++s)
-      Mf[s & 15] = (s < rl) ? br * __uint_as_float(val[s]) : 0.f;
+      Mf[(s & 15) * 16] = (s < rl) ? br * __uint_as_float(val[s]) : 0.f;
     __half* Mh = reinterpret_cast<__half*>(sm + kMh) + rl * kLdh;
 #pragma unroll
     for (int s0 = 0; s0 < 16 * BL; s0 += 8) {
@@ -294,17 +297,26 @@ __device__ __forceinline__ bool locate_item_chunk_major(const KdaParams& p, int6
 }
 
 // Group-wide barriers of the prepare body: the whole CTA in the split kernel; in a
-// prepare CTA of the fused launch, which runs two independent 256-thread groups,
-// named barrier 1 + grp over the group's threads.
+// CTA of the fused or stream launch, which runs more than one 256-thread group,
+// a named barrier of the group's own (`bar`) over the group's threads.
 template <bool kFused>
-__device__ __forceinline__ void prep_sync(int grp) {
-  if constexpr (kFused) named_bar_sync(1 + grp, prep::kThreads); else __syncthreads();
+__device__ __forceinline__ void prep_sync(uint32_t bar) {
+  if constexpr (kFused) named_bar_sync(bar, prep::kThreads); else __syncthreads();
 }
 template <bool kFused>
-__device__ __forceinline__ bool prep_sync_or(int grp, bool pred) {
-  if constexpr (kFused) return named_bar_or(1 + grp, prep::kThreads, pred);
+__device__ __forceinline__ bool prep_sync_or(uint32_t bar, bool pred) {
+  if constexpr (kFused) return named_bar_or(bar, prep::kThreads, pred);
   else return __syncthreads_or(pred) != 0;
 }
+
+// Where a prepare group's tensor memory and barrier come from: its own 256-column
+// allocation and named barrier 1 + grp (split and fused launches), or a part of the
+// CTA's allocation and a barrier id the caller assigns (stream launch).
+struct PrepGroupRes {
+  uint32_t tmem;   // kTmemOwn: the group allocates its own 256 columns
+  uint32_t bar;    // named barrier id of the group (fused / stream launches)
+};
+constexpr uint32_t kTmemOwn = 0xFFFFFFFFu;
 
 // Publish a finished record to the recurrence CTAs of the fused launch: its tile
 // stores (issued by this thread) are complete and every thread's plain stores
@@ -328,7 +340,8 @@ __device__ __forceinline__ void publish_record(const KdaParams& p, int64_t rec) 
 template <bool kFused, bool kFE = false, bool kStream = false>
 __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps& maps,
                                              uint8_t* smem_raw, int grp, int64_t first,
-                                             int64_t stride, int64_t nitems) {
+                                             int64_t stride, int64_t nitems,
+                                             PrepGroupRes res = PrepGroupRes{kTmemOwn, 0u}) {
   using namespace prep;
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023)) +
@@ -350,6 +363,8 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
 
   const int tid = threadIdx.x - grp * kThreads;
   const int warp = tid >> 5, lane = tid & 31;
+  const uint32_t gbar = res.bar != 0u ? res.bar : 1u + static_cast<uint32_t>(grp);
+  const bool own_tmem = res.tmem == kTmemOwn;
   if ((p.flags & kFlagValidate) && reinterpret_cast<const WsHeader*>(p.ws)->call_ok == 0) return;
   const long long budget = p.wait_budget;
   const long long drain_budget = 4000000000LL;
@@ -368,15 +383,21 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
     prefetch_tmap(&maps.q_in);
     prefetch_tmap(&maps.k_in);
     prefetch_tmap(&maps.g_in);
-    prefetch_tmap(&maps.wt);
-    prefetch_tmap(&maps.ut);
+    if constexpr (!kStream) {   // (the stream records are written without these maps)
+      prefetch_tmap(&maps.wt);
+      prefetch_tmap(&maps.ut);
+    }
     prefetch_tmap(&maps.aqk);
   }
-  if (warp == 0) {
-    tmem_alloc(&tmem_slot, 256);
-    tmem_relinquish();
+  if (own_tmem) {
+    if (warp == 0) {
+      tmem_alloc(&tmem_slot, 256);
+      tmem_relinquish();
+    }
+  } else if (tid == 0) {
+    tmem_slot = res.tmem;
   }
-  prep_sync<kFused>(grp);
+  prep_sync<kFused>(gbar);
   tc_fence_after();
   const uint32_t tbase = tmem_slot;
   const uint32_t sbase = smem_u32(sm);
@@ -396,12 +417,43 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
     tma_load_3d(sm + kGraw, &maps.g_in, &raw_g_bar, 0, it.h, it.t0);
   };
 
+  // Item order.  Static: first, first + stride, ...  Claimed (stream launch): thread 0
+  // takes the next valid item from a counter in the workspace one item ahead and
+  // publishes its index in shared memory; the other threads read it after the first
+  // barrier of the iteration (nothing before that barrier needs it but thread 0).
+  const bool claim = kFused && p.claim_items != 0;
+  int64_t* s_claim = reinterpret_cast<int64_t*>(sm + kAuxClaim);
+  auto claim_next = [&](PrepItem& it) -> int64_t {   // thread 0 only
+    unsigned long long* ctr = reinterpret_cast<unsigned long long*>(p.ws + p.lay.claim);
+    for (;;) {
+      const int64_t w = static_cast<int64_t>(atomicAdd(ctr, 1ull));
+      if (w >= nitems) return nitems;
+      if (locate(w, it)) return w;
+    }
+  };
   PrepItem cur;
-  bool cur_valid = first < nitems && locate(first, cur);
+  int64_t w0 = first;
+  if (claim) {
+    if (tid == 0) s_claim[0] = claim_next(cur);
+    prep_sync<kFused>(gbar);
+    w0 = s_claim[0];
+  }
+  bool cur_valid = w0 < nitems && locate(w0, cur);
   int64_t pending = -1;   // fused launch: record whose ready flag is still to be raised
-  for (int64_t w = first; w < nitems && ok; w += stride) {
+  int iter = 0;
+  for (int64_t w = w0, w_next = 0; w < nitems && ok; w = w_next, ++iter) {
     PrepItem nxt;
-    const bool nxt_valid = (w + stride < nitems) && locate(w + stride, nxt);
+    bool nxt_valid = false;
+    if (claim) {
+      if (tid == 0) {
+        w_next = claim_next(nxt);
+        s_claim[(iter + 1) & 1] = w_next;
+        nxt_valid = w_next < nitems;
+      }
+    } else {
+      w_next = w + stride;
+      nxt_valid = (w_next < nitems) && locate(w_next, nxt);
+    }
     if (!cur_valid) {
       cur = nxt;
       cur_valid = nxt_valid;
@@ -531,8 +583,12 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
     }
     // the previous item's TMA stores have finished reading their staging tiles
     if (tid == 0) bulk_wait_read();
-    ok = !prep_sync_or<kFused>(grp, !ok);
+    ok = !prep_sync_or<kFused>(gbar, !ok);
     if (!ok) break;
+    if (claim && tid != 0) {
+      w_next = s_claim[(iter + 1) & 1];
+      nxt_valid = w_next < nitems && locate(w_next, nxt);
+    }
     // ---- TMA: v tile straight into the MN-major A operand of U^T (the raw q tile
     // in that region has been read by every thread)
     if (tid == 0) {
@@ -649,7 +705,7 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
     // ---- UMMA 1: D[0:128, 0:160] = [K+; Q+] . R^T   (bf16 -> f32)
     fence_proxy_async_smem();
     tc_fence_before();
-    prep_sync<kFused>(grp);
+    prep_sync<kFused>(gbar);
     if (tid == 0) {
       tc_fence_after();
       const uint32_t idesc = idesc_f16(128, 160, kFmtBF16, kKMajor, kKMajor);
@@ -670,7 +726,7 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
     if constexpr (kFused) pending = -1;
     ++mma_commits;
     ok = mbar_wait(&mma_bar, static_cast<uint32_t>((mma_commits - 1) & 1), budget);
-    ok = !prep_sync_or<kFused>(grp, !ok);
+    ok = !prep_sync_or<kFused>(gbar, !ok);
     if (ok) {
       tc_fence_after();
       // ---- extract A (lane quarters 0,1) and Aqk (quarters 2,3): row rl, sub-block bl.
@@ -722,7 +778,7 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
     }
     fence_proxy_async_smem();
     tc_fence_before();
-    prep_sync<kFused>(grp);
+    prep_sync<kFused>(gbar);
     if (ok && tid == kGThread) {
       tma_store_2d(&maps.aqk, sm + kAqs, 0, static_cast<int32_t>(rec * 64));
       bulk_commit();
@@ -740,22 +796,21 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
 
     if (ok) {
       __half* Xh = reinterpret_cast<__half*>(sm + kXh);
-      __half* Zh = reinterpret_cast<__half*>(sm + kZh);
-      const uint32_t aMh = sbase + kMh, aXh = sbase + kXh, aZh = sbase + kZh, aTb = sbase + kTb;
+      const uint32_t aMh = sbase + kMh, aXh = sbase + kXh, aTb = sbase + kTb;
       if (tid < 64) {
-        // ---- diagonal blocks: forward substitution in FP32, one column per thread
+        // ---- diagonal blocks X_bb = (I + M_bb)^-1 in FP32, one column per thread,
+        // right-looking: once x[ss] is final it is folded into every later row, so the
+        // dependent chain is one FMA per row (the later rows' updates are independent)
         const int bi = tid >> 4, jj = tid & 15;
-        const float* Mf = reinterpret_cast<const float*>(sm + kMf) + bi * (16 * 17);
+        const float* Mc = reinterpret_cast<const float*>(sm + kMf) + bi * kMfBlk;   // [s][r]
         float x[16];
 #pragma unroll
-        for (int rr = 0; rr < 16; ++rr) {
-          float acc0 = 0.f, acc1 = 0.f;  // two partial sums halve the dependent chain
+        for (int rr = 0; rr < 16; ++rr) x[rr] = (rr == jj) ? 1.f : 0.f;
 #pragma unroll
-          for (int ss = 0; ss < rr; ss += 2) {
-            acc0 = fmaf(Mf[rr * 17 + ss], x[ss], acc0);
-            if (ss + 1 < rr) acc1 = fmaf(Mf[rr * 17 + ss + 1], x[ss + 1], acc1);
-          }
-          x[rr] = (rr < jj) ? 0.f : (rr == jj ? 1.f : -(acc0 + acc1));
+        for (int ss = 0; ss < 15; ++ss) {
+          const float xs = x[ss];
+#pragma unroll
+          for (int rr = ss + 1; rr < 16; ++rr) x[rr] = fmaf(-Mc[ss * 16 + rr], xs, x[rr]);
         }
         const int col = bi * 16 + jj;
         const float bcol = s_beta[col];
@@ -788,47 +843,36 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
           ok = false;
         }
       }
-      prep_sync<kFused>(grp);
-      // ---- Z_ik = -X_ii M_ik for the six blocks below the diagonal (one warp each)
-      if (warp < 6) {
-        const int zi = (warp < 3) ? warp + 1 : (warp < 5 ? warp - 1 : 3);
-        const int zk = (warp < 3) ? warp : (warp < 5 ? warp - 3 : 0);
-        float z0[4] = {0.f, 0.f, 0.f, 0.f}, z1[4] = {0.f, 0.f, 0.f, 0.f};
-        mma_block(z0, z1, aXh, zi * 16, zi * 16, aMh, zi * 16, zk * 16, lane);
-        store_frag16(Zh + (zi * 16) * kLdh + zk * 16, kLdh, z0, z1, -1.f, lane);
-      }
-      prep_sync<kFused>(grp);
-      // ---- level 1: X_{i,i-1} = Z_{i,i-1} X_{i-1,i-1}
+      prep_sync<kFused>(gbar);
+      // ---- off-diagonal blocks, one block column j per warp, down the column:
+      //   X_ij = -X_ii (sum_{k=j}^{i-1} M_ik X_kj),  i = j+1 .. 3,
+      // FP16 mma.sync with FP32 accumulation.  Column j only reads its own earlier
+      // blocks and the diagonal blocks, so the warps need no barrier between levels.
       if (warp < 3) {
-        const int i = warp + 1, j = warp;
-        float x0[4] = {0.f, 0.f, 0.f, 0.f}, x1[4] = {0.f, 0.f, 0.f, 0.f};
-        mma_block(x0, x1, aZh, i * 16, j * 16, aXh, j * 16, j * 16, lane);
-        store_frag16(Xh + (i * 16) * kLdh + j * 16, kLdh, x0, x1, 1.f, lane);
-        store_tb16(aTb, s_beta, i * 16, j * 16, x0, x1, lane);
-      }
-      prep_sync<kFused>(grp);
-      // ---- level 2: X_20 = Z_20 X_00 + Z_21 X_10, X_31 = Z_31 X_11 + Z_32 X_21,
-      // and the first two terms of X_30 (kept in warp 2's registers)
-      float y0[4] = {0.f, 0.f, 0.f, 0.f}, y1[4] = {0.f, 0.f, 0.f, 0.f};
-      if (warp < 3) {
-        const int i = (warp == 1) ? 3 : 2 + (warp == 2), j = (warp == 1) ? 1 : 0;
-        mma_block(y0, y1, aZh, i * 16, j * 16, aXh, j * 16, j * 16, lane);
-        mma_block(y0, y1, aZh, i * 16, (j + 1) * 16, aXh, (j + 1) * 16, j * 16, lane);
-        if (warp < 2) {
-          store_frag16(Xh + (i * 16) * kLdh + j * 16, kLdh, y0, y1, 1.f, lane);
-          store_tb16(aTb, s_beta, i * 16, j * 16, y0, y1, lane);
+        const int j = warp;
+        __half* wk = reinterpret_cast<__half*>(sm + kWk) + warp * 16 * kLdh;
+        const uint32_t aWk = sbase + kWk + static_cast<uint32_t>(warp * 16 * kLdh * 2);
+        for (int i = j + 1; i < 4; ++i) {
+          float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
+          for (int k = j; k < i; ++k) mma_block(a0, a1, aMh, i * 16, k * 16, aXh, k * 16, j * 16, lane);
+          store_frag16(wk, kLdh, a0, a1, 1.f, lane);
+          __syncwarp();
+          float x0[4] = {0.f, 0.f, 0.f, 0.f}, x1[4] = {0.f, 0.f, 0.f, 0.f};
+          mma_block(x0, x1, aXh, i * 16, i * 16, aWk, 0, 0, lane);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            x0[e] = -x0[e];
+            x1[e] = -x1[e];
+          }
+          store_frag16(Xh + (i * 16) * kLdh + j * 16, kLdh, x0, x1, 1.f, lane);
+          store_tb16(aTb, s_beta, i * 16, j * 16, x0, x1, lane);
+          __syncwarp();
         }
-      }
-      prep_sync<kFused>(grp);
-      // ---- level 3: X_30 += Z_32 X_20
-      if (warp == 2) {
-        mma_block(y0, y1, aZh, 48, 32, aXh, 32, 0, lane);
-        store_tb16(aTb, s_beta, 48, 0, y0, y1, lane);
       }
     }
     fence_proxy_async_smem();
     tc_fence_before();
-    ok = !prep_sync_or<kFused>(grp, !ok);
+    ok = !prep_sync_or<kFused>(gbar, !ok);
 
     // ---- UMMA 2: W^T = (K Gamma)^T (T diag beta)^T -> cols [0,64); U^T = V^T (T diag beta)^T -> [64,128)
     bool tma_seen = false;
@@ -861,12 +905,12 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
       }
     }
     if (tid == 0 && !tma_seen) ok = false;
-    ok = !prep_sync_or<kFused>(grp, !ok);
+    ok = !prep_sync_or<kFused>(gbar, !ok);
     if (ok) {
       ++mma_commits;
       ok = mbar_wait(&mma_bar, static_cast<uint32_t>((mma_commits - 1) & 1), budget);
     }
-    ok = !prep_sync_or<kFused>(grp, !ok);
+    ok = !prep_sync_or<kFused>(gbar, !ok);
     // the next item's q and k tiles go into v / K Gamma, free now that the second
     // UMMA has completed
     if (ok && nxt_valid) {
@@ -936,7 +980,7 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
     }
     fence_proxy_async_smem();
     tc_fence_before();
-    ok = !prep_sync_or<kFused>(grp, !ok);
+    ok = !prep_sync_or<kFused>(gbar, !ok);
     if (ok && tid == 0 && !kStream) {
       tma_store_2d(&maps.wt, sm + kWs, 0, static_cast<int32_t>(rec * 128));
       tma_store_2d(&maps.ut, sm + kUs, 0, static_cast<int32_t>(rec * 128));
@@ -970,8 +1014,8 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
     bulk_wait_all();
   }
   tc_fence_before();
-  prep_sync<kFused>(grp);
-  if (warp == 0) tmem_dealloc(tbase, 256);
+  prep_sync<kFused>(gbar);
+  if (own_tmem && warp == 0) tmem_dealloc(tbase, 256);
 }
 
 }  // namespace kda

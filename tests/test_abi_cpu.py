@@ -54,7 +54,7 @@ def test_describe_reports_grid_and_variant():
     h = capi.kda_prefill_describe(capi.make_shape(8, 65536, 12, 8192), False, {"variant": 3})
     assert "variant=hybrid" in h and "prepare_chunks=" in h and "recurrence CTAs 96" in h
     st = capi.kda_prefill_describe(capi.make_shape(8, 65536, 12, 8192), False, {"variant": 5})
-    assert "variant=stream" in st and "recurrence CTAs 96" in st and "2 CTAs per SM" in st
+    assert "variant=stream" in st and "recurrences 96" in st and "one CTA per SM" in st
     # stream and split records take the same workspace bytes
     ws = [capi.kda_prefill_workspace_size(capi.make_shape(8, 65536, 12, 8192), False,
                                           {"variant": v}) for v in (1, 5)]
@@ -62,13 +62,12 @@ def test_describe_reports_grid_and_variant():
 
 
 def test_stream_variant_needs_free_slots():
-    # two CTAs per SM: N H + 16 must fit twice the SM count (148 without a GPU)
+    # at most one chain per SM (148 without a GPU)
     big = capi.make_shape(2, 2 * 128, 160, 128)           # 320 chains
     assert capi.kda_prefill_describe(big, False, {"variant": 5}).startswith("variant=stream")
     o = capi.kda_options_t()
     o.variant = 5
-    # 290 chains leave fewer than 16 of the 2 x 148 slots for prepare CTAs
-    assert call(fake_args(T=1, H=290, h0=None, ht=None, opts=o)) == capi.KDA_ERR_BAD_OPTION
+    assert call(fake_args(T=1, H=150, h0=None, ht=None, opts=o)) == capi.KDA_ERR_BAD_OPTION
 
 
 # --- host-side validation with fake, never-dereferenced device addresses ----------

@@ -1,6 +1,6 @@
-"""The stream launch (recurrence CTAs with the state's key channel on the tensor-memory
-lanes, two CTAs per SM beside prepare CTAs of the same cooperative launch) vs the
-FP64 oracle (needs a B200)."""
+"""The stream launch (one CTA per SM; on up to one SM per chain, half the CTA carries a
+recurrence with the state's key channel on the tensor-memory lanes, beside a prepare
+group in the other half) vs the FP64 oracle (needs a B200)."""
 import numpy as np
 import pytest
 import torch
@@ -127,15 +127,23 @@ def test_stream_frontend_all_switches():
     assert_parity(compare(fe_inp, run_gpu(fe_inp, variant=STREAM, frontend=fe), frontend=fe))
 
 
-def test_stream_many_chains_two_per_sm():
-    # more chains than SMs: some SMs hold two recurrence CTAs
-    inp = make_inputs([130] * 20, 8, seed=621, with_h0=True)   # 160 chains
+def test_stream_many_chains_one_per_sm():
+    # 144 chains: nearly every SM carries a recurrence beside one prepare group
+    inp = make_inputs([130, 70] * 9, 8, seed=621, with_h0=True)
     res = run_gpu(inp, variant=STREAM)
-    assert_parity(compare(inp, res, seqs=[0, 9, 19]))
+    assert_parity(compare(inp, res, seqs=[0, 9, 17]))
+
+
+def test_stream_more_chains_than_sms_is_refused():
+    import kda_chunked_recurrent_b200 as K
+    inp = make_inputs([64] * 20, 8, seed=622)                  # 160 chains
+    with pytest.raises(K.KDAError) as e:
+        run_gpu(inp, variant=STREAM)
+    assert e.value.code == K.capi.KDA_ERR_BAD_OPTION
 
 
 @pytest.mark.parametrize("name", ["B1_T8192_H12", "B8_T8192_H12", "B4_T8192_H12_h0_ckpt",
-                                  "ragged16_H12_h0", "packed_1024x8_H12_h0"])
+                                  "B6_T8192_H12", "packed_1024x8_H12_h0"])
 def test_stream_full_size_workloads_sampled(name):
     inp = workload(name)
     res = run_gpu(inp, variant=STREAM)
