@@ -69,7 +69,8 @@ constexpr uint32_t kSmemAlloc = kBytes + 1024;
 constexpr uint32_t kTxA = 32768, kTxY = 16384 + 8192 + 16384;
 constexpr uint32_t kColS = 0, kColPQ = 128;
 constexpr int kIssuer = 64;         // warp 2, lane 0
-constexpr int kProducer = 32;       // warp 1, lane 0
+constexpr int kProducer = 32;       // warp 1, lane 0: record flags, A tiles
+constexpr int kLoaderY = 96;        // warp 3, lane 0: Kd / Aqk / U tiles
 constexpr uint32_t kBarAll = 1, kBarUd = 2;   // named barriers (ids 1, 2)
 static_assert(kUd + 16384 == kBytes && kKd + 16384 == kS0, "layout");
 }  // namespace chain
@@ -117,8 +118,7 @@ __device__ __forceinline__ bool acquire_record(const KdaParams& p, int64_t rec, 
 __device__ __forceinline__ void chain_body(const KdaParams& p, const SplitMaps& maps,
                                            uint8_t* smem_raw, int unit, uint32_t tbase) {
   using namespace chain;
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                           ~static_cast<uintptr_t>(1023));
+  uint8_t* sm = smem_align<1024>(smem_raw);
   __shared__ uint64_t fullA_bar, fullY_bar, p_bar, s_bar, o_bar, drain_bar;
   __shared__ int32_t s_abort;
   volatile int32_t* abort_flag = &s_abort;
@@ -179,9 +179,10 @@ __device__ __forceinline__ void chain_body(const KdaParams& p, const SplitMaps& 
     tma_load_2d(sm + kA + 16384, &maps.qw, &fullA_bar, 64, static_cast<int32_t>(r * 128));
     ++issuedA;
   };
-  auto load_Y = [&](int j) {
+  auto load_Y = [&](int j) {   // (the loader thread; the record was acquired by the producer)
     const int64_t r = rec_of(j);
     if (r < 0) return;
+    asm volatile("fence.proxy.async.global;" ::: "memory");
     mbar_arrive_expect_tx(&fullY_bar, kTxY);
     tma_load_2d(sm + kKd, &maps.kd, &fullY_bar, 0, static_cast<int32_t>(r * 64));
     tma_load_2d(sm + kKd + 8192, &maps.kd, &fullY_bar, 64, static_cast<int32_t>(r * 64));
@@ -227,13 +228,9 @@ __device__ __forceinline__ void chain_body(const KdaParams& p, const SplitMaps& 
   bool ok = true;
   if (tid == kProducer && nch > 0) {
     prefetch_tmap(&maps.qw);
-    prefetch_tmap(&maps.kd);
-    prefetch_tmap(&maps.aqk);
-    prefetch_tmap(&maps.u);
     ok = acquire(0);
     if (ok) {
       load_A(0);
-      load_Y(0);
       ok = acquire(1);
     }
   }
@@ -263,7 +260,15 @@ __device__ __forceinline__ void chain_body(const KdaParams& p, const SplitMaps& 
   // records 0 and 1 are visible to every thread after this barrier
   ok = !named_bar_or(kBarAll, kThreads, !ok);
   float gam = 1.f, gam_next = 1.f;   // Gamma_end[k = L] of the current / next chunk
-  if (ok && nch > 0) gam_next = load_gamma(0);
+  if (ok && nch > 0) {
+    gam_next = load_gamma(0);
+    if (tid == kLoaderY) {
+      prefetch_tmap(&maps.kd);
+      prefetch_tmap(&maps.aqk);
+      prefetch_tmap(&maps.u);
+      load_Y(0);
+    }
+  }
   int32_t o_t0 = 0, o_c = 0;          // token span of the chunk whose O is in PQ
 
   for (int j = 0; j < nch && ok; ++j) {
@@ -308,17 +313,17 @@ __device__ __forceinline__ void chain_body(const KdaParams& p, const SplitMaps& 
         tmem_st32(tmem_addr(tbase, lane_base, kColS + v0 + part * 32), a);
       }
     }
-    // output warps: drain and store O(j - 1) (PQ lanes 0..63) before P(j) overwrites it;
-    // the producer then brings chunk j's Kd / Aqk, whose last readers (update and O of
-    // chunk j - 1) are complete
-    if (out_warp && j > 0) {
+    // update and O of chunk j - 1 complete: the output warps drain and store O(j - 1)
+    // (PQ lanes 0..63) before P(j) overwrites it, and a Ud-warp thread (whose warps
+    // would otherwise wait at the barrier) brings chunk j's Kd / Aqk / U tiles
+    if (j > 0 && (out_warp || tid == kLoaderY)) {
       ok = ok && mbar_wait(&o_bar, static_cast<uint32_t>((j - 1) & 1), budget) && !*abort_flag;
+      if (ok && tid == kLoaderY) load_Y(j);
+    }
+    if (out_warp && j > 0) {
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
-      if (ok) {
-        if (tid == kProducer) load_Y(j);
-        drain_out(o_t0, o_c);
-      }
+      if (ok) drain_out(o_t0, o_c);
     }
     tmem_wait_st();
     fence_proxy_async_smem();
@@ -474,10 +479,10 @@ __device__ __forceinline__ void chain_body(const KdaParams& p, const SplitMaps& 
 
   // ---- teardown: every TMA copy and UMMA of this unit completes before the caller frees
   // tensor memory or the CTA exits
-  if (tid == kProducer) {
-    if (issuedA > 0) mbar_wait(&fullA_bar, static_cast<uint32_t>((issuedA - 1) & 1), drain_budget);
-    if (issuedY > 0) mbar_wait(&fullY_bar, static_cast<uint32_t>((issuedY - 1) & 1), drain_budget);
-  }
+  if (tid == kProducer && issuedA > 0)
+    mbar_wait(&fullA_bar, static_cast<uint32_t>((issuedA - 1) & 1), drain_budget);
+  if (tid == kLoaderY && issuedY > 0)
+    mbar_wait(&fullY_bar, static_cast<uint32_t>((issuedY - 1) & 1), drain_budget);
   if (tid == kIssuer) {
     umma_commit(&drain_bar);
     mbar_wait(&drain_bar, 0, drain_budget);

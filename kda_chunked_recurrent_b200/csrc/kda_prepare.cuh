@@ -343,9 +343,7 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
                                              int64_t stride, int64_t nitems,
                                              PrepGroupRes res = PrepGroupRes{kTmemOwn, 0u}) {
   using namespace prep;
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                           ~static_cast<uintptr_t>(1023)) +
-                static_cast<size_t>(grp) * kGroupBytes;
+  uint8_t* sm = smem_align<1024>(smem_raw) + static_cast<uint32_t>(grp) * kGroupBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kAuxBars);
   uint64_t& tma_bar = bars[0];
   uint64_t& mma_bar = bars[1];
@@ -508,9 +506,14 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
       }
     }
 
-    // ---- raw tiles -> registers: g (float2), k, q (bf16x2) for 16 tokens x 2 channels
-    ok = mbar_wait(&raw_g_bar, static_cast<uint32_t>((raw_g_issued - 1) & 1), budget);
-    ok = ok && mbar_wait(&raw_qk_bar, static_cast<uint32_t>((raw_qk_issued - 1) & 1), budget);
+    // ---- raw tiles -> registers: g (float2), k, q (bf16x2) for 16 tokens x 2 channels.
+    // One thread waits for the copies; the others sleep in the barrier instead of polling
+    // (their polls would take issue slots from the other group on the SM).
+    if (tid == 0) {
+      ok = mbar_wait(&raw_g_bar, static_cast<uint32_t>((raw_g_issued - 1) & 1), budget);
+      ok = ok && mbar_wait(&raw_qk_bar, static_cast<uint32_t>((raw_qk_issued - 1) & 1), budget);
+    }
+    ok = !prep_sync_or<kFused>(gbar, !ok);
     float2 G[16];
     uint32_t kw[16], qw[16];
     {
@@ -725,7 +728,7 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
     }
     if constexpr (kFused) pending = -1;
     ++mma_commits;
-    ok = mbar_wait(&mma_bar, static_cast<uint32_t>((mma_commits - 1) & 1), budget);
+    if (tid == 0) ok = mbar_wait(&mma_bar, static_cast<uint32_t>((mma_commits - 1) & 1), budget);
     ok = !prep_sync_or<kFused>(gbar, !ok);
     if (ok) {
       tc_fence_after();
@@ -905,8 +908,7 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
       }
     }
     if (tid == 0 && !tma_seen) ok = false;
-    ok = !prep_sync_or<kFused>(gbar, !ok);
-    if (ok) {
+    if (tid == 0 && ok) {
       ++mma_commits;
       ok = mbar_wait(&mma_bar, static_cast<uint32_t>((mma_commits - 1) & 1), budget);
     }

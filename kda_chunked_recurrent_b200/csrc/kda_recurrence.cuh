@@ -109,8 +109,7 @@ template <bool kFused>
 __device__ __forceinline__ void recurrence_body(const KdaParams& p, const SplitMaps& maps,
                                                 uint8_t* smem_raw, int unit) {
   using namespace rec;
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                           ~static_cast<uintptr_t>(1023));
+  uint8_t* sm = smem_align<1024>(smem_raw);
   __shared__ uint64_t full_bar[kStages], empty_bar[kStages], oready_bar[kRegions], ofree_bar[kRegions];
   __shared__ uint64_t mma1_bar, sready_bar, drain_bar;
   __shared__ uint32_t tmem_slot;

@@ -18,6 +18,16 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// The dynamic shared-memory base rounded up to `align` bytes, as an offset from the
+// __shared__ pointer itself: the compiler keeps knowing the result points into shared
+// memory, so accesses through it stay 32-bit shared-window loads and stores (an
+// integer round trip would turn every one into a generic 64-bit access).
+template <uint32_t align>
+__device__ __forceinline__ uint8_t* smem_align(uint8_t* smem_raw) {
+  const uint32_t a = smem_u32(smem_raw);
+  return smem_raw + (((a + (align - 1)) & ~(align - 1)) - a);
+}
+
 // ------------------------------------------------------------------ mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
