@@ -10,6 +10,7 @@
 // [schedule] -> ready-flag clear -> one cooperative launch (fused variant).
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <cstdio>
@@ -246,21 +247,39 @@ int choose_variant(const kda_shape_t* s, const kda_options_t* o) {
 }
 
 // Hybrid variant: how many of the last chunks of every sequence the fused launch's
-// prepare groups make while its recurrence CTAs run.  The recurrence takes about
-// 1.8 us per chunk; a prepare group inside the fused launch about 13.5 us per
-// record (measured: B6 T8192 H12 with a 47-chunk tail), so the free SMs (2
-// groups each) keep up with jmax * f * 41 / R rows of R records, f = free SM
-// share; 0.9 of that keeps the producer ahead.
-// With the input front end the prepare side is slower (measured 0.585 vs 0.369 ms for
-// the prepare launch at B8 T8192 H12), so its tail is shorter by that ratio.
+// prepare groups make while its recurrence CTAs run.  The recurrence CTAs walk all jmax
+// chunks (the first jmax - tail from the preceding prepare launch) at one chunk step per
+// kFusedStepCycles; the 2 (SMs - R) prepare groups on the free SMs make one record per
+// kFusedPrepCycles each, R records per chunk row.  The tail rows must be ready before the
+// chains reach them, which they do if the groups make them within the chain's time:
+//   tail R kFusedPrepCycles / (2 (SMs - R))  <=  jmax kFusedStepCycles,
+// so tail = slack jmax (2 (SMs - R) / R) (kFusedStepCycles / kFusedPrepCycles).  Only the
+// ratio of the two cycle counts enters, and it does not depend on the clock.  Measured on
+// a B200 (CUDA events, 1965 MHz): a chunk step of the fused launch 1.94 us at B8 T8192 H12
+// (3.8K cycles), a record of a fused prepare group 13.5 us (26.5K cycles) with a 47-chunk
+// tail at B6 T8192 H12; the front-end prepare is slower by the measured ratio of the
+// prepare launches at B8 T8192 H12 (0.585 / 0.369 ms).  The slack keeps the producer ahead.
+constexpr double kFusedStepCycles = 3800.0;
+constexpr double kFusedPrepCycles = 26500.0;
+constexpr double kFusedPrepCyclesFE = 26500.0 * 0.585 / 0.369;
+constexpr double kHybridTailSlack = 0.9;
 int64_t hybrid_tail_chunks(int64_t jmax, int64_t chains, bool frontend = false) {
-  const double sms = static_cast<double>(sm_count());
-  const double f = (sms - static_cast<double>(chains)) / sms;
-  const double rate = frontend ? 41.0 * 0.369 / 0.585 : 41.0;
-  int64_t tail = static_cast<int64_t>(0.9 * static_cast<double>(jmax) * f * rate /
-                                      static_cast<double>(chains));
-  return std::max<int64_t>(1, std::min<int64_t>(tail, jmax - 1));
+  const double free_groups = 2.0 * (static_cast<double>(sm_count()) - static_cast<double>(chains));
+  const double per_rec = frontend ? kFusedPrepCyclesFE : kFusedPrepCycles;
+  const double tail = kHybridTailSlack * static_cast<double>(jmax) * free_groups /
+                      static_cast<double>(chains) * (kFusedStepCycles / per_rec);
+  return std::max<int64_t>(1, std::min<int64_t>(static_cast<int64_t>(tail), jmax - 1));
 }
+
+// A named NVTX range over the host calls that enqueue one launch, so that a timeline
+// tool shows which kernel each launch API call belongs to.  Header-only NVTX: without
+// a tool attached the push and pop cost a few nanoseconds.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 // Upper bound on the chunks of one sequence (the fused launch's chunk-major items).
 int64_t max_chunks_per_seq(const kda_shape_t* s, bool fixed, bool ckpt) {
@@ -613,10 +632,12 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
                          ? (cu64 || (flags & KDA_FLAG_VALIDATE))
                          : (!fixed || ckpt || (flags & KDA_FLAG_VALIDATE));
   if (sched) {
+    NvtxRange nr("kda_schedule");
     kda_schedule_kernel<<<1, 1024, 0, s>>>(p);
     mark(0);
   }
   if (r.variant == KDA_VARIANT_TOKEN) {
+    NvtxRange nr("kda_token");
     mark(1);
     TokenParams tp{};
     tp.q = p.q;
@@ -648,6 +669,7 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
     if (st != KDA_OK) return st;
     mark(2);
   } else if (r.variant == KDA_VARIANT_STREAM) {
+    NvtxRange nr("kda_stream");
     mark(1);
     // one cooperative launch of two CTAs per SM: CTAs 0 .. N H - 1 run the recurrences,
     // the rest prepare the chunk records in chunk-major order
@@ -678,6 +700,7 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
     const int64_t jmax = max_chunks_per_seq(shape, fixed, ckpt);
     int64_t j0 = 0;
     if (r.variant == KDA_VARIANT_HYBRID && T > 0) {
+      NvtxRange nr("kda_prepare");
       // the prepare launch makes chunks [0, j0) of every sequence first
       j0 = jmax - hybrid_tail_chunks(jmax, N * H, p.fe_flags != 0);
       p.split_jmax = static_cast<int32_t>(j0);
@@ -690,6 +713,7 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
       p.split_jmax = INT32_MAX;
     }
     p.fused_j0 = static_cast<int32_t>(j0);
+    NvtxRange nr("kda_fused");
     mark(1);
     // one cooperative launch: CTAs 0 .. N H - 1 run the recurrences, the rest of
     // the SMs (one CTA each) prepare the chunk records in chunk-major order
@@ -719,6 +743,7 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
     mark(2);
   } else {
     if (T > 0) {
+      NvtxRange nr("kda_prepare");
       // persistent prepare grid: two CTAs per SM walk the (chunk slot, head) items
       const int64_t items = r.lay.slots * H;
       const int64_t grid = std::min<int64_t>(items, 2 * static_cast<int64_t>(sm_count()));
@@ -728,6 +753,7 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
         kda_prepare_kernel<<<static_cast<unsigned>(grid), 256, prep::kSmemAllocBytes, s>>>(p, maps);
     }
     mark(1);
+    NvtxRange nr("kda_recurrence");
     kda_recurrence_kernel<<<static_cast<unsigned>(N * H), rec::kThreadsPerCta,
                             rec::kSmemAllocBytes, s>>>(p, maps);
     mark(2);
@@ -817,6 +843,7 @@ kda_status_t kda_decode(const void* q, const void* k, const void* v, const float
   if (fe & KDA_FE_QK_L2NORM) tp.l2_eps = frontend->l2_eps;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   (void)cudaGetLastError();
+  NvtxRange nr("kda_decode");
   st = launch_token(tp, N * H, token_wide(N * H, flags), s);
   if (st != KDA_OK) return st;
   if (cudaGetLastError() != cudaSuccess) return KDA_ERR_LAUNCH_FAILED;

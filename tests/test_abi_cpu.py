@@ -173,6 +173,38 @@ def test_auto_variant_follows_the_table():
     assert "variant=split" in huge, huge
 
 
+def _hybrid_tail(N, T_seq, H, fe=False):
+    import re
+    opts = {"variant": 3}
+    if fe:
+        opts["frontend"] = {"flags": 7, "lower_bound": -5.0, "l2_eps": 1e-6}
+    d = capi.kda_prefill_describe(capi.make_shape(N, N * T_seq, H, T_seq), False, opts)
+    m = re.search(r"prepare_chunks=(\d+)/(\d+)", d)
+    assert m, d
+    first, jmax = int(m.group(1)), int(m.group(2))
+    return jmax - first, jmax
+
+
+def test_hybrid_tail_follows_the_throughput_rule():
+    # the tail (chunk rows made inside the fused launch) grows with the chunks per
+    # sequence and the free SMs, shrinks with the chains and with a slower prepare
+    tails = {N: _hybrid_tail(N, 8192, 12) for N in (5, 6, 7, 8, 9, 10)}
+    for N, (tail, jmax) in tails.items():
+        assert jmax == 128 and 1 <= tail <= jmax - 1, (N, tail)
+    seq = [tails[N][0] for N in sorted(tails)]
+    assert all(a > b for a, b in zip(seq, seq[1:])), seq
+    t_long, j_long = _hybrid_tail(8, 16384, 12)
+    assert j_long == 256 and abs(t_long - 2 * tails[8][0]) <= 1, (t_long, tails[8])
+    fe_tail, _ = _hybrid_tail(8, 8192, 12, fe=True)
+    assert 1 <= fe_tail < tails[8][0]
+    # two chunks per sequence: the tail is clamped to leave one row for the prepare launch
+    assert _hybrid_tail(8, 128, 12) == (1, 2)
+    # nearly every SM carries a chain: the fused prepare groups get the one-row minimum
+    assert _hybrid_tail(11, 8192, 12)[0] == 4 and _hybrid_tail(12, 8192, 12)[0] == 1
+    # the rule at the measured shape: 96 chains on 148 SMs keep 17 of 128 rows in the launch
+    assert tails[8][0] == 17 and tails[6][0] == 34, tails
+
+
 def test_fused_variant_needs_free_sms():
     torch = pytest.importorskip("torch")
     o = capi.kda_options_t()
