@@ -74,8 +74,11 @@ constexpr uint32_t kGraw = kR;                  // g [64 tok][128 ch] f32 (32 KB
 constexpr uint32_t kRawQKTx = 16384 + 16384;
 constexpr uint32_t kRawGTx = 32768;
 // the thread that stores Aqk and requests the next g tile (warp 7, idle in the
-// diagonal solve); thread 0 issues every other copy and UMMA
+// off-diagonal solve); thread 0 issues every other copy and UMMA
 constexpr int kGThread = 224;
+// the thread that prefetches the next item's tiles into L2 (warp 1, idle while thread 0
+// issues the first UMMA)
+constexpr int kPrefetchThread = 32;
 // aliases of [K+; Q+] once the first UMMA has completed: the solve scratch, and
 // after the solve the staging tiles of the W^T / U^T TMA stores
 constexpr int kLdh = 72;
@@ -83,7 +86,6 @@ constexpr int kMfBlk = 272;                     // floats per diagonal block of 
 constexpr uint32_t kMf = kL;                    // f32 [4][16 s][16 r] diagonal blocks of M, column-major
 constexpr uint32_t kMh = kMf + 4 * kMfBlk * 4;  // f16 [64][72] off-diagonal blocks of M
 constexpr uint32_t kXh = kMh + 64 * kLdh * 2;   // f16 [64][72] T = (I + M)^-1
-constexpr uint32_t kWk = kXh + 64 * kLdh * 2;   // f16 [3][16][72] one 16x16 scratch block per solve warp
 constexpr uint32_t kWs = kL;                    // W^T staging [128 k][64 tok] f16, 128B swizzle
 constexpr uint32_t kUs = kL + 16384;            // U^T staging [128 v][64 tok] f16, 128B swizzle
 // aliases of R once the first UMMA has completed
@@ -100,7 +102,7 @@ constexpr uint32_t kAuxNorm = kAuxFirst + 2048;  // f32 [2][64] inverse norms of
 constexpr uint32_t kAuxClaim = kAuxNorm + 512;   // i64 [2] claimed item indices (stream launch)
 constexpr uint32_t kGroupBytes = (kAuxClaim + 16 + 1023) / 1024 * 1024;   // one prepare group
 constexpr uint32_t kSmemAlloc = kGroupBytes + 1024;
-static_assert(kWk + 3 * 16 * kLdh * 2 <= kR, "solve scratch overlaps the Aqk staging tile");
+static_assert(kXh + 64 * kLdh * 2 <= kR, "solve scratch overlaps the Aqk staging tile");
 static_assert(kAqs + 8192 <= kTb, "Aqk staging overlaps the Tb tile");
 static_assert(kUs + 16384 <= kR, "W/U staging overlaps R");
 }  // namespace prep
@@ -183,6 +185,73 @@ __device__ __forceinline__ void store_tb16(uint32_t tb, const float* beta, int r
     const uint32_t off = static_cast<uint32_t>((s & 7) * 2);
     sts32(tb + sw128_offset(r0 + g, s >> 3) + off, pack_f16(x1[0] * b0, x1[1] * b1));
     sts32(tb + sw128_offset(r0 + g + 8, s >> 3) + off, pack_f16(x1[2] * b0, x1[3] * b1));
+  }
+}
+
+__device__ __forceinline__ void sts16(uint32_t addr, uint16_t v) {
+  asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
+}
+
+// One block column J of T = (I + M)^-1 below the diagonal, by one warp, in registers.
+// The transposed form
+//   P_i^T = sum_{k=J}^{i-1} X_kJ^T M_ik^T,   X_iJ^T = -P_i^T X_ii^T,   i = J+1 .. 3,
+// makes every product's FP32 accumulator the A fragment of the next product (rounded to
+// FP16), so the column's chain never goes through shared memory; the M_ik and X_ii
+// blocks it reads (B fragments: their rows, as stored) do not depend on the chain.
+// Each finished block is written as FP16 T diag(beta) into the swizzled Tb tile.
+template <int J>
+__device__ __forceinline__ void offdiag_column(uint32_t aMh, uint32_t aXh, uint32_t aTb,
+                                               const float* beta, int lane) {
+  using prep::kLdh;
+  // lane addresses of a 16x16 block's four 8x8 matrices, in the order (rows 0-7, col 0),
+  // (rows 0-7, col 8), (rows 8-15, col 0), (rows 8-15, col 8): the B fragment of the
+  // block's transpose, or with .trans the A fragment of it
+  const uint32_t lofs =
+      static_cast<uint32_t>((((lane & 7) + ((lane >> 4) & 1) * 8) * kLdh + ((lane >> 3) & 1) * 8) * 2);
+  auto at = [&](uint32_t base, int r0, int c0) {
+    return base + static_cast<uint32_t>((r0 * kLdh + c0) * 2) + lofs;
+  };
+  const int g = lane >> 2, q = lane & 3;
+  uint32_t xa[4 - J][4];   // A fragments of X_kJ^T, k = J .. 3 (FP16)
+  ldsm_x4_t(at(aXh, J * 16, J * 16), xa[0]);
+#pragma unroll
+  for (int i = J + 1; i < 4; ++i) {
+    float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int k = J; k < i; ++k) {
+      uint32_t b[4];
+      ldsm_x4(at(aMh, i * 16, k * 16), b);
+      mma16816(c0, xa[k - J], b[0], b[1]);
+      mma16816(c1, xa[k - J], b[2], b[3]);
+    }
+    const uint32_t pa[4] = {pack_f16(-c0[0], -c0[1]), pack_f16(-c0[2], -c0[3]),
+                            pack_f16(-c1[0], -c1[1]), pack_f16(-c1[2], -c1[3])};
+    uint32_t b[4];
+    ldsm_x4(at(aXh, i * 16, i * 16), b);
+    float x0[4] = {0.f, 0.f, 0.f, 0.f}, x1[4] = {0.f, 0.f, 0.f, 0.f};
+    mma16816(x0, pa, b[0], b[1]);
+    mma16816(x1, pa, b[2], b[3]);
+    if (i < 3) {
+      xa[i - J][0] = pack_f16(x0[0], x0[1]);
+      xa[i - J][1] = pack_f16(x0[2], x0[3]);
+      xa[i - J][2] = pack_f16(x1[0], x1[1]);
+      xa[i - J][3] = pack_f16(x1[2], x1[3]);
+    }
+    // X_iJ^T[s][r] -> Tb row 16 i + r, column 16 J + s, times beta of the column:
+    // x0 holds s = g (r = 2q, 2q+1) and s = g + 8; x1 the same for r + 8
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int s = J * 16 + g + 8 * h;
+      const float bs = beta[s];
+      const uint32_t cb = static_cast<uint32_t>(s >> 3), co = static_cast<uint32_t>((s & 7) * 2);
+      const float* lo = h ? x0 + 2 : x0;
+      const float* hi = h ? x1 + 2 : x1;
+      const uint32_t r0 = static_cast<uint32_t>(i * 16 + 2 * q);
+      sts16(aTb + sw128_offset(r0, cb) + co, __half_as_ushort(__float2half_rn(lo[0] * bs)));
+      sts16(aTb + sw128_offset(r0 + 1, cb) + co, __half_as_ushort(__float2half_rn(lo[1] * bs)));
+      sts16(aTb + sw128_offset(r0 + 8, cb) + co, __half_as_ushort(__float2half_rn(hi[0] * bs)));
+      sts16(aTb + sw128_offset(r0 + 9, cb) + co, __half_as_ushort(__float2half_rn(hi[1] * bs)));
+    }
   }
 }
 
@@ -361,6 +430,9 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
 
   const int tid = threadIdx.x - grp * kThreads;
   const int warp = tid >> 5, lane = tid & 31;
+  // packed FP32 pair arithmetic in the element-wise pass (same bits as the scalar
+  // form), where the register budget allows it: the split kernel's
+  constexpr bool kPack = !kFused;
   const uint32_t gbar = res.bar != 0u ? res.bar : 1u + static_cast<uint32_t>(grp);
   const bool own_tmem = res.tmem == kTmemOwn;
   if ((p.flags & kFlagValidate) && reinterpret_cast<const WsHeader*>(p.ws)->call_ok == 0) return;
@@ -486,26 +558,6 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
       }
     }
 
-    // ---- L2 prefetch of the next item's tiles (q, k, g, v) and beta rows
-    if (nxt_valid) {
-      if (tid == 0) {
-        tma_prefetch_3d(&maps.q_in, 0, nxt.h, nxt.t0);
-        tma_prefetch_3d(&maps.k_in, 0, nxt.h, nxt.t0);
-        tma_prefetch_3d(&maps.g_in, 0, nxt.h, nxt.t0);
-        tma_prefetch_3d(&maps.v_in, 0, nxt.h, nxt.t0);
-        tma_prefetch_3d(&maps.v_in, 64, nxt.h, nxt.t0);
-        // beta rows of the next chunk, all heads: 16-byte aligned and inside the tensor
-        const uintptr_t lo =
-            reinterpret_cast<uintptr_t>(p.beta + static_cast<int64_t>(nxt.t0) * p.H) & ~uintptr_t(15);
-        uintptr_t hi = (reinterpret_cast<uintptr_t>(p.beta + static_cast<int64_t>(nxt.t0 + nxt.c) * p.H) + 15) &
-                       ~uintptr_t(15);
-        const uintptr_t lim =
-            reinterpret_cast<uintptr_t>(p.beta + static_cast<int64_t>(p.T) * p.H) & ~uintptr_t(15);
-        hi = hi < lim ? hi : lim;
-        if (hi > lo) bulk_prefetch_l2(reinterpret_cast<const void*>(lo), static_cast<uint32_t>(hi - lo));
-      }
-    }
-
     // ---- raw tiles -> registers: g (float2), k, q (bf16x2) for 16 tokens x 2 channels.
     // One thread waits for the copies; the others sleep in the barrier instead of polling
     // (their polls would take issue slots from the other group on the SM).
@@ -575,10 +627,10 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
     // ---- gate scan within the sub-block; one exchange gives every sub-block start
     {
       float2 run = make_float2(0.f, 0.f);
+      const float2 l2e = make_float2(kLog2e, kLog2e);
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        run.x = fmaf(G[i].x, kLog2e, run.x);
-        run.y = fmaf(G[i].y, kLog2e, run.y);
+        run = fma2<kPack>(G[i], l2e, run);
         G[i] = run;
       }
       s_first[blk][cp] = G[0];
@@ -615,10 +667,7 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
       }
       E = acc;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        G[i].x += pre.x;
-        G[i].y += pre.y;
-      }
+      for (int i = 0; i < 16; ++i) G[i] = add2<kPack>(G[i], pre);
     }
 
     // ---- operands
@@ -650,32 +699,33 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
                              kStream ? p.ws + p.lay.qw + rec * kTileQW : p.ws + p.lay.qg + rec * kTileQG) +
                          blk * 16 * 64 + cp;
       uint32_t* kd_out = reinterpret_cast<uint32_t*>(p.ws + p.lay.kd + rec * kTileKd) + blk * 16 * 64 + cp;
+      const float2 nB = make_float2(-B.x, -B.y);
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const uint32_t xo = ((chunk ^ static_cast<uint32_t>(i & 7)) << 4) + static_cast<uint32_t>(i) * 128u;
-        const float2 g2 = G[i];
-        float e0 = ex2(g2.x - B.x), e1 = ex2(g2.y - B.y);
-        float i0 = ex2(B.x - g2.x), i1 = ex2(B.y - g2.y);
+        const float2 d = add2<kPack>(G[i], nB);                 // G_r - B_b
+        const float2 e = make_float2(ex2(d.x), ex2(d.y));       // e_r
+        float2 inv = make_float2(ex2(-d.x), ex2(-d.y));         // 1 / e_r
+        const float2 kf = bf2_to_f2(kw[i]), qf = bf2_to_f2(qw[i]);
+        const float2 gam = mul2<kPack>(e, cB);                  // Gamma_r, FP32
         if (kFE && fe_norm) {
           // front end: the row's inverse norms ride on the FP32 factors (one rounding each)
           const float rk = s_norm[blk * 16 + i], rq = s_norm[64 + blk * 16 + i];
-          const uint32_t e2k = pack_bf16(e0 * rk, e1 * rk), e2q = pack_bf16(e0 * rq, e1 * rq);
+          const float2 rk2 = make_float2(rk, rk), rq2 = make_float2(rq, rq);
+          const uint32_t e2k = pack_bf16(mul2<kPack>(e, rk2)), e2q = pack_bf16(mul2<kPack>(e, rq2));
           sts32(bL + xo, hmul2_bf16(kw[i], e2k));
           sts32(bL + xo + 64u * 128u, hmul2_bf16(qw[i], e2q));
-          const uint32_t rd2 = hmul2_bf16(kw[i], pack_bf16(i0 * rk, i1 * rk));
+          const uint32_t rd2 = hmul2_bf16(kw[i], pack_bf16(mul2<kPack>(inv, rk2)));
           sts32(bRo + xo, rd2);
           if (blk < 1) sts32(bR + xo + 16u * 128u, hmul2_bf16(rd2, c1b));
           if (blk < 2) sts32(bR + xo + 48u * 128u, hmul2_bf16(rd2, c2b));
           if (blk < 3) sts32(bR + xo + 96u * 128u, hmul2_bf16(rd2, c3b));
-          const float2 kf = bf2_to_f2(kw[i]), qf = bf2_to_f2(qw[i]);
-          const float gx = e0 * cB.x, gy = e1 * cB.y;   // Gamma_r, FP32
-          sts32(bKG + xo, pack_f16(kf.x * (gx * rk), kf.y * (gy * rk)));
-          qg_out[i * 64] = pack_f16(qf.x * (gx * rq), qf.y * (gy * rq));
-          i0 *= rk;
-          i1 *= rk;
+          sts32(bKG + xo, pack_f16(mul2<kPack>(kf, mul2<kPack>(gam, rk2))));
+          qg_out[i * 64] = pack_f16(mul2<kPack>(qf, mul2<kPack>(gam, rq2)));
+          inv = mul2<kPack>(inv, rk2);
         } else {
           // bf16 operands: factors rounded to bf16, products in packed bf16 math
-          const uint32_t e2 = pack_bf16(e0, e1), inv2 = pack_bf16(i0, i1);
+          const uint32_t e2 = pack_bf16(e), inv2 = pack_bf16(inv);
           sts32(bL + xo, hmul2_bf16(kw[i], e2));
           sts32(bL + xo + 64u * 128u, hmul2_bf16(qw[i], e2));
           const uint32_t rd2 = hmul2_bf16(kw[i], inv2);
@@ -685,14 +735,11 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
           if (blk < 3) sts32(bR + xo + 96u * 128u, hmul2_bf16(rd2, c3b));
           // K Gamma (A of the W UMMA) and Q Gamma (B of the state read): FP16 products of
           // FP32 factors, one rounding each
-          const float2 kf = bf2_to_f2(kw[i]), qf = bf2_to_f2(qw[i]);
-          const float gx = e0 * cB.x, gy = e1 * cB.y;   // Gamma_r, FP32
-          sts32(bKG + xo, pack_f16(kf.x * gx, kf.y * gy));
-          qg_out[i * 64] = pack_f16(qf.x * gx, qf.y * gy);
+          sts32(bKG + xo, pack_f16(mul2<kPack>(kf, gam)));
+          qg_out[i * 64] = pack_f16(mul2<kPack>(qf, gam));
         }
         // Kd feeds the FP16 state update: FP32 products, one rounding
-        const float2 kf = bf2_to_f2(kw[i]);
-        kd_out[i * 64] = pack_f16(kf.x * i0 * cE.x, kf.y * i1 * cE.y);
+        kd_out[i * 64] = pack_f16(mul2<kPack>(mul2<kPack>(kf, inv), cE));
       }
       if (blk == 0)
         reinterpret_cast<float2*>(p.ws + p.lay.gc + rec * kTileGC)[cp] =
@@ -727,6 +774,41 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
       }
     }
     if constexpr (kFused) pending = -1;
+    // While the first UMMA runs (it does not read the v tile), warps 1-7 turn the v tile,
+    // landed by TMA during the element-wise pass, from BF16 into FP16 in place: the U UMMA
+    // multiplies it by the FP16 T diag(beta), and both operands of one UMMA share a type
+    // (BF16 -> FP16 is exact for |v| in the FP16 normal range).  One of them first
+    // prefetches the next item's tiles (q, k, g, v) and beta rows into L2.
+    if (tid >= 32) {
+      if (tid == kPrefetchThread && nxt_valid) {
+        tma_prefetch_3d(&maps.q_in, 0, nxt.h, nxt.t0);
+        tma_prefetch_3d(&maps.k_in, 0, nxt.h, nxt.t0);
+        tma_prefetch_3d(&maps.g_in, 0, nxt.h, nxt.t0);
+        tma_prefetch_3d(&maps.v_in, 0, nxt.h, nxt.t0);
+        tma_prefetch_3d(&maps.v_in, 64, nxt.h, nxt.t0);
+        // beta rows of the next chunk, all heads: 16-byte aligned and inside the tensor
+        const uintptr_t lo =
+            reinterpret_cast<uintptr_t>(p.beta + static_cast<int64_t>(nxt.t0) * p.H) & ~uintptr_t(15);
+        uintptr_t hi = (reinterpret_cast<uintptr_t>(p.beta + static_cast<int64_t>(nxt.t0 + nxt.c) * p.H) + 15) &
+                       ~uintptr_t(15);
+        const uintptr_t lim =
+            reinterpret_cast<uintptr_t>(p.beta + static_cast<int64_t>(p.T) * p.H) & ~uintptr_t(15);
+        hi = hi < lim ? hi : lim;
+        if (hi > lo) bulk_prefetch_l2(reinterpret_cast<const void*>(lo), static_cast<uint32_t>(hi - lo));
+      }
+      if (mbar_wait(&tma_bar, tma_parity, budget)) {
+        uint4* vt = reinterpret_cast<uint4*>(sm + kV);
+        for (int i = tid - 32; i < 16384 / 16; i += kThreads - 32) {
+          const uint4 x = vt[i];
+          const float2 a = bf2_to_f2(x.x), b = bf2_to_f2(x.y), c2 = bf2_to_f2(x.z),
+                       d = bf2_to_f2(x.w);
+          vt[i] = make_uint4(pack_f16(a.x, a.y), pack_f16(b.x, b.y), pack_f16(c2.x, c2.y),
+                             pack_f16(d.x, d.y));
+        }
+      } else {
+        ok = false;
+      }
+    }
     ++mma_commits;
     if (tid == 0) ok = mbar_wait(&mma_bar, static_cast<uint32_t>((mma_commits - 1) & 1), budget);
     ok = !prep_sync_or<kFused>(gbar, !ok);
@@ -785,14 +867,13 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
     if (ok && tid == kGThread) {
       tma_store_2d(&maps.aqk, sm + kAqs, 0, static_cast<int32_t>(rec * 64));
       bulk_commit();
-      // R (UMMA1's operand, then the Aqk staging tile) is free once the store has
-      // read it: the next item's g tile goes there now, a whole solve early
-      if (nxt_valid) {
-        bulk_wait_read();
-        issue_g(nxt);
-      }
     }
-    if (ok && nxt_valid) {
+    // R (UMMA1's operand, then the Aqk staging tile) is free once that store has read
+    // it: kGThread requests the next item's g tile there during the off-diagonal solve,
+    // where its warp is idle (so waiting for the store does not hold up the diagonal
+    // phase), a whole UMMA 2 early
+    const bool g_next = ok && nxt_valid;
+    if (g_next) {
       ++raw_g_issued;
       g_for_cur = true;   // (for the next iteration)
     }
@@ -830,47 +911,20 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
           if (ch >= 2 * ((r >> 4) + 1))
             *reinterpret_cast<uint4*>(sm + kTb + sw128_offset(r, ch)) = make_uint4(0u, 0u, 0u, 0u);
         }
-        // ---- the v tile (BF16, landed by TMA in its operand layout) becomes FP16 in
-        // place: the U UMMA multiplies it by the FP16 T diag(beta), and both operands of
-        // one UMMA share a type.  (BF16 -> FP16 is exact for |v| in the FP16 normal range.)
-        if (mbar_wait(&tma_bar, tma_parity, budget)) {
-          uint4* vt = reinterpret_cast<uint4*>(sm + kV);
-          for (int i = tid - 64; i < 16384 / 16; i += kThreads - 64) {
-            const uint4 x = vt[i];
-            const float2 a = bf2_to_f2(x.x), b = bf2_to_f2(x.y), c2 = bf2_to_f2(x.z),
-                         d = bf2_to_f2(x.w);
-            vt[i] = make_uint4(pack_f16(a.x, a.y), pack_f16(b.x, b.y), pack_f16(c2.x, c2.y),
-                               pack_f16(d.x, d.y));
-          }
-        } else {
-          ok = false;
-        }
       }
       prep_sync<kFused>(gbar);
       // ---- off-diagonal blocks, one block column j per warp, down the column:
       //   X_ij = -X_ii (sum_{k=j}^{i-1} M_ik X_kj),  i = j+1 .. 3,
       // FP16 mma.sync with FP32 accumulation.  Column j only reads its own earlier
-      // blocks and the diagonal blocks, so the warps need no barrier between levels.
+      // blocks (held in registers) and the diagonal blocks, so the warps need no
+      // barrier between levels.
       if (warp < 3) {
-        const int j = warp;
-        __half* wk = reinterpret_cast<__half*>(sm + kWk) + warp * 16 * kLdh;
-        const uint32_t aWk = sbase + kWk + static_cast<uint32_t>(warp * 16 * kLdh * 2);
-        for (int i = j + 1; i < 4; ++i) {
-          float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
-          for (int k = j; k < i; ++k) mma_block(a0, a1, aMh, i * 16, k * 16, aXh, k * 16, j * 16, lane);
-          store_frag16(wk, kLdh, a0, a1, 1.f, lane);
-          __syncwarp();
-          float x0[4] = {0.f, 0.f, 0.f, 0.f}, x1[4] = {0.f, 0.f, 0.f, 0.f};
-          mma_block(x0, x1, aXh, i * 16, i * 16, aWk, 0, 0, lane);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            x0[e] = -x0[e];
-            x1[e] = -x1[e];
-          }
-          store_frag16(Xh + (i * 16) * kLdh + j * 16, kLdh, x0, x1, 1.f, lane);
-          store_tb16(aTb, s_beta, i * 16, j * 16, x0, x1, lane);
-          __syncwarp();
-        }
+        if (warp == 0) offdiag_column<0>(aMh, aXh, aTb, s_beta, lane);
+        else if (warp == 1) offdiag_column<1>(aMh, aXh, aTb, s_beta, lane);
+        else offdiag_column<2>(aMh, aXh, aTb, s_beta, lane);
+      } else if (tid == kGThread && g_next) {
+        bulk_wait_read();
+        issue_g(nxt);
       }
     }
     fence_proxy_async_smem();

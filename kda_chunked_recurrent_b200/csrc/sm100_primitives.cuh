@@ -356,6 +356,25 @@ __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
   asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
+__device__ __forceinline__ uint32_t pack_bf16(float2 v) { return pack_bf16(v.x, v.y); }
+__device__ __forceinline__ uint32_t pack_f16(float2 v) { return pack_f16(v.x, v.y); }
+// FP32 pairs: with kPack one packed instruction for both lanes (sm_100), else two
+// scalar ones; each lane is rounded to nearest like the scalar operation, so both
+// forms give the same bits.  (The packed form wants its operands in aligned register
+// pairs, which can cost spills in kernels already at their register limit.)
+template <bool kPack>
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  if constexpr (kPack) return __fadd2_rn(a, b); else return make_float2(a.x + b.x, a.y + b.y);
+}
+template <bool kPack>
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  if constexpr (kPack) return __fmul2_rn(a, b); else return make_float2(a.x * b.x, a.y * b.y);
+}
+template <bool kPack>
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  if constexpr (kPack) return __ffma2_rn(a, b, c);
+  else return make_float2(fmaf(a.x, b.x, c.x), fmaf(a.y, b.y, c.y));
+}
 __device__ __forceinline__ float bf16_to_f32(uint16_t h) {
   return __uint_as_float(static_cast<uint32_t>(h) << 16);
 }
