@@ -46,6 +46,7 @@ struct WorkspaceLayout {
   size_t cu32;         // int32 [N+1]   narrowed copy of INT64 cu_seqlens
   size_t chunk_base;   // int32 [N+1]   first slot of each sequence
   size_t seq_order;    // int32 [N]     longest-first order of sequences
+  size_t slot_span;    // int2 [slots]  chunk slot -> {first token, count | chunk index << 7}
   size_t wt, qg, ut, kd, aqk, gc;     // per-record tiles
   size_t qw, u;                       // per-record tiles of the stream variant
   size_t ready;        // int32 [recs]  per-record ready flags (fused variant)
@@ -74,8 +75,10 @@ inline WorkspaceLayout make_layout(int64_t N, int64_t T, int64_t H, bool fixed, 
   L.chunk_base = off;
   off = align_up(off + sizeof(int32_t) * (N + 1), 256);
   L.seq_order = off;
-  off = align_up(off + sizeof(int32_t) * N, 1024);
+  off = align_up(off + sizeof(int32_t) * N, 256);
   L.slots = (N > 0 && T > 0) ? chunk_slots(N, T, fixed, ckpt) : 0;
+  L.slot_span = off;
+  off = align_up(off + 2 * sizeof(int32_t) * static_cast<size_t>(L.slots), 1024);
   const size_t recs = split ? static_cast<size_t>(L.slots * H) : 0;
   if (stream) {   // [Q Gamma; W] and U replace W^T, Q Gamma and U^T (same bytes)
     L.qw = off;  off = align_up(off + recs * kTileQW, 1024);

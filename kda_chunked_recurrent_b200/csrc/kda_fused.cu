@@ -20,6 +20,7 @@ constexpr uint32_t kPrepBytes = 2 * prep::kGroupBytes + 1024;
 extern const int kThreadsPerCta = kThreads;
 extern const uint32_t kSmemAllocBytes = rec::kSmemAlloc > kPrepBytes ? rec::kSmemAlloc : kPrepBytes;
 static_assert(rec::kThreads <= kThreads, "recurrence warps fit the CTA");
+static_assert(kPrepBytes <= 227 * 1024 && rec::kSmemAlloc <= 227 * 1024, "shared memory budget");
 }
 
 // prep_groups: prepare groups per prepare CTA (1 or 2).  Few chains need little

@@ -19,11 +19,11 @@
 // #4633 calls decomp ("Description").
 //
 // Inputs of a chunk: q, k (bf16) and g (f32) arrive by TMA as whole [64 tok][128 ch]
-// tiles into shared memory the previous chunk no longer needs: g into R as soon
-// as that chunk's first UMMA and its Aqk store are done with R (the start of its
-// solve), q and k once its second UMMA has completed; all of them were
-// prefetched into L2 one chunk earlier.  v follows by TMA straight into its
-// UMMA operand layout and is converted from BF16 to FP16 in place during the solve.
+// tiles into shared memory the previous chunk no longer needs: g into R once that
+// chunk's Aqk store has read R (during its off-diagonal solve), q and k into L once its
+// solve is done with the scratch there; all of them were prefetched into L2 one chunk
+// earlier.  v follows by TMA straight into its UMMA operand layout and is converted
+// from BF16 to FP16 in place while the first UMMA runs.
 //
 // Thread mapping for the element-wise part: thread t owns the channel pair
 // (2p, 2p+1), p = t % 64, in sub-block b = t / 64 (tokens 16b .. 16b+15), so a
@@ -68,8 +68,8 @@ constexpr uint32_t kR = 65536;       // 40 KB  R^0..R^3, K-major B: 2 panels [16
 constexpr uint32_t kBytes = 65536 + 40960;
 // raw input tiles of a chunk, landed before its element-wise pass (which reads
 // them into registers before anything overwrites these regions)
-constexpr uint32_t kQraw = kV;                  // q [64 tok][128 ch] bf16
-constexpr uint32_t kKraw = kKG;                 // k [64 tok][128 ch] bf16
+constexpr uint32_t kQraw = kL;                  // q [64 tok][128 ch] bf16
+constexpr uint32_t kKraw = kL + 16384;          // k [64 tok][128 ch] bf16
 constexpr uint32_t kGraw = kR;                  // g [64 tok][128 ch] f32 (32 KB)
 constexpr uint32_t kRawQKTx = 16384 + 16384;
 constexpr uint32_t kRawGTx = 32768;
@@ -79,15 +79,16 @@ constexpr int kGThread = 224;
 // the thread that prefetches the next item's tiles into L2 (warp 1, idle while thread 0
 // issues the first UMMA)
 constexpr int kPrefetchThread = 32;
-// aliases of [K+; Q+] once the first UMMA has completed: the solve scratch, and
-// after the solve the staging tiles of the W^T / U^T TMA stores
+// aliases of [K+; Q+] once the first UMMA has completed: the solve scratch, then the
+// next chunk's raw q/k tiles; aliases of v / K Gamma once the second UMMA has
+// completed: the staging tiles of the W^T / U^T TMA stores
 constexpr int kLdh = 72;
 constexpr int kMfBlk = 272;                     // floats per diagonal block of Mf (16 x 16 + 16 pad)
 constexpr uint32_t kMf = kL;                    // f32 [4][16 s][16 r] diagonal blocks of M, column-major
 constexpr uint32_t kMh = kMf + 4 * kMfBlk * 4;  // f16 [64][72] off-diagonal blocks of M
 constexpr uint32_t kXh = kMh + 64 * kLdh * 2;   // f16 [64][72] T = (I + M)^-1
-constexpr uint32_t kWs = kL;                    // W^T staging [128 k][64 tok] f16, 128B swizzle
-constexpr uint32_t kUs = kL + 16384;            // U^T staging [128 v][64 tok] f16, 128B swizzle
+constexpr uint32_t kWs = kV;                    // W^T staging [128 k][64 tok] f16, 128B swizzle
+constexpr uint32_t kUs = kKG;                   // U^T staging [128 v][64 tok] f16, 128B swizzle
 // aliases of R once the first UMMA has completed
 constexpr uint32_t kAqs = kR;                   // Aqk staging [64 r][64 s] f16, 128B swizzle
 constexpr uint32_t kTb = 98304;                 // 8 KB T diag(beta) f16, K-major [64 r][64 s]
@@ -100,11 +101,14 @@ constexpr uint32_t kAuxTot = kAuxBeta + 256;     // float2 [4][64]
 constexpr uint32_t kAuxFirst = kAuxTot + 2048;   // float2 [4][64]
 constexpr uint32_t kAuxNorm = kAuxFirst + 2048;  // f32 [2][64] inverse norms of k, q rows (front end)
 constexpr uint32_t kAuxClaim = kAuxNorm + 512;   // i64 [2] claimed item indices (stream launch)
-constexpr uint32_t kGroupBytes = (kAuxClaim + 16 + 1023) / 1024 * 1024;   // one prepare group
+constexpr uint32_t kAuxSpan = kAuxClaim + 16;    // int4 [kSpanBatch] looked-up items {t0, c, h, rec}
+constexpr int kSpanBatch = 64;
+constexpr uint32_t kGroupBytes = (kAuxSpan + 16 * kSpanBatch + 1023) / 1024 * 1024;   // one prepare group
 constexpr uint32_t kSmemAlloc = kGroupBytes + 1024;
 static_assert(kXh + 64 * kLdh * 2 <= kR, "solve scratch overlaps the Aqk staging tile");
 static_assert(kAqs + 8192 <= kTb, "Aqk staging overlaps the Tb tile");
-static_assert(kUs + 16384 <= kR, "W/U staging overlaps R");
+static_assert(kUs + 16384 <= kL, "W/U staging overlaps L");
+static_assert(kKraw + 16384 <= kR, "raw q/k tiles overlap R");
 }  // namespace prep
 
 // Packed bf16x2 product (round to nearest even), for operands that are rounded
@@ -282,14 +286,23 @@ __device__ __forceinline__ void emit_rows(const uint32_t* val, bool is_q, int rl
       *reinterpret_cast<uint4*>(Mh + s0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
     }
   } else {
+    // columns before the row's sub-block are all kept, those after it are zero; only
+    // inside the diagonal block does the row index decide (s <= rl)
+    const int d = rl & 15;
 #pragma unroll
     for (int s0 = 0; s0 < kC; s0 += 8) {
       uint32_t pk[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int s = s0 + 2 * u;
-        const float a = (s < NV && s <= rl) ? __uint_as_float(val[s < NV ? s : 0]) : 0.f;
-        const float b2 = (s + 1 < NV && s + 1 <= rl) ? __uint_as_float(val[s + 1 < NV ? s + 1 : 0]) : 0.f;
+        float a = 0.f, b2 = 0.f;
+        if (s < 16 * BL) {
+          a = __uint_as_float(val[s]);
+          b2 = __uint_as_float(val[s + 1]);
+        } else if (s < NV) {
+          a = (s - 16 * BL <= d) ? __uint_as_float(val[s]) : 0.f;
+          b2 = (s + 1 - 16 * BL <= d) ? __uint_as_float(val[s + 1]) : 0.f;
+        }
         pk[u] = pack_f16(a, b2);
       }
       *reinterpret_cast<uint4*>(sm + kAqs + sw128_offset(rl, s0 >> 3)) =
@@ -318,30 +331,24 @@ __device__ __forceinline__ bool locate_item(const KdaParams& p, int64_t w, PrepI
     it.h = static_cast<int32_t>(w % p.H);
   }
   if (it.slot >= p.slots) return false;
-  int32_t n = 0, j = 0;
+  it.rec = it.slot * p.H + it.h;
   if (p.cu_seqlens == nullptr && p.ckpt_offsets == nullptr) {
     const uint32_t cps = static_cast<uint32_t>((p.fixed_len + kC - 1) / kC);
     const uint32_t s32 = static_cast<uint32_t>(it.slot);   // slot < slots < 2^31 here
-    n = static_cast<int32_t>(s32 / cps);
-    j = static_cast<int32_t>(s32 - static_cast<uint32_t>(n) * cps);
-  } else {
-    const int32_t* cb = reinterpret_cast<const int32_t*>(p.ws + p.lay.chunk_base);
-    if (it.slot >= cb[p.N]) return false;
-    int32_t lo = 0, hi = p.N;  // largest n with cb[n] <= slot
-    while (hi - lo > 1) {
-      const int32_t mid = (lo + hi) >> 1;
-      if (cb[mid] <= it.slot) lo = mid; else hi = mid;
-    }
-    n = lo;
-    j = static_cast<int32_t>(it.slot - cb[n]);
+    const int32_t n = static_cast<int32_t>(s32 / cps);
+    const int32_t j = static_cast<int32_t>(s32 - static_cast<uint32_t>(n) * cps);
+    if (n >= p.N) return false;
+    const SeqInfo si = seq_info(p, n, false);
+    if (j >= si.nch || j >= p.split_jmax) return false;
+    chunk_span(si, j, it.t0, it.c);
+    it.t0 += si.start;
+    return it.c > 0;
   }
-  if (n >= p.N) return false;
-  const SeqInfo si = seq_info(p, n, false);
-  if (j >= si.nch || j >= p.split_jmax) return false;
-  chunk_span(si, j, it.t0, it.c);
-  it.t0 += si.start;
-  it.rec = it.slot * p.H + it.h;
-  return it.c > 0;
+  // packed or checkpointed batches: the schedule kernel's slot span, one load
+  const int2 v = reinterpret_cast<const int2*>(p.ws + p.lay.slot_span)[it.slot];
+  it.t0 = v.x;
+  it.c = v.y & 127;
+  return it.c > 0 && (v.y >> 7) < p.split_jmax;
 }
 
 // Work item w in chunk-major order, used when prepare CTAs feed recurrence CTAs
@@ -501,14 +508,40 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
       if (locate(w, it)) return w;
     }
   };
+  // Static order: the items' chunk spans are looked up kSpanBatch items at a time, one
+  // item per thread, into shared memory (one global round trip per batch instead of one
+  // on every item's critical path); an item that holds no chunk reads as c = 0.
+  int4* s_span = reinterpret_cast<int4*>(sm + kAuxSpan);
+  auto load_batch = [&](int64_t i0) {   // items i0 .. i0 + kSpanBatch - 1 of this group
+    if (tid < kSpanBatch) {
+      const int64_t w = first + (i0 + tid) * stride;
+      PrepItem it;
+      int4 v = make_int4(0, 0, 0, 0);
+      if (w < nitems && locate(w, it)) v = make_int4(it.t0, it.c, it.h, static_cast<int32_t>(it.rec));
+      s_span[tid] = v;
+    }
+  };
+  auto batch_item = [&](int64_t i, PrepItem& it) -> bool {
+    const int4 v = s_span[i % kSpanBatch];
+    it.t0 = v.x;
+    it.c = v.y;
+    it.h = v.z;
+    it.rec = v.w;
+    return v.y > 0;
+  };
   PrepItem cur;
   int64_t w0 = first;
+  bool cur_valid;
   if (claim) {
     if (tid == 0) s_claim[0] = claim_next(cur);
     prep_sync<kFused>(gbar);
     w0 = s_claim[0];
+    cur_valid = w0 < nitems && locate(w0, cur);
+  } else {
+    load_batch(0);
+    prep_sync<kFused>(gbar);
+    cur_valid = batch_item(0, cur);
   }
-  bool cur_valid = w0 < nitems && locate(w0, cur);
   int64_t pending = -1;   // fused launch: record whose ready flag is still to be raised
   int iter = 0;
   for (int64_t w = w0, w_next = 0; w < nitems && ok; w = w_next, ++iter) {
@@ -521,8 +554,13 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
         nxt_valid = w_next < nitems;
       }
     } else {
+      // (the entries of the previous batch were all read before an earlier barrier)
       w_next = w + stride;
-      nxt_valid = (w_next < nitems) && locate(w_next, nxt);
+      if ((iter + 1) % kSpanBatch == 0 && w_next < nitems) {
+        load_batch(iter + 1);
+        prep_sync<kFused>(gbar);
+      }
+      nxt_valid = w_next < nitems && batch_item(iter + 1, nxt);
     }
     if (!cur_valid) {
       cur = nxt;
@@ -549,12 +587,16 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
     qk_for_cur = g_for_cur = false;
     uint16_t beta_raw = 0;   // consumed only after the operand pass, so its latency hides
     if (tid < c) beta_raw = p.beta[static_cast<int64_t>(t0 + tid) * p.H + h];
-    float fe_rate = 0.f;                          // front end: exp(A_log[h]), dt_bias pair
-    float2 fe_dtb = make_float2(0.f, 0.f);
+    // front end: the gate's exponent -log2(e) exp(A_log[h]) (a + dt_bias) as a * cz + cb,
+    // one FMA per lane of the channel pair
+    float2 fe_cz = make_float2(0.f, 0.f), fe_cb = make_float2(0.f, 0.f);
     if constexpr (kFE) {
       if (fe_gate) {
-        fe_rate = expf(__ldg(p.A_log + h));
-        fe_dtb = __ldg(reinterpret_cast<const float2*>(p.dt_bias + static_cast<int64_t>(h) * kD) + cp);
+        const float cz = -kLog2e * expf(__ldg(p.A_log + h));
+        const float2 dtb =
+            __ldg(reinterpret_cast<const float2*>(p.dt_bias + static_cast<int64_t>(h) * kD) + cp);
+        fe_cz = make_float2(cz, cz);
+        fe_cb = make_float2(cz * dtb.x, cz * dtb.y);
       }
     }
 
@@ -578,12 +620,12 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
         if (fe_gate) {
           // g = lower_bound * sigmoid(exp(A_log) (a + dt_bias)) from the raw BF16 gate a
           const uint32_t a2 = in ? reinterpret_cast<const uint32_t*>(sm + kGraw)[(blk * 16 + i) * 64 + cp] : 0u;
-          const float2 a = bf2_to_f2(a2);
-          const float x0 = fe_rate * (a.x + fe_dtb.x), x1 = fe_rate * (a.y + fe_dtb.y);
-          // (fast reciprocal: 1 + 2^y is at least 1, and a huge denominator gives 0, the
-          // limit of the logistic)
-          G[i] = in ? make_float2(__fdividef(p.lower_bound, 1.f + ex2(-x0 * kLog2e)),
-                                  __fdividef(p.lower_bound, 1.f + ex2(-x1 * kLog2e)))
+          const float2 z = fma2<kPack>(bf2_to_f2(a2), fe_cz, fe_cb);
+          // (approximate reciprocal: 1 + 2^z is at least 1, and an infinite denominator
+          // gives 0, the limit of the logistic)
+          const float2 den = add2<kPack>(make_float2(ex2(z.x), ex2(z.y)), make_float2(1.f, 1.f));
+          G[i] = in ? mul2<kPack>(make_float2(rcp_approx(den.x), rcp_approx(den.y)),
+                                  make_float2(p.lower_bound, p.lower_bound))
                     : make_float2(0.f, 0.f);
         } else {
           G[i] = in ? gs[i * 64] : make_float2(0.f, 0.f);
@@ -644,8 +686,8 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
       w_next = s_claim[(iter + 1) & 1];
       nxt_valid = w_next < nitems && locate(w_next, nxt);
     }
-    // ---- TMA: v tile straight into the MN-major A operand of U^T (the raw q tile
-    // in that region has been read by every thread)
+    // ---- TMA: v tile straight into the MN-major A operand of U^T (the previous item's
+    // W^T staging tile there has been read by its TMA store: waited for above)
     if (tid == 0) {
       mbar_arrive_expect_tx(&tma_bar, 16384);
       tma_load_3d(sm + kV, &maps.v_in, &tma_bar, 0, h, t0);
@@ -887,6 +929,7 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
         // dependent chain is one FMA per row (the later rows' updates are independent)
         const int bi = tid >> 4, jj = tid & 15;
         const float* Mc = reinterpret_cast<const float*>(sm + kMf) + bi * kMfBlk;   // [s][r]
+        const float4* Mc4 = reinterpret_cast<const float4*>(Mc);   // 16-byte aligned columns
         float x[16];
 #pragma unroll
         for (int rr = 0; rr < 16; ++rr) x[rr] = (rr == jj) ? 1.f : 0.f;
@@ -894,7 +937,13 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
         for (int ss = 0; ss < 15; ++ss) {
           const float xs = x[ss];
 #pragma unroll
-          for (int rr = ss + 1; rr < 16; ++rr) x[rr] = fmaf(-Mc[ss * 16 + rr], xs, x[rr]);
+          for (int q4 = (ss + 1) >> 2; q4 < 4; ++q4) {
+            const float4 m = Mc4[ss * 4 + q4];
+            const float mv[4] = {m.x, m.y, m.z, m.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              if (4 * q4 + e > ss) x[4 * q4 + e] = fmaf(-mv[e], xs, x[4 * q4 + e]);
+          }
         }
         const int col = bi * 16 + jj;
         const float bcol = s_beta[col];
@@ -930,6 +979,13 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
     fence_proxy_async_smem();
     tc_fence_before();
     ok = !prep_sync_or<kFused>(gbar, !ok);
+    // the solve is done with its scratch in L: the next item's q and k tiles go there
+    // now, a whole second UMMA and epilogue early
+    if (ok && nxt_valid) {
+      if (tid == 0) issue_qk(nxt);
+      ++raw_qk_issued;
+      qk_for_cur = true;
+    }
 
     // ---- UMMA 2: W^T = (K Gamma)^T (T diag beta)^T -> cols [0,64); U^T = V^T (T diag beta)^T -> [64,128)
     bool tma_seen = false;
@@ -967,13 +1023,6 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
       ok = mbar_wait(&mma_bar, static_cast<uint32_t>((mma_commits - 1) & 1), budget);
     }
     ok = !prep_sync_or<kFused>(gbar, !ok);
-    // the next item's q and k tiles go into v / K Gamma, free now that the second
-    // UMMA has completed
-    if (ok && nxt_valid) {
-      if (tid == 0) issue_qk(nxt);
-      ++raw_qk_issued;
-      qk_for_cur = true;
-    }
     if (ok && kStream) {
       tc_fence_after();
       // TMEM lanes 64..127 hold token row r = lane - 64 of [U | W]: warps 2, 3 write the

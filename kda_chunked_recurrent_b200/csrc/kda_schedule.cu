@@ -2,7 +2,8 @@
 //
 // From cu_seqlens (and the checkpoint offsets, which add one chunk boundary each)
 // it builds the chunk table chunk_base[n] = sum_{m<n} chunks_m (so every
-// (chunk, head) gets a workspace slot) and a
+// (chunk, head) gets a workspace slot), the span of every slot (first token, token
+// count, chunk index), so that a prepare CTA finds its chunk with one load, and a
 // longest-first order of the sequences for the recurrence grid, the tail-
 // utilisation ordering FlashInfer PR #4262 "Dispatch contract" exposes as
 // seq_order.  In validate mode it checks the metadata the host never reads
@@ -98,6 +99,29 @@ __global__ void __launch_bounds__(kSchedThreads) kda_schedule_kernel(const KdaPa
     __syncthreads();
   }
   if (tid == 0) cb[p.N] = carry;
+  __syncthreads();
+  // slot spans: the sequence holding slot s is the largest n with cb[n] <= s (empty
+  // sequences share their successor's base); slots past the last chunk get count 0
+  {
+    int2* span = reinterpret_cast<int2*>(p.ws + p.lay.slot_span);
+    const int32_t total = cb[p.N];
+    for (int64_t s = tid; s < p.slots; s += kSchedThreads) {
+      int2 v = make_int2(0, 0);
+      if (s < total) {
+        int32_t lo = 0, hi = p.N;
+        while (hi - lo > 1) {
+          const int32_t mid = (lo + hi) >> 1;
+          if (cb[mid] <= s) lo = mid; else hi = mid;
+        }
+        const SeqInfo si = seq_info(p, lo, false);
+        const int32_t j = static_cast<int32_t>(s) - cb[lo];
+        int32_t t0 = 0, c = 0;
+        if (j < si.nch) chunk_span(si, j, t0, c);
+        v = make_int2(si.start + t0, c | (j << 7));
+      }
+      span[s] = v;
+    }
+  }
   // longest-first order (stable on ties); identity beyond kLptMax sequences
   if (p.N <= kLptMax) {
     __syncthreads();
