@@ -20,10 +20,12 @@
 //
 // Inputs of a chunk: q, k (bf16) and g (f32) arrive by TMA as whole [64 tok][128 ch]
 // tiles into shared memory the previous chunk no longer needs: g into R once that
-// chunk's Aqk store has read R (during its off-diagonal solve), q and k into L once its
-// solve is done with the scratch there; all of them were prefetched into L2 one chunk
-// earlier.  v follows by TMA straight into its UMMA operand layout and is converted
-// from BF16 to FP16 in place while the first UMMA runs.
+// chunk's Aqk store has read R (during its off-diagonal solve), q and k into the v and
+// K Gamma tiles once its second UMMA has completed; all of them were prefetched into L2
+// one chunk earlier.  k and g go to registers before the element-wise pass; q is read
+// from its tile row by row during it (fewer live registers), so v follows by TMA into
+// its UMMA operand layout only after that pass, and is converted from BF16 to FP16 in
+// place during the off-diagonal solve.
 //
 // Thread mapping for the element-wise part: thread t owns the channel pair
 // (2p, 2p+1), p = t % 64, in sub-block b = t / 64 (tokens 16b .. 16b+15), so a
@@ -68,8 +70,9 @@ constexpr uint32_t kR = 65536;       // 40 KB  R^0..R^3, K-major B: 2 panels [16
 constexpr uint32_t kBytes = 65536 + 40960;
 // raw input tiles of a chunk, landed before its element-wise pass (which reads
 // them into registers before anything overwrites these regions)
-constexpr uint32_t kQraw = kL;                  // q [64 tok][128 ch] bf16
-constexpr uint32_t kKraw = kL + 16384;          // k [64 tok][128 ch] bf16
+constexpr uint32_t kQraw = kV;                  // q [64 tok][128 ch] bf16 (read row by row
+                                                //   by the element-wise pass)
+constexpr uint32_t kKraw = kKG;                 // k [64 tok][128 ch] bf16
 constexpr uint32_t kGraw = kR;                  // g [64 tok][128 ch] f32 (32 KB)
 constexpr uint32_t kRawQKTx = 16384 + 16384;
 constexpr uint32_t kRawGTx = 32768;
@@ -79,16 +82,15 @@ constexpr int kGThread = 224;
 // the thread that prefetches the next item's tiles into L2 (warp 1, idle while thread 0
 // issues the first UMMA)
 constexpr int kPrefetchThread = 32;
-// aliases of [K+; Q+] once the first UMMA has completed: the solve scratch, then the
-// next chunk's raw q/k tiles; aliases of v / K Gamma once the second UMMA has
-// completed: the staging tiles of the W^T / U^T TMA stores
+// aliases of [K+; Q+] once the first UMMA has completed: the solve scratch, and
+// after the solve the staging tiles of the W^T / U^T TMA stores
 constexpr int kLdh = 72;
 constexpr int kMfBlk = 272;                     // floats per diagonal block of Mf (16 x 16 + 16 pad)
 constexpr uint32_t kMf = kL;                    // f32 [4][16 s][16 r] diagonal blocks of M, column-major
 constexpr uint32_t kMh = kMf + 4 * kMfBlk * 4;  // f16 [64][72] off-diagonal blocks of M
 constexpr uint32_t kXh = kMh + 64 * kLdh * 2;   // f16 [64][72] T = (I + M)^-1
-constexpr uint32_t kWs = kV;                    // W^T staging [128 k][64 tok] f16, 128B swizzle
-constexpr uint32_t kUs = kKG;                   // U^T staging [128 v][64 tok] f16, 128B swizzle
+constexpr uint32_t kWs = kL;                    // W^T staging [128 k][64 tok] f16, 128B swizzle
+constexpr uint32_t kUs = kL + 16384;            // U^T staging [128 v][64 tok] f16, 128B swizzle
 // aliases of R once the first UMMA has completed
 constexpr uint32_t kAqs = kR;                   // Aqk staging [64 r][64 s] f16, 128B swizzle
 constexpr uint32_t kTb = 98304;                 // 8 KB T diag(beta) f16, K-major [64 r][64 s]
@@ -107,8 +109,7 @@ constexpr uint32_t kGroupBytes = (kAuxSpan + 16 * kSpanBatch + 1023) / 1024 * 10
 constexpr uint32_t kSmemAlloc = kGroupBytes + 1024;
 static_assert(kXh + 64 * kLdh * 2 <= kR, "solve scratch overlaps the Aqk staging tile");
 static_assert(kAqs + 8192 <= kTb, "Aqk staging overlaps the Tb tile");
-static_assert(kUs + 16384 <= kL, "W/U staging overlaps L");
-static_assert(kKraw + 16384 <= kR, "raw q/k tiles overlap R");
+static_assert(kUs + 16384 <= kR, "W/U staging overlaps R");
 }  // namespace prep
 
 // Packed bf16x2 product (round to nearest even), for operands that are rounded
@@ -609,11 +610,10 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
     }
     ok = !prep_sync_or<kFused>(gbar, !ok);
     float2 G[16];
-    uint32_t kw[16], qw[16];
+    uint32_t kw[16];
     {
       const float2* gs = reinterpret_cast<const float2*>(sm + kGraw) + blk * 16 * 64 + cp;
       const uint32_t* ks = reinterpret_cast<const uint32_t*>(sm + kKraw) + blk * 16 * 64 + cp;
-      const uint32_t* qs = reinterpret_cast<const uint32_t*>(sm + kQraw) + blk * 16 * 64 + cp;
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const bool in = ok && blk * 16 + i < c;   // rows past the chunk read as zero
@@ -631,7 +631,6 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
           G[i] = in ? gs[i * 64] : make_float2(0.f, 0.f);
         }
         kw[i] = in ? ks[i * 64] : 0u;
-        qw[i] = in ? qs[i * 64] : 0u;
       }
     }
     if constexpr (kFE) {
@@ -686,15 +685,6 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
       w_next = s_claim[(iter + 1) & 1];
       nxt_valid = w_next < nitems && locate(w_next, nxt);
     }
-    // ---- TMA: v tile straight into the MN-major A operand of U^T (the previous item's
-    // W^T staging tile there has been read by its TMA store: waited for above)
-    if (tid == 0) {
-      mbar_arrive_expect_tx(&tma_bar, 16384);
-      tma_load_3d(sm + kV, &maps.v_in, &tma_bar, 0, h, t0);
-      tma_load_3d(sm + kV + 8192, &maps.v_in, &tma_bar, 64, h, t0);
-    }
-    const uint32_t tma_parity = static_cast<uint32_t>(tma_issued & 1);
-    ++tma_issued;
     float2 Bs[4];   // B_i: G at the first token of sub-block i
     float2 E;       // G at the chunk end
     {
@@ -742,13 +732,16 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
                          blk * 16 * 64 + cp;
       uint32_t* kd_out = reinterpret_cast<uint32_t*>(p.ws + p.lay.kd + rec * kTileKd) + blk * 16 * 64 + cp;
       const float2 nB = make_float2(-B.x, -B.y);
+      // the raw q tile, row by row (rows past the chunk read as zero)
+      const uint32_t* qs = reinterpret_cast<const uint32_t*>(sm + kQraw) + blk * 16 * 64 + cp;
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const uint32_t xo = ((chunk ^ static_cast<uint32_t>(i & 7)) << 4) + static_cast<uint32_t>(i) * 128u;
+        const uint32_t qv = (blk * 16 + i < c) ? qs[i * 64] : 0u;
         const float2 d = add2<kPack>(G[i], nB);                 // G_r - B_b
         const float2 e = make_float2(ex2(d.x), ex2(d.y));       // e_r
         float2 inv = make_float2(ex2(-d.x), ex2(-d.y));         // 1 / e_r
-        const float2 kf = bf2_to_f2(kw[i]), qf = bf2_to_f2(qw[i]);
+        const float2 kf = bf2_to_f2(kw[i]), qf = bf2_to_f2(qv);
         const float2 gam = mul2<kPack>(e, cB);                  // Gamma_r, FP32
         if (kFE && fe_norm) {
           // front end: the row's inverse norms ride on the FP32 factors (one rounding each)
@@ -756,7 +749,7 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
           const float2 rk2 = make_float2(rk, rk), rq2 = make_float2(rq, rq);
           const uint32_t e2k = pack_bf16(mul2<kPack>(e, rk2)), e2q = pack_bf16(mul2<kPack>(e, rq2));
           sts32(bL + xo, hmul2_bf16(kw[i], e2k));
-          sts32(bL + xo + 64u * 128u, hmul2_bf16(qw[i], e2q));
+          sts32(bL + xo + 64u * 128u, hmul2_bf16(qv, e2q));
           const uint32_t rd2 = hmul2_bf16(kw[i], pack_bf16(mul2<kPack>(inv, rk2)));
           sts32(bRo + xo, rd2);
           if (blk < 1) sts32(bR + xo + 16u * 128u, hmul2_bf16(rd2, c1b));
@@ -769,7 +762,7 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
           // bf16 operands: factors rounded to bf16, products in packed bf16 math
           const uint32_t e2 = pack_bf16(e), inv2 = pack_bf16(inv);
           sts32(bL + xo, hmul2_bf16(kw[i], e2));
-          sts32(bL + xo + 64u * 128u, hmul2_bf16(qw[i], e2));
+          sts32(bL + xo + 64u * 128u, hmul2_bf16(qv, e2));
           const uint32_t rd2 = hmul2_bf16(kw[i], inv2);
           sts32(bRo + xo, rd2);
           if (blk < 1) sts32(bR + xo + 16u * 128u, hmul2_bf16(rd2, c1b));
@@ -798,6 +791,15 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
     fence_proxy_async_smem();
     tc_fence_before();
     prep_sync<kFused>(gbar);
+    // every thread has read the raw q tile: the v tile goes there now, by TMA straight
+    // into the MN-major A operand of U^T
+    if (tid == 0) {
+      mbar_arrive_expect_tx(&tma_bar, 16384);
+      tma_load_3d(sm + kV, &maps.v_in, &tma_bar, 0, h, t0);
+      tma_load_3d(sm + kV + 8192, &maps.v_in, &tma_bar, 64, h, t0);
+    }
+    const uint32_t tma_parity = static_cast<uint32_t>(tma_issued & 1);
+    ++tma_issued;
     if (tid == 0) {
       tc_fence_after();
       const uint32_t idesc = idesc_f16(128, 160, kFmtBF16, kKMajor, kKMajor);
@@ -816,13 +818,9 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
       }
     }
     if constexpr (kFused) pending = -1;
-    // While the first UMMA runs (it does not read the v tile), warps 1-7 turn the v tile,
-    // landed by TMA during the element-wise pass, from BF16 into FP16 in place: the U UMMA
-    // multiplies it by the FP16 T diag(beta), and both operands of one UMMA share a type
-    // (BF16 -> FP16 is exact for |v| in the FP16 normal range).  One of them first
-    // prefetches the next item's tiles (q, k, g, v) and beta rows into L2.
-    if (tid >= 32) {
-      if (tid == kPrefetchThread && nxt_valid) {
+    // While the first UMMA runs, one otherwise idle thread prefetches the next item's
+    // tiles (q, k, g, v) and beta rows into L2.
+    if (tid == kPrefetchThread && nxt_valid) {
         tma_prefetch_3d(&maps.q_in, 0, nxt.h, nxt.t0);
         tma_prefetch_3d(&maps.k_in, 0, nxt.h, nxt.t0);
         tma_prefetch_3d(&maps.g_in, 0, nxt.h, nxt.t0);
@@ -838,19 +836,6 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
         hi = hi < lim ? hi : lim;
         if (hi > lo) bulk_prefetch_l2(reinterpret_cast<const void*>(lo), static_cast<uint32_t>(hi - lo));
       }
-      if (mbar_wait(&tma_bar, tma_parity, budget)) {
-        uint4* vt = reinterpret_cast<uint4*>(sm + kV);
-        for (int i = tid - 32; i < 16384 / 16; i += kThreads - 32) {
-          const uint4 x = vt[i];
-          const float2 a = bf2_to_f2(x.x), b = bf2_to_f2(x.y), c2 = bf2_to_f2(x.z),
-                       d = bf2_to_f2(x.w);
-          vt[i] = make_uint4(pack_f16(a.x, a.y), pack_f16(b.x, b.y), pack_f16(c2.x, c2.y),
-                             pack_f16(d.x, d.y));
-        }
-      } else {
-        ok = false;
-      }
-    }
     ++mma_commits;
     if (tid == 0) ok = mbar_wait(&mma_bar, static_cast<uint32_t>((mma_commits - 1) & 1), budget);
     ok = !prep_sync_or<kFused>(gbar, !ok);
@@ -971,21 +956,32 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
         if (warp == 0) offdiag_column<0>(aMh, aXh, aTb, s_beta, lane);
         else if (warp == 1) offdiag_column<1>(aMh, aXh, aTb, s_beta, lane);
         else offdiag_column<2>(aMh, aXh, aTb, s_beta, lane);
-      } else if (tid == kGThread && g_next) {
-        bulk_wait_read();
-        issue_g(nxt);
+      } else if (warp == 7) {
+        if (tid == kGThread && g_next) {
+          bulk_wait_read();
+          issue_g(nxt);
+        }
+      } else {
+        // ---- warps 3-6: the v tile (BF16, landed by TMA in its operand layout) becomes FP16 in
+        // place: the U UMMA multiplies it by the FP16 T diag(beta), and both operands of
+        // one UMMA share a type (BF16 -> FP16 is exact for |v| in the FP16 normal range)
+        if (mbar_wait(&tma_bar, tma_parity, budget)) {
+          uint4* vt = reinterpret_cast<uint4*>(sm + kV);
+          for (int i = tid - 96; i < 16384 / 16; i += 128) {
+            const uint4 x = vt[i];
+            const float2 a = bf2_to_f2(x.x), b = bf2_to_f2(x.y), c2 = bf2_to_f2(x.z),
+                         d = bf2_to_f2(x.w);
+            vt[i] = make_uint4(pack_f16(a.x, a.y), pack_f16(b.x, b.y), pack_f16(c2.x, c2.y),
+                               pack_f16(d.x, d.y));
+          }
+        } else {
+          ok = false;
+        }
       }
     }
     fence_proxy_async_smem();
     tc_fence_before();
     ok = !prep_sync_or<kFused>(gbar, !ok);
-    // the solve is done with its scratch in L: the next item's q and k tiles go there
-    // now, a whole second UMMA and epilogue early
-    if (ok && nxt_valid) {
-      if (tid == 0) issue_qk(nxt);
-      ++raw_qk_issued;
-      qk_for_cur = true;
-    }
 
     // ---- UMMA 2: W^T = (K Gamma)^T (T diag beta)^T -> cols [0,64); U^T = V^T (T diag beta)^T -> [64,128)
     bool tma_seen = false;
@@ -1023,6 +1019,13 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
       ok = mbar_wait(&mma_bar, static_cast<uint32_t>((mma_commits - 1) & 1), budget);
     }
     ok = !prep_sync_or<kFused>(gbar, !ok);
+    // the next item's q and k tiles go into v / K Gamma, free now that the second
+    // UMMA has completed
+    if (ok && nxt_valid) {
+      if (tid == 0) issue_qk(nxt);
+      ++raw_qk_issued;
+      qk_for_cur = true;
+    }
     if (ok && kStream) {
       tc_fence_after();
       // TMEM lanes 64..127 hold token row r = lane - 64 of [U | W]: warps 2, 3 write the
