@@ -255,13 +255,16 @@ int choose_variant(const kda_shape_t* s, const kda_options_t* o) {
 //   tail R kFusedPrepCycles / (2 (SMs - R))  <=  jmax kFusedStepCycles,
 // so tail = slack jmax (2 (SMs - R) / R) (kFusedStepCycles / kFusedPrepCycles).  Only the
 // ratio of the two cycle counts enters, and it does not depend on the clock.  Measured on
-// a B200 (CUDA events, 1965 MHz): a chunk step of the fused launch 1.94 us at B8 T8192 H12
-// (3.8K cycles), a record of a fused prepare group 13.5 us (26.5K cycles) with a 47-chunk
-// tail at B6 T8192 H12; the front-end prepare is slower by the measured ratio of the
-// prepare launches at B8 T8192 H12 (0.585 / 0.369 ms).  The slack keeps the producer ahead.
-constexpr double kFusedStepCycles = 3800.0;
-constexpr double kFusedPrepCycles = 26500.0;
-constexpr double kFusedPrepCyclesFE = 26500.0 * 0.585 / 0.369;
+// a B200 (CUDA events, 1965 MHz): a chunk step of the fused launch 1.87 us at B8 T8192 H12
+// (3.7K cycles) while its records are ready in time.  A prepare group inside the fused
+// launch makes a record in 10-11 us when the launch is prepare-bound (B6 and B4 T8192 H12
+// fused: 20-22K cycles), but beside 96 busy recurrence SMs the tail keeps the chain at its
+// own pace only up to 17 of 128 rows (21 rows: 2.01 us per step), so the rule uses 26K
+// cycles.  The front-end prepare is slower by the measured ratio of the prepare launches
+// at B8 T8192 H12 (0.506 / 0.355 ms).  The slack keeps the producer ahead.
+constexpr double kFusedStepCycles = 3700.0;
+constexpr double kFusedPrepCycles = 26000.0;
+constexpr double kFusedPrepCyclesFE = 26000.0 * 0.506 / 0.355;
 constexpr double kHybridTailSlack = 0.9;
 int64_t hybrid_tail_chunks(int64_t jmax, int64_t chains, bool frontend = false) {
   const double free_groups = 2.0 * (static_cast<double>(sm_count()) - static_cast<double>(chains));
