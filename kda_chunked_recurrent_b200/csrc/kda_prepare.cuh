@@ -555,9 +555,12 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
         nxt_valid = w_next < nitems;
       }
     } else {
-      // (the entries of the previous batch were all read before an earlier barrier)
+      // refill: the first barrier ends the reads of the previous batch (the item just
+      // before may have been skipped, with no barrier since its entry was read), the
+      // second publishes the new entries
       w_next = w + stride;
       if ((iter + 1) % kSpanBatch == 0 && w_next < nitems) {
+        prep_sync<kFused>(gbar);
         load_batch(iter + 1);
         prep_sync<kFused>(gbar);
       }
