@@ -513,16 +513,16 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
   // item per thread, into shared memory (one global round trip per batch instead of one
   // on every item's critical path); an item that holds no chunk reads as c = 0.
   int4* s_span = reinterpret_cast<int4*>(sm + kAuxSpan);
-  auto load_batch = [&](int64_t i0) {   // items i0 .. i0 + kSpanBatch - 1 of this group
+  auto load_batch = [&](int32_t i0) {   // items i0 .. i0 + kSpanBatch - 1 of this group
     if (tid < kSpanBatch) {
-      const int64_t w = first + (i0 + tid) * stride;
+      const int64_t w = first + static_cast<int64_t>(i0 + tid) * stride;
       PrepItem it;
       int4 v = make_int4(0, 0, 0, 0);
       if (w < nitems && locate(w, it)) v = make_int4(it.t0, it.c, it.h, static_cast<int32_t>(it.rec));
       s_span[tid] = v;
     }
   };
-  auto batch_item = [&](int64_t i, PrepItem& it) -> bool {
+  auto batch_item = [&](int32_t i, PrepItem& it) -> bool {
     const int4 v = s_span[i % kSpanBatch];
     it.t0 = v.x;
     it.c = v.y;
@@ -530,8 +530,29 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
     it.rec = v.w;
     return v.y > 0;
   };
+  // The next valid item from index i of this group's sequence on (-1: none), refilling
+  // the batch where it crosses one; every thread of the group takes the same steps, so
+  // the refill's barriers match.  The first barrier of a refill ends the reads of the old
+  // batch, the second publishes the new entries.
+  // (item indices fit 32 bits: there are fewer than 2^31 records)
+  const int32_t first32 = static_cast<int32_t>(first), stride32 = static_cast<int32_t>(stride),
+                nitems32 = static_cast<int32_t>(nitems);
+  int32_t loaded = 0;   // index of the first item of the batch in shared memory
+  auto next_valid = [&](int32_t i, PrepItem& it) -> int32_t {
+    for (;; ++i) {
+      if (first32 + i * stride32 >= nitems32) return -1;
+      if (i - loaded >= kSpanBatch) {
+        prep_sync<kFused>(gbar);
+        loaded = i - i % kSpanBatch;
+        load_batch(loaded);
+        prep_sync<kFused>(gbar);
+      }
+      if (batch_item(i, it)) return i;
+    }
+  };
   PrepItem cur;
   int64_t w0 = first;
+  int32_t i_cur = -1;   // static order: index of the current item in the group's sequence
   bool cur_valid;
   if (claim) {
     if (tid == 0) s_claim[0] = claim_next(cur);
@@ -541,7 +562,9 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
   } else {
     load_batch(0);
     prep_sync<kFused>(gbar);
-    cur_valid = batch_item(0, cur);
+    i_cur = next_valid(0, cur);
+    cur_valid = i_cur >= 0;
+    w0 = cur_valid ? first32 + i_cur * stride32 : nitems;
   }
   int64_t pending = -1;   // fused launch: record whose ready flag is still to be raised
   int iter = 0;
@@ -555,16 +578,12 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
         nxt_valid = w_next < nitems;
       }
     } else {
-      // refill: the first barrier ends the reads of the previous batch (the item just
-      // before may have been skipped, with no barrier since its entry was read), the
-      // second publishes the new entries
-      w_next = w + stride;
-      if ((iter + 1) % kSpanBatch == 0 && w_next < nitems) {
-        prep_sync<kFused>(gbar);
-        load_batch(iter + 1);
-        prep_sync<kFused>(gbar);
-      }
-      nxt_valid = w_next < nitems && batch_item(iter + 1, nxt);
+      // items that hold no chunk (past the chunk table, or the hybrid's tail rows) are
+      // skipped here, so the next item's tiles are always requested one item ahead
+      const int32_t i_nxt = next_valid(i_cur + 1, nxt);
+      nxt_valid = i_nxt >= 0;
+      w_next = nxt_valid ? first32 + i_nxt * stride32 : nitems;
+      i_cur = i_nxt;
     }
     if (!cur_valid) {
       cur = nxt;
