@@ -480,10 +480,14 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
   const uint32_t tbase = tmem_slot;
   const uint32_t sbase = smem_u32(sm);
   bool ok = true;
-  int mma_commits = 0;     // UMMA commits issued so far (their mbarrier phases)
-  int tma_issued = 0;      // v tiles issued so far (tma_bar phases)
-  int raw_qk_issued = 0;   // raw q/k tile pairs issued so far (raw_qk_bar phases)
-  int raw_g_issued = 0;    // raw g tiles issued so far (raw_g_bar phases)
+  // Phase bookkeeping of the four mbarriers in one word (fewer registers live across the
+  // item loop): for each, bit `kPh*` is the parity of the phases completed so far, i.e.
+  // of the number of copies or commits issued, and bit `kPh* << 4` records that at
+  // least one was issued.  A wait for the last one uses the complement of its parity bit.
+  uint32_t ph = 0;
+  constexpr uint32_t kPhTma = 1, kPhMma = 2, kPhQk = 4, kPhG = 8;
+  auto bump = [&](uint32_t b) { ph = (ph ^ b) | (b << 4); };
+  auto last_parity = [&](uint32_t b) -> uint32_t { return (ph & b) ? 0u : 1u; };
   bool qk_for_cur = false, g_for_cur = false;  // the current item's tiles are in flight
   auto issue_qk = [&](const PrepItem& it) {  // thread 0 only
     mbar_arrive_expect_tx(&raw_qk_bar, kRawQKTx);
@@ -598,14 +602,14 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
     const int blk = tid >> 6;        // sub-block 0..3
     if (!qk_for_cur) {
       if (tid == 0) issue_qk(cur);
-      ++raw_qk_issued;
+      bump(kPhQk);
     }
     if (!g_for_cur) {
       if (tid == kGThread) {
         bulk_wait_read();
         issue_g(cur);
       }
-      ++raw_g_issued;
+      bump(kPhG);
     }
     qk_for_cur = g_for_cur = false;
     uint16_t beta_raw = 0;   // consumed only after the operand pass, so its latency hides
@@ -627,8 +631,8 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
     // One thread waits for the copies; the others sleep in the barrier instead of polling
     // (their polls would take issue slots from the other group on the SM).
     if (tid == 0) {
-      ok = mbar_wait(&raw_g_bar, static_cast<uint32_t>((raw_g_issued - 1) & 1), budget);
-      ok = ok && mbar_wait(&raw_qk_bar, static_cast<uint32_t>((raw_qk_issued - 1) & 1), budget);
+      ok = mbar_wait(&raw_g_bar, last_parity(kPhG), budget);
+      ok = ok && mbar_wait(&raw_qk_bar, last_parity(kPhQk), budget);
     }
     ok = !prep_sync_or<kFused>(gbar, !ok);
     float2 G[16];
@@ -820,8 +824,8 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
       tma_load_3d(sm + kV, &maps.v_in, &tma_bar, 0, h, t0);
       tma_load_3d(sm + kV + 8192, &maps.v_in, &tma_bar, 64, h, t0);
     }
-    const uint32_t tma_parity = static_cast<uint32_t>(tma_issued & 1);
-    ++tma_issued;
+    bump(kPhTma);
+    const uint32_t tma_parity = last_parity(kPhTma);
     if (tid == 0) {
       tc_fence_after();
       const uint32_t idesc = idesc_f16(128, 160, kFmtBF16, kKMajor, kKMajor);
@@ -858,8 +862,8 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
         hi = hi < lim ? hi : lim;
         if (hi > lo) bulk_prefetch_l2(reinterpret_cast<const void*>(lo), static_cast<uint32_t>(hi - lo));
       }
-    ++mma_commits;
-    if (tid == 0) ok = mbar_wait(&mma_bar, static_cast<uint32_t>((mma_commits - 1) & 1), budget);
+    bump(kPhMma);
+    if (tid == 0) ok = mbar_wait(&mma_bar, last_parity(kPhMma), budget);
     ok = !prep_sync_or<kFused>(gbar, !ok);
     if (ok) {
       tc_fence_after();
@@ -923,7 +927,7 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
     // phase), a whole UMMA 2 early
     const bool g_next = ok && nxt_valid;
     if (g_next) {
-      ++raw_g_issued;
+      bump(kPhG);
       g_for_cur = true;   // (for the next iteration)
     }
 
@@ -1037,15 +1041,15 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
     }
     if (tid == 0 && !tma_seen) ok = false;
     if (tid == 0 && ok) {
-      ++mma_commits;
-      ok = mbar_wait(&mma_bar, static_cast<uint32_t>((mma_commits - 1) & 1), budget);
+      bump(kPhMma);
+      ok = mbar_wait(&mma_bar, last_parity(kPhMma), budget);
     }
     ok = !prep_sync_or<kFused>(gbar, !ok);
     // the next item's q and k tiles go into v / K Gamma, free now that the second
     // UMMA has completed
     if (ok && nxt_valid) {
       if (tid == 0) issue_qk(nxt);
-      ++raw_qk_issued;
+      bump(kPhQk);
       qk_for_cur = true;
     }
     if (ok && kStream) {
@@ -1126,12 +1130,9 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
     if (!ok) {
       record_status(p.ws, kStatusTimeout);
       // copies and commits complete in issue order: waiting for the last drains all
-      if (tma_issued > 0)
-        mbar_wait(&tma_bar, static_cast<uint32_t>((tma_issued - 1) & 1), drain_budget);
-      if (mma_commits > 0)
-        mbar_wait(&mma_bar, static_cast<uint32_t>((mma_commits - 1) & 1), drain_budget);
-      if (raw_qk_issued > 0)
-        mbar_wait(&raw_qk_bar, static_cast<uint32_t>((raw_qk_issued - 1) & 1), drain_budget);
+      if (ph & (kPhTma << 4)) mbar_wait(&tma_bar, last_parity(kPhTma), drain_budget);
+      if (ph & (kPhMma << 4)) mbar_wait(&mma_bar, last_parity(kPhMma), drain_budget);
+      if (ph & (kPhQk << 4)) mbar_wait(&raw_qk_bar, last_parity(kPhQk), drain_budget);
     }
     bulk_wait_all();   // the tile stores this thread issued are complete
     if constexpr (kFused) {
@@ -1139,8 +1140,7 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
     }
   }
   if (tid == kGThread) {
-    if (!ok && raw_g_issued > 0)
-      mbar_wait(&raw_g_bar, static_cast<uint32_t>((raw_g_issued - 1) & 1), drain_budget);
+    if (!ok && (ph & (kPhG << 4))) mbar_wait(&raw_g_bar, last_parity(kPhG), drain_budget);
     bulk_wait_all();
   }
   tc_fence_before();
