@@ -42,7 +42,7 @@ def test_int64_validate_rejects_out_of_range_offsets():
     assert torch.all(out == 5.0)
 
 
-@pytest.mark.parametrize("variant", [1, 2])
+@pytest.mark.parametrize("variant", [1, 2, 3, 5])   # split, fused, hybrid, stream
 def test_cuda_graph_capture_replays_bitwise(variant):
     """A warmed call captured into a CUDA graph replays with new inputs in the same
     buffers and gives exactly the eager results (no host reads, no allocation)."""
