@@ -113,7 +113,9 @@ typedef enum {
                             groups, so prepare work runs on every SM beside the
                             recurrences; records reach the recurrence through L2 and are
                             dropped from it once read.  Needs N*H <= SM count, else
-                            KDA_ERR_BAD_OPTION.                                            */
+                            KDA_ERR_BAD_OPTION.  Opt-in only: AUTO does not pick it (it
+                            moves the fewest DRAM bytes but was slower than the others
+                            on every measured shape).                                     */
 } kda_variant_t;
 
 enum {

@@ -48,9 +48,15 @@
 // UT solve: T = (I + M)^-1 with M = diag(beta) A_strict, in 16x16 blocks.  The
 // diagonal blocks X_ii are inverted in FP32 by right-looking forward substitution;
 // then each of three warps walks one block column down, X_ij = -X_ii (sum_{k=j}^{i-1}
-// M_ik X_kj), as FP16 mma.sync products with FP32 accumulation.  Each block of
+// M_ik X_kj), as FP16 mma.sync products with FP32 accumulation, kept in registers (in
+// transposed form every accumulator is the next product's A fragment).  Each block of
 // T diag(beta), the operand of the W/U UMMA, is written from the accumulator as soon
 // as it is final.
+//
+// Item order: each 256-thread group walks its items (first, first + stride, ...) with
+// their chunk spans looked up 64 at a time into shared memory, skipping items that hold
+// no chunk, so that the next item's tiles are always requested one item ahead; the
+// stream launch's groups claim items from a counter instead.
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
