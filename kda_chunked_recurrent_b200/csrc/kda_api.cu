@@ -613,7 +613,7 @@ kda_status_t kda_prefill(const void* q, const void* k, const void* v, const floa
     cudaError_t e7 = cudaFuncSetAttribute(kda_stream_fe_kernel,
                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           stream::kSmemAllocBytes);
-    // the stream CTA's two halves (about 217 KB) need the largest shared-memory carveout
+    // the stream CTA's two halves (about 223 KB) need the largest shared-memory carveout
     cudaError_t e8 = cudaFuncSetAttribute(kda_stream_kernel,
                                           cudaFuncAttributePreferredSharedMemoryCarveout,
                                           cudaSharedmemCarveoutMaxShared);

@@ -1,5 +1,5 @@
 // kda_stream.cu — the stream variant: one cooperative launch of one 512-thread CTA per
-// SM that holds the whole SM's tensor memory (512 columns) and about 217 KB of shared
+// SM that holds the whole SM's tensor memory (512 columns) and about 223 KB of shared
 // memory, split in two halves.  On CTA b < R (R = N H chains) the first half (threads
 // 0..255, 256 columns, 104 KB) carries the recurrence of one (sequence, head) (body in
 // kda_chain.cuh) and the second half runs a prepare group; on the other CTAs both halves
