@@ -242,6 +242,7 @@ __device__ __forceinline__ void chain_body(const KdaParams& p, const SplitMaps& 
 #pragma unroll
     for (int part = 0; part < 2; ++part) {
       uint32_t r[32];
+      // all loads first (a checkpoint store between them would serialise them)
 #pragma unroll
       for (int i4 = 0; i4 < 8; ++i4) {
         float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -250,7 +251,13 @@ __device__ __forceinline__ void chain_body(const KdaParams& p, const SplitMaps& 
         r[4 * i4 + 1] = __float_as_uint(x.y);
         r[4 * i4 + 2] = __float_as_uint(x.z);
         r[4 * i4 + 3] = __float_as_uint(x.w);
-        if (ckr && si.ck == 0) *reinterpret_cast<float4*>(ckr + part * 32 + i4 * 4) = x;
+      }
+      if (ckr && si.ck == 0) {
+#pragma unroll
+        for (int i4 = 0; i4 < 8; ++i4)
+          *reinterpret_cast<float4*>(ckr + part * 32 + i4 * 4) =
+              make_float4(__uint_as_float(r[4 * i4]), __uint_as_float(r[4 * i4 + 1]),
+                          __uint_as_float(r[4 * i4 + 2]), __uint_as_float(r[4 * i4 + 3]));
       }
       tmem_st32(tmem_addr(tbase, lane_base, kColS + v0 + part * 32), r);
     }

@@ -361,11 +361,13 @@ __device__ __forceinline__ void recurrence_body(const KdaParams& p, const SplitM
       for (int kc = 0; kc < 2; ++kc) {
         uint32_t r[32];
         const int k0 = hw * 64 + kc * 32;
+        // all loads first: a checkpoint store between them (a buffer the compiler cannot
+        // prove apart from h0) would make every load wait for the previous one
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float x = h0c ? h0c[(k0 + i) * kD] : 0.f;
-          r[i] = __float_as_uint(x);
-          if (ckc && si.ck == 0) ckc[(k0 + i) * kD] = x;
+        for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(h0c ? h0c[(k0 + i) * kD] : 0.f);
+        if (ckc && si.ck == 0) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ckc[(k0 + i) * kD] = __uint_as_float(r[i]);
         }
         tmem_st32(tmem_addr(tbase, lane_base, kColS + k0), r);
       }
