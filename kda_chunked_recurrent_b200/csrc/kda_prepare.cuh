@@ -673,26 +673,34 @@ __device__ __forceinline__ void prepare_body(const KdaParams& p, const SplitMaps
         const uint4* kr = reinterpret_cast<const uint4*>(sm + kKraw);
         const uint4* qr = reinterpret_cast<const uint4*>(sm + kQraw);
         const int hl = lane & 15;
+        // (the partial sums of all four row pairs first, so that no store to s_norm
+        // sits between the loads and keeps the later ones waiting)
+        float sk[4], sq[4];
 #pragma unroll
         for (int rr = 0; rr < 4; ++rr) {
           const int row = warp * 8 + rr * 2 + (lane >> 4);
           const uint4 kv = kr[row * 16 + hl], qv = qr[row * 16 + hl];
-          float sk = 0.f, sq = 0.f;
+          sk[rr] = 0.f;
+          sq[rr] = 0.f;
           const uint32_t kx[4] = {kv.x, kv.y, kv.z, kv.w}, qx[4] = {qv.x, qv.y, qv.z, qv.w};
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const float2 a = bf2_to_f2(kx[j]), b = bf2_to_f2(qx[j]);
-            sk = fmaf(a.x, a.x, fmaf(a.y, a.y, sk));
-            sq = fmaf(b.x, b.x, fmaf(b.y, b.y, sq));
+            sk[rr] = fmaf(a.x, a.x, fmaf(a.y, a.y, sk[rr]));
+            sq[rr] = fmaf(b.x, b.x, fmaf(b.y, b.y, sq[rr]));
           }
+        }
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr) {
+          const int row = warp * 8 + rr * 2 + (lane >> 4);
 #pragma unroll
           for (int o = 8; o > 0; o >>= 1) {
-            sk += __shfl_xor_sync(0xffffffffu, sk, o);
-            sq += __shfl_xor_sync(0xffffffffu, sq, o);
+            sk[rr] += __shfl_xor_sync(0xffffffffu, sk[rr], o);
+            sq[rr] += __shfl_xor_sync(0xffffffffu, sq[rr], o);
           }
           if (hl == 0) {
-            s_norm[row] = rsqrtf(sk + p.l2_eps);
-            s_norm[64 + row] = rsqrtf(sq + p.l2_eps);
+            s_norm[row] = rsqrtf(sk[rr] + p.l2_eps);
+            s_norm[64 + row] = rsqrtf(sq[rr] + p.l2_eps);
           }
         }
       }
