@@ -258,13 +258,15 @@ int choose_variant(const kda_shape_t* s, const kda_options_t* o) {
 // a B200 (CUDA events, 1965 MHz): a chunk step of the fused launch 1.87 us at B8 T8192 H12
 // (3.7K cycles) while its records are ready in time.  A prepare group inside the fused
 // launch makes a record in 10-11 us when the launch is prepare-bound (B6 and B4 T8192 H12
-// fused: 20-22K cycles), but beside 96 busy recurrence SMs the tail keeps the chain at its
-// own pace only up to 17 of 128 rows (21 rows: 2.01 us per step), so the rule uses 26K
-// cycles.  The front-end prepare is slower by the measured ratio of the prepare launches
-// at B8 T8192 H12 (0.506 / 0.355 ms).  The slack keeps the producer ahead.
+// fused: 20-22K cycles).  Swept on the hybrid at B8 and B6 T8192 H12, 22K per record is
+// the best value of the rule (B8: tail 20 rows, 0.555 ms, against 0.556 at 24K, 0.558 at
+// 26K and 0.559 at 29K; B6: tail 40, 0.437 against 0.441, 0.445 and 0.452), so the rule
+// uses it.  The front-end
+// prepare is slower by the measured ratio of the prepare launches at B8 T8192 H12
+// (0.506 / 0.355 ms).  The slack keeps the producer ahead.
 constexpr double kFusedStepCycles = 3700.0;
-constexpr double kFusedPrepCycles = 26000.0;
-constexpr double kFusedPrepCyclesFE = 26000.0 * 0.506 / 0.355;
+constexpr double kFusedPrepCycles = 22000.0;
+constexpr double kFusedPrepCyclesFE = 22000.0 * 0.506 / 0.355;
 constexpr double kHybridTailSlack = 0.9;
 int64_t hybrid_tail_chunks(int64_t jmax, int64_t chains, bool frontend = false) {
   const double free_groups = 2.0 * (static_cast<double>(sm_count()) - static_cast<double>(chains));

@@ -200,10 +200,10 @@ def test_hybrid_tail_follows_the_throughput_rule():
     # two chunks per sequence: the tail is clamped to leave one row for the prepare launch
     assert _hybrid_tail(8, 128, 12) == (1, 2)
     # nearly every SM carries a chain: the fused prepare groups get the one-row minimum
-    assert _hybrid_tail(11, 8192, 12)[0] == 3 and _hybrid_tail(12, 8192, 12)[0] == 1
-    # the rule at the measured shapes: 96 chains on 148 SMs keep 17 of 128 rows in the
-    # fused launch, 72 chains 34
-    assert tails[8][0] == 17 and tails[6][0] == 34, tails
+    assert _hybrid_tail(11, 8192, 12)[0] == 4 and _hybrid_tail(12, 8192, 12)[0] == 1
+    # the rule at the measured shapes: 96 chains on 148 SMs keep 20 of 128 rows in the
+    # fused launch, 72 chains 40
+    assert tails[8][0] == 20 and tails[6][0] == 40, tails
 
 
 def test_fused_variant_needs_free_sms():
