@@ -17,7 +17,7 @@ whole chunks at the endpoints:
     the header states.
 
 Each case runs with an initial state and a checkpoint inside a chunk, element by
-element against the oracle at the benchmark spec's tolerances (2e-2 max-abs on o, 1e-3
+element against the oracle at the path's tolerances (2e-2 max-abs on o, 1e-3
 relative Frobenius on the final and checkpoint states).
 """
 import numpy as np
